@@ -1,0 +1,117 @@
+"""Seeded synthetic inputs shaped like the linear layers of FLUX.1-dev at 1024x1024.
+
+This module only draws random numbers and lists shapes; it holds none of the
+ternary method's arithmetic, so the CUDA path and the CPU oracle can both be
+fed from it without sharing any of the computation.
+
+Shapes follow page "1.58-bit FLUX" (arXiv 2412.18653), Section 3.1: every
+linear layer of the double-stream (FluxTransformerBlock) and single-stream
+(FluxSingleTransformerBlock) blocks is ternary.  One 1024x1024 image gives
+4096 image tokens; the text stream has 512 tokens, hidden size 3072, MLP
+width 12288.  Distributions: x ~ N(0, 1) (N(0, 0.5) into the MLP down
+projection), W ~ N(0, 0.02), bias ~ N(0, 0.01); every tensor is drawn in
+fp32 from a seeded CPU generator and rounded to bf16.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import torch
+
+HIDDEN = 3072
+MLP = 12288
+IMG_TOKENS = 4096
+TXT_TOKENS = 512
+N_DOUBLE = 19
+N_SINGLE = 38
+W_STD = 0.02
+B_STD = 0.01
+EPS = 1e-5
+
+
+@dataclasses.dataclass(frozen=True)
+class Layer:
+    name: str
+    M: int
+    K: int
+    N: int
+    seed: int
+    x_std: float = 1.0
+    w_std: float = W_STD
+    b_std: float = B_STD
+
+    @property
+    def flop(self) -> float:
+        return 2.0 * self.M * self.N * self.K
+
+    @property
+    def packed_bytes(self) -> int:
+        return self.N * self.K // 4
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """codes + fp32 scales + bf16 bias + bf16 x + bf16 y."""
+        return self.N * self.K // 4 + 4 * self.N + 2 * self.N + 2 * self.M * self.K + 2 * self.M * self.N
+
+
+# The single-layer workloads.  "mod_*" is the adaLN modulation GEMV sweep.
+CONFIGS = {
+    "tiny": Layer("tiny", M=16, K=256, N=256, seed=0),
+    "qkv": Layer("qkv", M=IMG_TOKENS, K=HIDDEN, N=3 * HIDDEN, seed=1),
+    "mlp_up": Layer("mlp_up", M=IMG_TOKENS + TXT_TOKENS, K=HIDDEN, N=MLP, seed=2),
+    "mlp_down": Layer("mlp_down", M=IMG_TOKENS + TXT_TOKENS, K=MLP, N=HIDDEN, seed=3, x_std=0.5),
+}
+for _m in (1, 4, 16, 64):
+    CONFIGS[f"mod6_m{_m}"] = Layer(f"mod6_m{_m}", M=_m, K=HIDDEN, N=6 * HIDDEN, seed=4)
+    CONFIGS[f"mod3_m{_m}"] = Layer(f"mod3_m{_m}", M=_m, K=HIDDEN, N=3 * HIDDEN, seed=4)
+
+
+def flux_stack() -> List[Layer]:
+    """Every ternary linear of one FLUX.1-dev transformer forward (one image)."""
+    layers: List[Layer] = []
+    idx = 0
+
+    def add(name, M, K, N, x_std=1.0):
+        nonlocal idx
+        layers.append(Layer(name, M=M, K=K, N=N, seed=1000 + idx, x_std=x_std))
+        idx += 1
+
+    for b in range(N_DOUBLE):
+        for stream, M in (("img", IMG_TOKENS), ("txt", TXT_TOKENS)):
+            add(f"double{b}.{stream}.mod", 1, HIDDEN, 6 * HIDDEN)
+            add(f"double{b}.{stream}.qkv", M, HIDDEN, 3 * HIDDEN)
+            add(f"double{b}.{stream}.proj", M, HIDDEN, HIDDEN)
+            add(f"double{b}.{stream}.mlp_up", M, HIDDEN, MLP)
+            add(f"double{b}.{stream}.mlp_down", M, MLP, HIDDEN, x_std=0.5)
+    for b in range(N_SINGLE):
+        M = IMG_TOKENS + TXT_TOKENS
+        add(f"single{b}.mod", 1, HIDDEN, 3 * HIDDEN)
+        add(f"single{b}.qkv_mlp", M, HIDDEN, 3 * HIDDEN + MLP)
+        add(f"single{b}.proj_out", M, HIDDEN + MLP, HIDDEN, x_std=0.5)
+    return layers
+
+
+def _normal(shape, std: float, gen: torch.Generator) -> torch.Tensor:
+    return (torch.randn(shape, generator=gen, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def make_inputs(layer: Layer, M: Optional[int] = None):
+    """Returns CPU bf16 tensors (x [M,K], W [N,K], b [N]) for a layer.
+
+    W and b depend only on the seed; x is drawn after them so a smaller M
+    gives the leading rows of the same stream only when the caller passes
+    the same M.
+    """
+    gen = torch.Generator().manual_seed(layer.seed)
+    W = _normal((layer.N, layer.K), layer.w_std, gen)
+    b = _normal((layer.N,), layer.b_std, gen)
+    x = _normal((layer.M if M is None else M, layer.K), layer.x_std, gen)
+    return x, W, b
+
+
+def bf16_bits(t: torch.Tensor):
+    """Raw uint16 bit patterns of a CPU bf16 tensor, as a numpy array."""
+    import numpy as np
+
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -1,0 +1,187 @@
+"""fp64 CPU oracle for the ternary linear layer of "1.58-bit FLUX".
+
+TEST INFRASTRUCTURE ONLY.  The test suite, the smoke check and the
+benchmark's CPU-baseline leg are the only users; the product library never
+imports, links or runs anything here.  The arithmetic lives in
+``tern_oracle.c`` (plain C, IEEE double), which shares no code with the CUDA
+library.  This module builds it with gcc on first use and marshals numpy
+arrays through ctypes.
+
+Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
+
+* ``quantize(W_bits, eps)`` -- absmean ternarisation per output channel
+  (Section 1: weights in {-1, 0, +1}, "akin to BitNet b1.58"):
+  ``s = mean|W| + eps``, ``T = RoundClip(W / s, -1, 1)``, ties to even.
+* ``ternarize(W_bits, s)`` -- the same RoundClip with given scales, used to
+  compare codes "given the scales" of another implementation.
+* ``near_threshold(W_bits, s, band)`` -- elements with ``| |w|/s - 0.5 | <
+  band``; the rounding decision there is not fixed by the scale's precision.
+* ``pack_canonical / unpack_canonical`` -- 2-bit signed codes, four per byte,
+  row-major (Section 1: "stored using 2-bit signed integers").
+* ``pack_tiled / unpack_tiled`` -- the tile-interleaved device layout.
+* ``linear(x_bits, T, s, b_bits)`` -- ``y = s * (x @ T^T) + b`` in double
+  (Section 4: activations are not quantised).
+
+bf16 tensors are passed as their raw uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tern_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_i64 = ctypes.c_int64
+_ptr = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile tern_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fno-fast-math", "-fPIC", "-shared",
+             _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_absmean_scales.argtypes = [_ptr, _i64, _i64, ctypes.c_double, _ptr]
+        lib.oracle_ternarize.argtypes = [_ptr, _i64, _i64, _ptr, _ptr]
+        lib.oracle_near_threshold.argtypes = [_ptr, _i64, _i64, _ptr, ctypes.c_double, _ptr]
+        lib.oracle_near_threshold.restype = _i64
+        lib.oracle_quantize.argtypes = [_ptr, _i64, _i64, ctypes.c_double, _ptr, _ptr]
+        lib.oracle_pack_canonical.argtypes = [_ptr, _i64, _i64, _ptr]
+        lib.oracle_unpack_canonical.argtypes = [_ptr, _i64, _i64, _ptr]
+        lib.oracle_unpack_canonical.restype = ctypes.c_int
+        lib.oracle_pack_tiled.argtypes = [_ptr, _i64, _i64, _ptr]
+        lib.oracle_pack_tiled.restype = ctypes.c_int
+        lib.oracle_unpack_tiled.argtypes = [_ptr, _i64, _i64, _ptr]
+        lib.oracle_unpack_tiled.restype = ctypes.c_int
+        lib.oracle_linear.argtypes = [_ptr, _i64, _i64, _ptr, _ptr, _ptr, _i64, _ptr]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loop uses (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float64 (for test-side use)."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def absmean_scales(W_bits: np.ndarray, eps: float) -> np.ndarray:
+    W_bits = _c(W_bits, np.uint16)
+    N, K = W_bits.shape
+    s = np.empty(N, np.float64)
+    _load().oracle_absmean_scales(_p(W_bits), N, K, float(eps), _p(s))
+    return s
+
+
+def ternarize(W_bits: np.ndarray, s: np.ndarray) -> np.ndarray:
+    W_bits = _c(W_bits, np.uint16)
+    s = _c(s, np.float64)
+    N, K = W_bits.shape
+    T = np.empty((N, K), np.int8)
+    _load().oracle_ternarize(_p(W_bits), N, K, _p(s), _p(T))
+    return T
+
+
+def near_threshold(W_bits: np.ndarray, s: np.ndarray, band: float = 1e-6):
+    """Returns (count, boolean mask [N,K])."""
+    W_bits = _c(W_bits, np.uint16)
+    s = _c(s, np.float64)
+    N, K = W_bits.shape
+    mask = np.empty((N, K), np.uint8)
+    cnt = _load().oracle_near_threshold(_p(W_bits), N, K, _p(s), float(band), _p(mask))
+    return int(cnt), mask.astype(bool)
+
+
+def quantize(W_bits: np.ndarray, eps: float):
+    """Returns (T int8 [N,K], s float64 [N])."""
+    W_bits = _c(W_bits, np.uint16)
+    N, K = W_bits.shape
+    T = np.empty((N, K), np.int8)
+    s = np.empty(N, np.float64)
+    _load().oracle_quantize(_p(W_bits), N, K, float(eps), _p(T), _p(s))
+    return T, s
+
+
+def pack_canonical(T: np.ndarray) -> np.ndarray:
+    T = _c(T, np.int8)
+    N, K = T.shape
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    P = np.empty(N * K // 4, np.uint8)
+    _load().oracle_pack_canonical(_p(T), N, K, _p(P))
+    return P
+
+
+def unpack_canonical(P: np.ndarray, N: int, K: int):
+    """Returns (T, number of invalid codes)."""
+    P = _c(P, np.uint8)
+    T = np.empty((N, K), np.int8)
+    bad = _load().oracle_unpack_canonical(_p(P), N, K, _p(T))
+    return T, int(bad)
+
+
+def pack_tiled(T: np.ndarray) -> np.ndarray:
+    T = _c(T, np.int8)
+    N, K = T.shape
+    P = np.empty(N * K // 4, np.uint8)
+    if _load().oracle_pack_tiled(_p(T), N, K, _p(P)) != 0:
+        raise ValueError("tiled layout needs N % 128 == 0 and K % 64 == 0")
+    return P
+
+
+def unpack_tiled(P: np.ndarray, N: int, K: int):
+    """Returns (T, number of invalid codes)."""
+    P = _c(P, np.uint8)
+    T = np.empty((N, K), np.int8)
+    bad = _load().oracle_unpack_tiled(_p(P), N, K, _p(T))
+    if bad < 0:
+        raise ValueError("tiled layout needs N % 128 == 0 and K % 64 == 0")
+    return T, int(bad)
+
+
+def linear(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None) -> np.ndarray:
+    """y[m,n] = s_n * sum_k x[m,k] T[n,k] + b_n in float64, shape [M,N]."""
+    x_bits = _c(x_bits, np.uint16)
+    T = _c(T, np.int8)
+    s = _c(s, np.float64)
+    M, K = x_bits.shape
+    N, K2 = T.shape
+    if K2 != K or s.shape != (N,):
+        raise ValueError("shape mismatch")
+    bp = None
+    if b_bits is not None:
+        b_bits = _c(b_bits, np.uint16)
+        if b_bits.shape != (N,):
+            raise ValueError("bias shape mismatch")
+        bp = _p(b_bits)
+    y = np.empty((M, N), np.float64)
+    _load().oracle_linear(_p(x_bits), M, K, _p(T), _p(s), bp, N, _p(y))
+    return y

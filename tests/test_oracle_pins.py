@@ -1,0 +1,301 @@
+"""Pins for the fp64 CPU oracle, each independent of the oracle's own code.
+
+CPU only.  The oracle is checked against: a hand-worked example, exact
+rational brute force, a library routine (numpy's dense float64 matmul of the
+dequantised weights), hand-computed layout positions, invariants of the
+method, and the storage figures printed on page "1.58-bit FLUX"
+(arXiv 2412.18653): 7.7x smaller storage with 99.5% of the 11.9B
+vision-transformer parameters quantised (Abstract; Section 1).
+"""
+from __future__ import annotations
+
+import itertools
+import os
+import random
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_post_quantised_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def to_bf16_bits(values) -> np.ndarray:
+    """Bit patterns of values that must be exactly representable in bf16."""
+    a = np.asarray(values, dtype=np.float32)
+    bits = (a.view(np.uint32) >> 16).astype(np.uint16)
+    back = (bits.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(back, a), "value not exact in bf16"
+    return bits
+
+
+def read_hand_example():
+    rows = {}
+    with open(os.path.join(GOLDEN, "hand_worked_4x4.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            rows.setdefault(key, []).append(vals)
+    return rows
+
+
+# ---------------------------------------------------------------- hand-worked
+def test_hand_worked_example():
+    g = read_hand_example()
+    eps = float(g["eps"][0][0])
+    W = to_bf16_bits([[float(v) for v in r] for r in g["W"]])
+    T_exp = np.array([[int(v) for v in r] for r in g["T"]], np.int8)
+    s_exp = np.array([float(v) for v in g["s"][0]])
+    gamma_exp = np.array([float(v) for v in g["gamma"][0]])
+
+    T, s = oracle.quantize(W, eps)
+    np.testing.assert_allclose(s, s_exp, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(s - eps, gamma_exp, rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(T, T_exp)
+
+    P = oracle.pack_canonical(T)
+    assert [int(b) for b in P] == [int(v, 16) for v in g["bytes"][0]]
+
+    x = to_bf16_bits([[float(v) for v in g["x"][0]]])
+    b = to_bf16_bits([float(v) for v in g["b"][0]])
+    y = oracle.linear(x, T, s, b)[0]
+    np.testing.assert_allclose(y, [float(v) for v in g["y"][0]], rtol=1e-12)
+    y_bf16 = torch.tensor(y, dtype=torch.float64).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(y_bf16, [float(v) for v in g["y_bf16"][0]])
+    acc = oracle.linear(x, T, np.ones(4), None)[0]
+    np.testing.assert_array_equal(acc, [float(v) for v in g["acc"][0]])
+
+
+# ------------------------------------------------------- exact brute force
+def exact_round_clip(w: Fraction, s: Fraction) -> int:
+    """Nearest of {-1, 0, +1} to w/s; an exact tie goes to the even value 0."""
+    if s == 0:
+        return 0
+    r = w / s
+    best = min((abs(r - t), t != 0, t) for t in (-1, 0, 1))
+    return best[2]
+
+
+def bf16_grid_value(rng: random.Random) -> float:
+    mant = rng.randint(-255, 255)
+    exp = rng.randint(-14, -4)
+    return float(mant) * 2.0 ** exp
+
+
+@pytest.mark.parametrize("eps", [0.0, 1e-5, 0.25])
+@pytest.mark.parametrize("seed", range(6))
+def test_quantize_matches_exact_rational_brute_force(eps, seed):
+    rng = random.Random(seed * 7 + int(eps * 1e6))
+    N, K = rng.randint(1, 8), rng.randint(1, 8)
+    vals = [[bf16_grid_value(rng) if rng.random() > 0.15 else 0.0 for _ in range(K)] for _ in range(N)]
+    W = to_bf16_bits(vals)
+    T, s = oracle.quantize(W, eps)
+    e = Fraction(eps)
+    for n in range(N):
+        row = [Fraction(v) for v in vals[n]]
+        s_exact = sum(abs(w) for w in row) / K + e
+        assert abs(Fraction(s[n]) - s_exact) <= s_exact * Fraction(1, 10**15)
+        for k in range(K):
+            r = abs(row[k] / s_exact) if s_exact else Fraction(0)
+            if r != Fraction(1, 2) and abs(r - Fraction(1, 2)) < Fraction(1, 10**12):
+                continue  # a double rounding of s could decide this one either way
+            assert T[n, k] == exact_round_clip(row[k], s_exact), (n, k, vals[n])
+
+
+def test_round_half_to_even_ties():
+    # eps = 0 makes the ratios exact: [1, 3] -> s = 2 -> r = [0.5, 1.5].
+    W = to_bf16_bits([[1, 3, 0, 0], [-1, -3, 0, 0], [1, 1, 1, 5], [3, 1, 0, 0]])
+    T, s = oracle.quantize(W, 0.0)
+    np.testing.assert_array_equal(s, [1.0, 1.0, 2.0, 1.0])
+    # row 0: s = 1 -> r = [1, 3, 0, 0] ; row 2: r = [0.5, 0.5, 0.5, 2.5]
+    np.testing.assert_array_equal(T, [[1, 1, 0, 0], [-1, -1, 0, 0], [0, 0, 0, 1], [1, 1, 0, 0]])
+    W2 = to_bf16_bits([[1, 3], [-1, -3], [3, 1]])
+    T2, s2 = oracle.quantize(W2, 0.0)
+    np.testing.assert_array_equal(s2, [2.0, 2.0, 2.0])
+    np.testing.assert_array_equal(T2, [[0, 1], [0, -1], [1, 0]])
+
+
+def test_linear_exact_over_every_code_row():
+    """All 3^4 ternary rows against exact rational arithmetic."""
+    rng = np.random.default_rng(5)
+    rows = np.array(list(itertools.product((-1, 0, 1), repeat=4)), np.int8)  # N = 81
+    N, K, M = rows.shape[0], 4, 3
+    x_vals = [[bf16_grid_value(random.Random(int(v))) for v in rng.integers(0, 1 << 30, K)] for _ in range(M)]
+    b_vals = [bf16_grid_value(random.Random(int(v))) for v in rng.integers(0, 1 << 30, N)]
+    x = to_bf16_bits(x_vals)
+    b = to_bf16_bits(b_vals)
+    s = rng.uniform(0.01, 0.05, N)
+    y = oracle.linear(x, rows, s, b)
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(s[n]) * sum(Fraction(x_vals[m][k]) * int(rows[n, k]) for k in range(K)) + Fraction(b_vals[n])
+            # a few double roundings, relative to the size of the terms summed
+            size = Fraction(s[n]) * sum(abs(Fraction(v)) for v in x_vals[m]) + abs(Fraction(b_vals[n]))
+            assert abs(Fraction(y[m, n]) - exact) <= size * Fraction(1, 10**15)
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 12, 7), (33, 200, 130), (1, 64, 3)])
+def test_linear_equals_dense_matmul_of_dequantised_weight(M, K, N):
+    """numpy's float64 matmul of T*s (scale before the sum) is the library check."""
+    rng = np.random.default_rng(M * 1000 + N)
+    x = workloads.bf16_bits(torch.randn(M, K, generator=torch.Generator().manual_seed(N)).to(torch.bfloat16))
+    b = workloads.bf16_bits((0.1 * torch.randn(N, generator=torch.Generator().manual_seed(M))).to(torch.bfloat16))
+    T = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    s = rng.uniform(0.001, 0.1, N)
+    y = oracle.linear(x, T, s, b)
+    xd = oracle.bf16_bits_to_f64(x)
+    bd = oracle.bf16_bits_to_f64(b)
+    y_lib = xd @ (T.astype(np.float64) * s[:, None]).T + bd
+    np.testing.assert_allclose(y, y_lib, rtol=1e-12, atol=1e-13)
+    y_nobias = oracle.linear(x, T, s, None)
+    np.testing.assert_allclose(y_nobias, y_lib - bd, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- packing
+def two_bit_fields(P: np.ndarray) -> np.ndarray:
+    return np.stack([(P >> sh) & 3 for sh in (0, 2, 4, 6)], axis=-1).ravel()
+
+
+def test_canonical_pack_roundtrip_and_codes():
+    rng = np.random.default_rng(0)
+    T = rng.integers(-1, 2, (37, 48)).astype(np.int8)
+    P = oracle.pack_canonical(T)
+    assert P.size == 37 * 48 // 4
+    fields = two_bit_fields(P)
+    assert not np.any(fields == 2), "pattern 10 must never be written"
+    # counts of each code equal the counts of each value
+    assert np.sum(fields == 1) == np.sum(T == 1)
+    assert np.sum(fields == 3) == np.sum(T == -1)
+    U, bad = oracle.unpack_canonical(P, 37, 48)
+    assert bad == 0
+    np.testing.assert_array_equal(U, T)
+    # a byte holding only the invalid pattern is reported
+    _, bad = oracle.unpack_canonical(np.array([0b10], np.uint8), 1, 4)
+    assert bad == 1
+
+
+def test_canonical_single_rows():
+    assert oracle.pack_canonical(np.array([[-1, -1, -1, -1]], np.int8))[0] == 0xFF
+    assert oracle.pack_canonical(np.array([[0, 0, 1, 0]], np.int8))[0] == 0x10
+    assert oracle.pack_canonical(np.array([[0, -1, 0, 0]], np.int8))[0] == 0x0C
+
+
+def read_positions():
+    out = []
+    with open(os.path.join(GOLDEN, "tiled_positions.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                out.append(tuple(int(v) for v in line.split()))
+    return out
+
+
+@pytest.mark.parametrize("pos", read_positions())
+def test_tiled_layout_hand_positions(pos):
+    N, K, n, k, value, byte, shift = pos
+    T = np.zeros((N, K), np.int8)
+    T[n, k] = value
+    P = oracle.pack_tiled(T)
+    assert P.size == N * K // 4
+    nz = np.nonzero(P)[0]
+    assert list(nz) == [byte]
+    assert P[byte] == ((value & 3) << shift)
+    U, bad = oracle.unpack_tiled(P, N, K)
+    assert bad == 0
+    np.testing.assert_array_equal(U, T)
+
+
+def test_tiled_is_a_permutation_of_canonical():
+    rng = np.random.default_rng(1)
+    N, K = 256, 192
+    T = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    Pt = oracle.pack_tiled(T)
+    Pc = oracle.pack_canonical(T)
+    assert Pt.size == Pc.size == N * K // 4
+    ft, fc = two_bit_fields(Pt), two_bit_fields(Pc)
+    assert np.array_equal(np.bincount(ft, minlength=4), np.bincount(fc, minlength=4))
+    U, bad = oracle.unpack_tiled(Pt, N, K)
+    assert bad == 0
+    np.testing.assert_array_equal(U, T)
+    with pytest.raises(ValueError):
+        oracle.pack_tiled(np.zeros((100, 64), np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack_tiled(np.zeros((128, 48), np.int8))
+
+
+# ------------------------------------------------------------- invariants
+def random_W(N, K, seed, std=0.02):
+    g = torch.Generator().manual_seed(seed)
+    return workloads.bf16_bits((torch.randn(N, K, generator=g) * std).to(torch.bfloat16))
+
+
+def test_quantizer_invariants():
+    W = random_W(64, 96, 3)
+    T, s = oracle.quantize(W, 1e-5)
+    assert set(np.unique(T)) <= {-1, 0, 1}
+    assert np.all(s > 0)
+    # scaling by 2 is exact in bf16: with eps = 0 the scales double, codes stay
+    Wd = oracle.bf16_bits_to_f64(W)
+    W2 = to_bf16_bits((2.0 * Wd).astype(np.float32))
+    T0, s0 = oracle.quantize(W, 0.0)
+    T2, s2 = oracle.quantize(W2, 0.0)
+    np.testing.assert_array_equal(s2, 2.0 * s0)
+    np.testing.assert_array_equal(T2, T0)
+    # negation flips every code and keeps the scale
+    Wn = W ^ np.uint16(0x8000)
+    Tn, sn = oracle.quantize(Wn, 1e-5)
+    np.testing.assert_array_equal(sn, s)
+    np.testing.assert_array_equal(Tn, -T)
+    # a zero row: s = eps and all codes 0; with eps = 0 still all codes 0
+    Z = np.zeros((2, 8), np.uint16)
+    Tz, sz = oracle.quantize(Z, 1e-5)
+    np.testing.assert_array_equal(sz, [1e-5, 1e-5])
+    assert not Tz.any()
+    Tz0, sz0 = oracle.quantize(Z, 0.0)
+    assert not Tz0.any() and not sz0.any()
+    # equal magnitudes: every code is the sign
+    E = to_bf16_bits([[0.5, -0.5, 0.5, 0.5, -0.5, -0.5, 0.5, -0.5]])
+    Te, _ = oracle.quantize(E, 1e-5)
+    np.testing.assert_array_equal(Te[0], np.sign(oracle.bf16_bits_to_f64(E)[0]).astype(np.int8))
+
+
+def test_given_scale_ternarize_and_near_threshold():
+    # eps = 0, row [1, 3]: s = 2, r = [0.5, 1.5]; the 0.5 element sits on the threshold
+    W = to_bf16_bits([[1, 3]])
+    T, s = oracle.quantize(W, 0.0)
+    assert s[0] == 2.0
+    cnt, mask = oracle.near_threshold(W, s, 1e-6)
+    assert cnt == 1 and mask[0, 0] and not mask[0, 1:].any()
+    # a scale a hair off moves r off the threshold by ~1e-7: still counted
+    s_off = s * (1 + 2e-7)
+    cnt2, _ = oracle.near_threshold(W, s_off, 1e-6)
+    assert cnt2 == 1
+    # far from it: not counted
+    cnt3, _ = oracle.near_threshold(W, s * 0.8, 1e-6)
+    assert cnt3 == 0
+    np.testing.assert_array_equal(oracle.ternarize(W, s * 0.8), [[1, 1]])
+    np.testing.assert_array_equal(oracle.ternarize(W, s * 1.2), [[0, 1]])
+
+
+# ------------------------------------------------- the pages' storage figure
+def test_storage_ratio_matches_pages():
+    """7.7x smaller storage with 99.5% of 11.9B parameters ternary (Abstract; Section 1)."""
+    for N, K in [(256, 256), (9216, 3072)]:
+        assert oracle.pack_canonical(np.zeros((N, K), np.int8)).nbytes * 8 == N * K * 2  # 2 bits each
+    layers = workloads.flux_stack()
+    assert len(layers) == 19 * 2 * 5 + 38 * 3
+    p_ternary = sum(l.N * l.K for l in layers)
+    channels = sum(l.N for l in layers)
+    total = 11.9e9
+    assert abs(p_ternary / total - 0.995) < 1e-3  # "99.5% of the 11.9B parameters"
+    bits_bf16 = 16 * total
+    bits_ternary = 2 * p_ternary + 32 * channels + 16 * (total - p_ternary)
+    ratio = bits_bf16 / bits_ternary
+    assert round(ratio, 1) == 7.7
+    # without the per-channel scales and the 0.5% kept in 16 bit it would be 8x
+    assert 16 / 2 == 8.0
