@@ -1,0 +1,75 @@
+// internal.h -- structures shared by the host API (tern_api.cu) and the
+// kernels.  Not part of the public ABI.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace tern {
+
+// One ternary linear problem as the grouped tcgen05 kernel sees it.
+struct alignas(64) Problem {
+  CUtensorMap tmap_x;       // x [M, K] bf16, box {64 k, TOK rows}, 128-byte swizzle
+  const uint8_t* packed;    // tile-interleaved codes
+  const float* scales;      // [N]
+  const __nv_bfloat16* bias;  // [N] or null
+  __nv_bfloat16* y;         // [M, N]
+  float* ws;                // split-K partials [splits][tiles][TOK][128] (splits > 1)
+  int* counters;            // one arrival counter per output tile (splits > 1), zero at rest
+  int M, N, K;
+  int n_tiles, m_tiles, splits;
+  int chunks_per_split;     // 64-wide k chunks per split
+  int cta_begin;            // first CTA of this problem in the grid
+};
+
+constexpr int kMaxProblems = 15;  // keeps the kernel parameter block under 4 KiB
+
+struct Batch {
+  Problem p[kMaxProblems];
+  int count;
+  int total_ctas;
+  unsigned long long wait_limit_ns;
+  unsigned int* status;     // per-device status word (bounded waits report here)
+};
+
+// Token-tile sizes (UMMA N) with a compiled kernel.
+constexpr int kTokTiles[] = {16, 32, 64, 128};
+
+// Per-tile geometry, shared by host (launch) and device (kernel).
+template <int TOK>
+struct TileCfg {
+  static constexpr int kCh = 128;                 // output channels per CTA (UMMA M)
+  static constexpr int kBK = 64;                  // k per pipeline stage
+  static constexpr int kXBytes = TOK * 128;       // TOK rows x 64 bf16, 128-byte swizzled
+  static constexpr int kCBytes = kCh * 16;        // 128 rows x 16 bytes of codes
+  static constexpr int kStageBytes = kXBytes + kCBytes;
+  // Stage counts also size shared memory so that at most two CTAs fit on an
+  // SM: two CTAs use all 512 TMEM columns.
+  static constexpr int kStages = TOK <= 16 ? 20 : TOK <= 32 ? 14 : TOK <= 64 ? 8 : 5;
+  static constexpr int kASlots = 4;               // decoded-weight slots in TMEM
+  static constexpr int kACols = kBK / 2;          // 32-bit TMEM columns per slot (bf16x2)
+  static constexpr int kDCols = TOK < 32 ? 32 : TOK;
+  static constexpr int kTmemCols = (kDCols + kASlots * kACols) <= 256 ? 256 : 512;
+  static constexpr int kDecWarps = TOK <= 64 ? 8 : 4;
+  static constexpr int kThreads = (2 + kDecWarps) * 32;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // Instruction descriptor, kind::f16: D fp32, A bf16, B bf16, both K-major,
+  // N = TOK, M = 128.
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                     (uint32_t(TOK >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+  static_assert(TOK % 16 == 0 && TOK >= 16 && TOK <= 256, "UMMA N for M=128");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(3 * (kSmemBytes + 1024) > 228 * 1024, "a third CTA per SM would exceed TMEM");
+};
+
+cudaError_t launch_ternary_mma(int tok, const Batch& batch, cudaStream_t stream);
+cudaError_t launch_quantize_pack(const __nv_bfloat16* W, int N, int K, float eps, uint8_t* packed,
+                                 float* scales, cudaStream_t stream);
+cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N, int K,
+                              __nv_bfloat16* out, cudaStream_t stream);
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, unsigned int* status,
+                                 cudaStream_t stream);
+int smem_bytes_for_tok(int tok);
+
+}  // namespace tern

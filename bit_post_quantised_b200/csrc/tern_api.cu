@@ -1,0 +1,439 @@
+// tern_api.cu -- host side of the libtern C ABI (include/tern.h): argument
+// checks, tile/split choice, TMA tensor maps, the per-(device, stream)
+// split-K workspace, and the device status word.
+//
+// Page "1.58-bit FLUX" (arXiv 2412.18653): Section 1 defines the ternary
+// weights and their 2-bit storage, Section 4 the unquantised 16-bit
+// activations; this file only routes calls to the kernels that compute them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tern.h"
+
+namespace tern {
+namespace {
+
+__device__ unsigned int g_status_word = 0;  // one instance per device
+
+thread_local std::string t_last_error;
+std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+tern_status fail(tern_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+tern_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(TERN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------ device state
+struct DeviceState {
+  bool checked = false;
+  bool supported = false;
+  int sms = 0;
+  unsigned int* status = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+tern_status current_device(int* dev_out, DeviceState** st_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TERN_ERR_NO_DEVICE, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    if (d.supported) {
+      e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    }
+    d.checked = true;
+  }
+  if (!d.supported)
+    return fail(TERN_ERR_NO_DEVICE, "device %d is not an sm_100 (B200-class) GPU", dev);
+  *dev_out = dev;
+  *st_out = &d;
+  return TERN_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// x [M, K] bf16 row-major; box = 64 k x tok rows; 128-byte swizzle; rows past
+// M read as zero.
+tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int tok) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+  const cuuint32_t box[2] = {64, cuuint32_t(tok)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return TERN_OK;
+}
+
+// ------------------------------------------------------------ workspace
+struct Workspace {
+  float* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* counters = nullptr;
+  size_t n_counters = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+tern_status get_workspace(int dev, cudaStream_t stream, size_t ws_bytes, size_t n_counters,
+                          float** ws, int** counters) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[{dev, stream}];
+  cudaError_t e;
+  if (w.ws_bytes < ws_bytes || w.n_counters < n_counters) {
+    // Kernels queued on this stream may still use the old buffers.
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return cuda_fail(e, "workspace sync");
+    const size_t nb = std::max(ws_bytes, w.ws_bytes), nc = std::max(n_counters, w.n_counters);
+    if (w.ws) cudaFree(w.ws);
+    if (w.counters) cudaFree(w.counters);
+    w = Workspace{};
+    if ((e = cudaMalloc(&w.ws, nb)) != cudaSuccess) return cuda_fail(e, "workspace cudaMalloc");
+    if ((e = cudaMalloc(&w.counters, nc * sizeof(int))) != cudaSuccess) {
+      cudaFree(w.ws);
+      w = Workspace{};
+      return cuda_fail(e, "counter cudaMalloc");
+    }
+    if ((e = cudaMemset(w.counters, 0, nc * sizeof(int))) != cudaSuccess)
+      return cuda_fail(e, "counter cudaMemset");
+    w.ws_bytes = nb;
+    w.n_counters = nc;
+  }
+  *ws = w.ws;
+  *counters = w.counters;
+  return TERN_OK;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+constexpr int64_t kMaxN = int64_t(1) << 20;
+constexpr int64_t kMaxK = int64_t(1) << 20;
+constexpr int64_t kMaxM = int64_t(1) << 26;
+
+tern_status check_nk(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return fail(TERN_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
+  if (N == 0 || K == 0 || N % 128 != 0 || K % 64 != 0)
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "need N %% 128 == 0 and K %% 64 == 0, got N=%lld K=%lld",
+                (long long)N, (long long)K);
+  if (N > kMaxN || K > kMaxK)
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "N or K above 2^20 (N=%lld K=%lld)", (long long)N, (long long)K);
+  return TERN_OK;
+}
+
+tern_status check_linear(const tern_linear_args& a) {
+  tern_status s = check_nk(a.N, a.K);
+  if (s != TERN_OK) return s;
+  if (a.M < 0) return fail(TERN_ERR_INVALID_ARG, "negative M=%lld", (long long)a.M);
+  if (a.M > kMaxM) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "M above 2^26 (M=%lld)", (long long)a.M);
+  if (!a.packed || !a.scales || (a.M > 0 && (!a.x || !a.y)))
+    return fail(TERN_ERR_INVALID_ARG, "null x, packed, scales or y");
+  if (!aligned(a.x, 16) || !aligned(a.packed, 16) || !aligned(a.y, 16) || !aligned(a.scales, 4) ||
+      (a.bias && !aligned(a.bias, 2)))
+    return fail(TERN_ERR_MISALIGNED, "x, packed and y need 16-byte, scales 4-byte, bias 2-byte alignment");
+  const size_t ybytes = size_t(a.M) * size_t(a.N) * 2;
+  if (overlaps(a.y, ybytes, a.x, size_t(a.M) * size_t(a.K) * 2) ||
+      overlaps(a.y, ybytes, a.packed, size_t(a.N) * size_t(a.K) / 4) ||
+      overlaps(a.y, ybytes, a.scales, size_t(a.N) * 4) ||
+      overlaps(a.y, ybytes, a.bias, a.bias ? size_t(a.N) * 2 : 0))
+    return fail(TERN_ERR_INVALID_ARG, "y overlaps an input");
+  return TERN_OK;
+}
+
+int pick_tok(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+// Fills everything of a Problem except cta_begin; returns its CTA count.
+tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, Problem* p,
+                         int64_t* ctas) {
+  std::memset(static_cast<void*>(p), 0, sizeof(Problem));
+  tern_status s = make_x_map(&p->tmap_x, a.x, a.M, a.K, tok);
+  if (s != TERN_OK) return s;
+  p->packed = static_cast<const uint8_t*>(a.packed);
+  p->scales = a.scales;
+  p->bias = static_cast<const __nv_bfloat16*>(a.bias);
+  p->y = static_cast<__nv_bfloat16*>(a.y);
+  p->M = int(a.M);
+  p->N = int(a.N);
+  p->K = int(a.K);
+  p->n_tiles = int(a.N / 128);
+  p->m_tiles = int((a.M + tok - 1) / tok);
+  const int kc_total = int(a.K / 64);
+  int splits = std::max(1, std::min(splits_wanted, kc_total));
+  const int per = (kc_total + splits - 1) / splits;
+  splits = (kc_total + per - 1) / per;  // no empty split
+  p->splits = splits;
+  p->chunks_per_split = per;
+  *ctas = int64_t(p->n_tiles) * p->m_tiles * splits;
+  if (*ctas > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "too many tiles");
+  return TERN_OK;
+}
+
+int ctas_per_sm(int tok) {
+  const int smem = smem_bytes_for_tok(tok);
+  const int by_smem = (228 * 1024) / (smem + 1024);
+  const int by_tmem = 2;  // each CTA allocates 256 of the 512 TMEM columns (tok <= 128)
+  return std::max(1, std::min(by_smem, by_tmem));
+}
+
+}  // namespace
+}  // namespace tern
+
+using namespace tern;
+
+extern "C" {
+
+size_t tern_packed_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || N > kMaxN || K > kMaxK) return 0;
+  return size_t(N) * size_t(K) / 4;
+}
+
+tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float eps, void* packed,
+                               float* scales, tern_stream_t stream) {
+  tern_status s = check_nk(N, K);
+  if (s != TERN_OK) return s;
+  if (!W_bf16 || !packed || !scales) return fail(TERN_ERR_INVALID_ARG, "null W, packed or scales");
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(TERN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (!aligned(W_bf16, 16) || !aligned(packed, 16) || !aligned(scales, 4))
+    return fail(TERN_ERR_MISALIGNED, "W and packed need 16-byte, scales 4-byte alignment");
+  const size_t wb = size_t(N) * size_t(K) * 2, pb = size_t(N) * size_t(K) / 4, sb = size_t(N) * 4;
+  if (overlaps(packed, pb, W_bf16, wb) || overlaps(scales, sb, W_bf16, wb) || overlaps(packed, pb, scales, sb))
+    return fail(TERN_ERR_INVALID_ARG, "outputs overlap each other or W");
+  int dev;
+  DeviceState* ds;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  cudaError_t e = launch_quantize_pack(static_cast<const __nv_bfloat16*>(W_bf16), int(N), int(K), eps,
+                                       static_cast<uint8_t*>(packed), scales,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
+  return TERN_OK;
+}
+
+tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                        const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                        tern_stream_t stream) {
+  const tern_linear_args a{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K};
+  tern_status s = check_linear(a);
+  if (s != TERN_OK) return s;
+  if (M == 0) return TERN_OK;
+  int dev;
+  DeviceState* ds;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  const int tok = pick_tok(M);
+  int splits = 1;
+  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  if (tok <= 64) {
+    // Few tokens: split K so that every SM streams codes.
+    const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
+    if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
+    splits = std::max(1, std::min(splits, 16));
+  }
+  static Batch batch;  // built under the lock below; ~4 KiB, copied into the launch
+  static std::mutex batch_mu;
+  std::lock_guard<std::mutex> lock(batch_mu);
+  std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+  int64_t ctas = 0;
+  if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;
+  Problem& p = batch.p[0];
+  if (p.splits > 1) {
+    const size_t ws_bytes = size_t(p.splits) * size_t(tiles) * tok * 128 * sizeof(float);
+    if ((s = get_workspace(dev, cs, ws_bytes, size_t(tiles), &p.ws, &p.counters)) != TERN_OK) return s;
+  }
+  p.cta_begin = 0;
+  batch.count = 1;
+  batch.total_ctas = int(ctas);
+  batch.wait_limit_ns = g_wait_limit_ns.load();
+  batch.status = ds->status;
+  cudaError_t e = launch_ternary_mma(tok, batch, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "ternary_mma launch");
+  return TERN_OK;
+}
+
+tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream) {
+  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+  for (int i = 0; i < count; ++i) {
+    tern_status s = check_linear(args[i]);
+    if (s != TERN_OK) {
+      t_last_error = "problem " + std::to_string(i) + ": " + t_last_error;
+      return s;
+    }
+  }
+  if (count == 0) return TERN_OK;
+  int dev;
+  DeviceState* ds;
+  tern_status s = current_device(&dev, &ds);
+  if (s != TERN_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  static Batch batch;
+  static std::mutex batch_mu;
+  std::lock_guard<std::mutex> lock(batch_mu);
+  for (int tok : kTokTiles) {
+    std::vector<int> group;
+    for (int i = 0; i < count; ++i)
+      if (args[i].M > 0 && pick_tok(args[i].M) == tok) group.push_back(i);
+    for (size_t g0 = 0; g0 < group.size(); g0 += kMaxProblems) {
+      std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+      int64_t total = 0;
+      int n = 0;
+      for (size_t g = g0; g < group.size() && n < kMaxProblems; ++g, ++n) {
+        int64_t ctas = 0;
+        if ((s = fill_problem(args[group[g]], tok, 1, &batch.p[n], &ctas)) != TERN_OK) return s;
+        batch.p[n].cta_begin = int(total);
+        total += ctas;
+        if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
+      }
+      batch.count = n;
+      batch.total_ctas = int(total);
+      batch.wait_limit_ns = g_wait_limit_ns.load();
+      batch.status = ds->status;
+      cudaError_t e = launch_ternary_mma(tok, batch, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "ternary_mma batch launch");
+    }
+  }
+  return TERN_OK;
+}
+
+tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,
+                            void* W_bf16_out, tern_stream_t stream) {
+  tern_status s = check_nk(N, K);
+  if (s != TERN_OK) return s;
+  if (!packed || !scales || !W_bf16_out) return fail(TERN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(packed, 16) || !aligned(W_bf16_out, 16) || !aligned(scales, 4))
+    return fail(TERN_ERR_MISALIGNED, "packed and output need 16-byte, scales 4-byte alignment");
+  if (overlaps(W_bf16_out, size_t(N) * size_t(K) * 2, packed, size_t(N) * size_t(K) / 4) ||
+      overlaps(W_bf16_out, size_t(N) * size_t(K) * 2, scales, size_t(N) * 4))
+    return fail(TERN_ERR_INVALID_ARG, "output overlaps an input");
+  int dev;
+  DeviceState* ds;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  cudaError_t e = launch_dequantize(static_cast<const uint8_t*>(packed), scales, int(N), int(K),
+                                    static_cast<__nv_bfloat16*>(W_bf16_out),
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return TERN_OK;
+}
+
+tern_status tern_get_device_status(tern_stream_t stream) {
+  int dev;
+  DeviceState* ds;
+  tern_status s = current_device(&dev, &ds);
+  if (s != TERN_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0;
+  if ((e = cudaMemcpy(&word, ds->status, sizeof word, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "status read");
+  if ((e = cudaMemset(ds->status, 0, sizeof word)) != cudaSuccess) return cuda_fail(e, "status clear");
+  if (word & kStatusTimeout) {
+    // A CTA that gave up may have left a split-K arrival counter non-zero;
+    // zero them all so later calls start clean.
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto& kv : g_ws)
+      if (kv.first.first == dev && kv.second.counters) {
+        if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "sync");
+        if ((e = cudaMemset(kv.second.counters, 0, kv.second.n_counters * sizeof(int))) != cudaSuccess)
+          return cuda_fail(e, "counter reset");
+      }
+    return fail(TERN_ERR_TIMEOUT, "a device-side wait ran out of time");
+  }
+  return TERN_OK;
+}
+
+void tern_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(std::max<uint64_t>(limit_ns, 1000));
+}
+
+tern_status tern_selftest_wait_timeout(uint64_t limit_ns, tern_stream_t stream) {
+  int dev;
+  DeviceState* ds;
+  tern_status s = current_device(&dev, &ds);
+  if (s != TERN_OK) return s;
+  if (limit_ns < 1000 || limit_ns > 10000000000ull)
+    return fail(TERN_ERR_INVALID_ARG, "limit_ns must lie in [1e3, 1e10]");
+  cudaError_t e = launch_wait_selftest(limit_ns, ds->status, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return TERN_OK;
+}
+
+const char* tern_status_string(tern_status status) {
+  switch (status) {
+    case TERN_OK: return "ok";
+    case TERN_ERR_INVALID_ARG: return "invalid argument";
+    case TERN_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case TERN_ERR_MISALIGNED: return "misaligned pointer";
+    case TERN_ERR_CUDA: return "CUDA error";
+    case TERN_ERR_TIMEOUT: return "device wait timed out";
+    case TERN_ERR_NO_DEVICE: return "no supported device";
+  }
+  return "unknown status";
+}
+
+const char* tern_last_error(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+"""Python binding of libtern (include/tern.h): argument marshalling only.
+
+Every step of the ternary linear path runs in the library's sm_100a kernels;
+this module only turns torch tensors into pointers, sizes and the current
+CUDA stream, calls the C ABI, and raises on a non-OK status.  There is no
+fallback: if libtern.so is missing or the device is not an sm_100 GPU, the
+calls fail loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern.so")
+_lib = None
+
+TERN_OK = 0
+STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPORTED_SHAPE",
+                -3: "TERN_ERR_MISALIGNED", -4: "TERN_ERR_CUDA", -5: "TERN_ERR_TIMEOUT",
+                -6: "TERN_ERR_NO_DEVICE"}
+
+EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_batch",
+            "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
+            "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
+
+
+class TernError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+
+
+class LinearArgs(ctypes.Structure):
+    """Mirror of tern_linear_args."""
+    _fields_ = [("x", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libtern.so (raising if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libtern.so not found at {_LIB_PATH}; build it with "
+                              "bit_post_quantised_b200._build.build()")
+        L = ctypes.CDLL(_LIB_PATH)
+        i64, vp, st = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        L.tern_packed_bytes.argtypes = [i64, i64]
+        L.tern_packed_bytes.restype = ctypes.c_size_t
+        L.tern_quantize_pack.argtypes = [vp, i64, i64, ctypes.c_float, vp, vp, vp]
+        L.tern_quantize_pack.restype = st
+        L.tern_linear.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
+        L.tern_linear.restype = st
+        L.tern_linear_batch.argtypes = [ctypes.POINTER(LinearArgs), ctypes.c_int, vp]
+        L.tern_linear_batch.restype = st
+        L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
+        L.tern_dequantize.restype = st
+        L.tern_get_device_status.argtypes = [vp]
+        L.tern_get_device_status.restype = st
+        L.tern_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.tern_set_wait_limit_ns.restype = None
+        L.tern_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.tern_selftest_wait_timeout.restype = st
+        L.tern_status_string.argtypes = [st]
+        L.tern_status_string.restype = ctypes.c_char_p
+        L.tern_last_error.argtypes = []
+        L.tern_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != TERN_OK:
+        raise TernError(status, lib().tern_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(lib().tern_packed_bytes(N, K))
+
+
+def quantize_pack(W: torch.Tensor, eps: float = 1e-5, packed: Optional[torch.Tensor] = None,
+                  scales: Optional[torch.Tensor] = None, stream=None):
+    """tern_quantize_pack: W bf16 [N,K] -> (packed uint8 [N*K/4], scales fp32 [N])."""
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty(max(packed_bytes(N, K), 1), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib().tern_quantize_pack(_ptr(W), N, K, float(eps), _ptr(packed), _ptr(scales),
+                                    _stream(stream)))
+    return packed, scales
+
+
+def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+           bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """tern_linear: y = (x . T^T) * s + b, x bf16 [M,K] -> y bf16 [M,N]."""
+    M, K = x.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().tern_linear(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
+                             _stream(stream)))
+    return out
+
+
+def linear_batch(problems: Sequence[dict], stream=None) -> None:
+    """tern_linear_batch over dicts with keys x, packed, scales, bias (or None), y."""
+    arr = (LinearArgs * max(1, len(problems)))()
+    for i, p in enumerate(problems):
+        M, K = p["x"].shape
+        N = p["scales"].shape[0]
+        arr[i] = LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
+                            None if p.get("bias") is None else p["bias"].data_ptr(),
+                            p["y"].data_ptr(), M, N, K)
+    _check(lib().tern_linear_batch(arr, len(problems), _stream(stream)))
+
+
+def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """tern_dequantize: codes -> bf16 [N,K] with W'[n,k] = T[n,k] * s_n."""
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=scales.device)
+    _check(lib().tern_dequantize(_ptr(packed), _ptr(scales), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def device_status(stream=None) -> int:
+    """tern_get_device_status (synchronises the stream); returns the raw status."""
+    return int(lib().tern_get_device_status(_stream(stream)))
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    lib().tern_set_wait_limit_ns(int(limit_ns))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(lib().tern_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def status_string(status: int) -> str:
+    return lib().tern_status_string(int(status)).decode()

@@ -1,0 +1,161 @@
+/*
+ * tern.h -- C ABI of libtern, the B200 (sm_100a) ternary linear layer of
+ * "1.58-bit FLUX" (arXiv 2412.18653).
+ *
+ * The method (page "1.58-bit FLUX", HTML v1):
+ *   Section 1 -- the weights of every linear layer of the vision transformer
+ *     take only the values {-1, 0, +1} ("akin to BitNet b1.58") and are stored
+ *     as 2-bit signed integers instead of 16-bit numbers.
+ *   Section 3.1 -- all linear layers of the double- and single-stream
+ *     transformer blocks are quantised that way.
+ *   Section 4 -- activations are not quantised: x and y stay 16-bit (bf16).
+ * With the absmean quantiser of BitNet b1.58 per output channel n,
+ *     s_n = mean_k |W[n,k]| + eps,   T[n,k] = RoundClip(W[n,k] / s_n, -1, +1),
+ * the layer computes
+ *     y[m,n] = s_n * sum_k x[m,k] * T[n,k] + b_n     (fp32 accumulation).
+ *
+ * Conventions for every call:
+ *   - Every tensor is caller-owned DEVICE memory on the current CUDA device,
+ *     dense and row-major.  The library never frees or keeps a caller pointer.
+ *   - bf16 tensors are passed as `const void*` / `void*` (IEEE bfloat16).
+ *   - Calls are asynchronous and stream-ordered on `stream` (NULL = the legacy
+ *     default stream).  A host-detectable error returns at once with nothing
+ *     launched.  Errors found on the device (a bounded wait that ran out) are
+ *     reported later by tern_get_device_status().
+ *   - Shapes: N % 128 == 0, K % 64 == 0, N, K >= 1; M >= 0 (M == 0 is a
+ *     no-op, and x and y may then be NULL).  Pointers to bf16/packed data must
+ *     be 16-byte aligned, `scales` 4-byte aligned.  Outputs must not overlap
+ *     inputs.
+ *
+ * Packed weight layout ("tile-interleaved", N*K/4 bytes, four codes per byte):
+ *   a code is the 2-bit two's complement integer (+1 -> 01, 0 -> 00,
+ *   -1 -> 11; 10 never occurs).  Codes are grouped in 16-byte groups, one per
+ *   (row n, 64-wide chunk c = k/64), the group at byte offset
+ *       ((n/128) * (K/64) + c) * 2048 + (n % 128) * 16,
+ *   so the 128 rows x 64 k of one tile are one contiguous 2 KiB block and the
+ *   K-chunks of a 128-row slab follow each other.  Inside a group, the
+ *   little-endian 32-bit word w = (k % 64) / 16 holds 16 consecutive k; with
+ *   j = (k % 16) / 2 and h = k % 2 the code of k sits at bits 16*h + 2*j.
+ *   (Even k fill the low half-word and odd k the high half-word, so one
+ *   shift-and-mask yields a bf16x2 pair.)
+ */
+#ifndef TERN_H
+#define TERN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TERN_API __attribute__((visibility("default")))
+#else
+#define TERN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* tern_stream_t;
+
+typedef enum {
+  TERN_OK = 0,
+  TERN_ERR_INVALID_ARG = -1,      /* null pointer, negative size, overlap, bad eps */
+  TERN_ERR_UNSUPPORTED_SHAPE = -2, /* N % 128, K % 64, or a size beyond the limits */
+  TERN_ERR_MISALIGNED = -3,       /* a pointer breaks the alignment rule above */
+  TERN_ERR_CUDA = -4,             /* a CUDA runtime call or launch failed */
+  TERN_ERR_TIMEOUT = -5,          /* a bounded device wait ran out (device status) */
+  TERN_ERR_NO_DEVICE = -6         /* the current device is not an sm_100 GPU */
+} tern_status;
+
+/* Bytes of the packed codes of an N x K ternary matrix: N*K/4.  Returns 0 for
+ * a shape the layout does not support (N % 128, K % 64, or non-positive). */
+TERN_API size_t tern_packed_bytes(int64_t N, int64_t K);
+
+/*
+ * Absmean ternarisation and packing (page "1.58-bit FLUX", Section 1; the
+ * BitNet b1.58 absmean rule it points to).
+ *   W_bf16  [N, K] bf16, read only.
+ *   eps     >= 0 and finite, added to the mean magnitude: s_n = mean|W_n| + eps.
+ *   packed  [N*K/4] bytes, written in the tile-interleaved layout above.
+ *   scales  [N] fp32, written: s_n (the dequantised weight is T[n,k] * s_n).
+ * The mean is accumulated at better than fp32 precision and rounded once to
+ * fp32; a code is +-1 exactly when |W[n,k]| > s_n / 2 (fp32 s_n), else 0,
+ * which is RoundClip with ties to even.  An all-zero row gets s_n = eps and
+ * all-zero codes.
+ */
+TERN_API tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float eps, void* packed,
+                               float* scales, tern_stream_t stream);
+
+/*
+ * Ternary linear layer y = (x . T^T) * s + b (page "1.58-bit FLUX",
+ * Sections 1 and 4).
+ *   x_bf16  [M, K] bf16 activations.
+ *   packed  [N*K/4] codes from tern_quantize_pack (tile-interleaved layout).
+ *   scales  [N] fp32 per-output-channel scales.
+ *   bias    [N] bf16, or NULL for no bias.
+ *   y_bf16  [M, N] bf16 output, overwritten (round to nearest even).
+ * Products are exact (T is +-1/0), sums are fp32, then y = fp32 sum * s + b.
+ * Small M (<= 64) splits K across CTAs and uses a library-owned fp32
+ * workspace per (device, stream), allocated on the first such call; make that
+ * first call outside CUDA stream capture.  Calls on the same stream are
+ * ordered; calls on different streams use different workspaces.
+ */
+TERN_API tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                        const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                        tern_stream_t stream);
+
+/* One independent linear problem of a batch (same meaning as tern_linear). */
+typedef struct {
+  const void* x;      /* [M, K] bf16 */
+  const void* packed; /* [N*K/4] codes */
+  const float* scales; /* [N] fp32 */
+  const void* bias;   /* [N] bf16 or NULL */
+  void* y;            /* [M, N] bf16 */
+  int64_t M, N, K;
+} tern_linear_args;
+
+/*
+ * Several independent ternary linears (for instance the per-stream adaLN
+ * modulation GEMVs and projections of one FLUX block) with as few launches as
+ * possible: problems with similar M share one grouped launch.  `args` is host
+ * memory, read before the call returns.  Every problem is validated before
+ * anything is launched; on an error nothing runs.  count == 0 is a no-op.
+ * Batched problems do not split K, so they need no workspace.
+ */
+TERN_API tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream);
+
+/*
+ * Expands packed codes to the dequantised bf16 weight W'[n,k] = T[n,k] * s_n
+ * ([N, K] row-major).  Not on the inference path: it feeds dense reference
+ * GEMMs for comparison.
+ */
+TERN_API tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,
+                            void* W_bf16_out, tern_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: TERN_ERR_TIMEOUT if any kernel's bounded wait ran out since
+ * the last call, TERN_OK otherwise (TERN_ERR_CUDA if the sync itself failed). */
+TERN_API tern_status tern_get_device_status(tern_stream_t stream);
+
+/* Wall-time limit of every device-side wait, in nanoseconds (default 1e9).
+ * Values below 1000 are clamped to 1000. */
+TERN_API void tern_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Launches one tiny kernel whose wait on an mbarrier nothing ever arrives at
+ * must run out after `limit_ns`; it exists so tests can see a device-side
+ * timeout reported through tern_get_device_status() without faulting or
+ * hanging the GPU. */
+TERN_API tern_status tern_selftest_wait_timeout(uint64_t limit_ns, tern_stream_t stream);
+
+/* Static description of a status code. */
+TERN_API const char* tern_status_string(tern_status status);
+
+/* Detail of the last failure on the calling host thread ("" if none). */
+TERN_API const char* tern_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERN_H */

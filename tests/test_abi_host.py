@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load, export every entry point include/tern.h declares, and
+reject every invalid call on the host with the documented status before
+anything is launched.  Pointers here are fake addresses: every call below is
+invalid in at least one way, so nothing is ever dereferenced or launched.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+from bit_post_quantised_b200 import _build, tern
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, SHAPE, MISALIGNED = 0, -1, -2, -3
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return tern.lib()
+
+
+def declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "tern.h")).read()
+    return re.findall(r"^TERN_API\s+[^;(]*?\b(tern_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for required in ("tern_quantize_pack", "tern_linear", "tern_linear_batch"):
+        assert required in names
+    assert set(names) == set(tern.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", tern.library_path()], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in declared_entry_points():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_packed_bytes(L):
+    assert tern.packed_bytes(9216, 3072) == 9216 * 3072 // 4
+    assert tern.packed_bytes(128, 64) == 2048
+    for N, K in [(0, 64), (128, 0), (100, 64), (128, 48), (-128, 64), (1 << 21, 64)]:
+        assert tern.packed_bytes(N, K) == 0
+
+
+def test_status_strings(L):
+    assert tern.status_string(0) == "ok"
+    assert "timed out" in tern.status_string(-5)
+    assert tern.status_string(123) == "unknown status"
+
+
+F = 0x7F0000000000  # a fake, 256-byte aligned address that is never dereferenced
+
+
+def call_linear(L, x=F, M=16, K=256, packed=F + 0x100000, scales=F + 0x200000, bias=None, N=256,
+                y=F + 0x300000):
+    return L.tern_linear(ctypes.c_void_p(x), M, K, ctypes.c_void_p(packed), ctypes.c_void_p(scales),
+                         None if bias is None else ctypes.c_void_p(bias), N, ctypes.c_void_p(y), None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(N=100), SHAPE), (dict(K=100), SHAPE), (dict(N=0), SHAPE), (dict(K=0), SHAPE),
+    (dict(N=-128), INVALID), (dict(M=-1), INVALID), (dict(N=1 << 21), SHAPE), (dict(M=1 << 27), SHAPE),
+    (dict(x=0), INVALID), (dict(packed=0), INVALID), (dict(scales=0), INVALID), (dict(y=0), INVALID),
+    (dict(x=F + 2), MISALIGNED), (dict(packed=F + 0x100008), MISALIGNED), (dict(y=F + 0x300004), MISALIGNED),
+    (dict(scales=F + 0x200002), MISALIGNED), (dict(bias=F + 0x400001), MISALIGNED),
+    (dict(y=F), INVALID),                 # y aliases x
+    (dict(y=F + 0x100000), INVALID),      # y aliases packed
+    (dict(bias=F + 0x300010), INVALID),   # bias inside y
+])
+def test_linear_rejects_on_host(L, kw, expected):
+    assert call_linear(L, **kw) == expected
+    assert L.tern_last_error().decode() != ""
+
+
+def test_quantize_rejects_on_host(L):
+    q = lambda W=F, N=256, K=256, eps=1e-5, P=F + 0x1000000, S=F + 0x2000000: L.tern_quantize_pack(
+        ctypes.c_void_p(W), N, K, eps, ctypes.c_void_p(P), ctypes.c_void_p(S), None)
+    assert q(N=200) == SHAPE
+    assert q(K=32) == SHAPE
+    assert q(W=0) == INVALID
+    assert q(eps=-1.0) == INVALID
+    assert q(eps=float("nan")) == INVALID
+    assert q(eps=float("inf")) == INVALID
+    assert q(W=F + 8) == MISALIGNED
+    assert q(S=F + 0x2000001) == MISALIGNED
+    assert q(P=F + 0x10) == INVALID  # packed overlaps W
+
+
+def test_batch_rejects_on_host(L):
+    arr = (tern.LinearArgs * 2)()
+    arr[0] = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, 16, 256, 256)
+    arr[1] = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, 16, 100, 256)
+    assert L.tern_linear_batch(arr, 2, None) == SHAPE
+    assert "problem 1" in L.tern_last_error().decode()
+    assert L.tern_linear_batch(arr, -1, None) == INVALID
+    assert L.tern_linear_batch(None, 3, None) == INVALID
+
+
+def test_dequantize_rejects_on_host(L):
+    d = lambda P=F, S=F + 0x100000, N=256, K=256, O=F + 0x200000: L.tern_dequantize(
+        ctypes.c_void_p(P), ctypes.c_void_p(S), N, K, ctypes.c_void_p(O), None)
+    assert d(N=12) == SHAPE
+    assert d(P=0) == INVALID
+    assert d(O=F + 2) == MISALIGNED
+    assert d(O=F) == INVALID
+
+
+def test_selftest_rejects_bad_limit_without_gpu(L):
+    # no GPU here: the device check fails before any launch
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-only check")
+    assert L.tern_selftest_wait_timeout(10, None) != OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    code = ("import bit_post_quantised_b200.tern as t; t._LIB_PATH = '/nonexistent/libtern.so'\n"
+            "try:\n    t.packed_bytes(128, 64)\nexcept ImportError as e:\n    print('LOUD', e)\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert "LOUD" in out.stdout, out.stderr
+
+
+def test_linear_with_no_tokens_is_a_host_noop(L):
+    assert call_linear(L, M=0, x=0, y=0) == OK

@@ -1,0 +1,285 @@
+"""GPU parity: the sm_100a kernels behind the C ABI against the fp64 CPU oracle.
+
+Rules (written here, checked element by element):
+  * scales: |s_gpu - s_oracle| <= 1e-6 * s_oracle;
+  * codes: bit-exact given the GPU's scales, except elements whose |w|/s lies
+    within 1e-6 of the 0.5 rounding threshold, which are counted and reported;
+  * linear: |y - y_ref| <= 8e-3 |y_ref| + 1e-3 rms(y_ref), with y_ref the
+    oracle's fp64 linear on the GPU-produced codes and scales.  The bound
+    covers bf16's 2^-9 relative output rounding plus fp32 accumulation.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_post_quantised_b200 import tern, workloads
+
+pytestmark = pytest.mark.gpu
+
+SCALE_RTOL = 1e-6
+BAND = 1e-6
+Y_RTOL = 8e-3
+Y_RMS = 1e-3
+EPS = workloads.EPS
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return workloads.bf16_bits(t.detach().cpu())
+
+
+def rand_bf16(shape, std, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+
+
+def quantize_on_gpu(W_cpu: torch.Tensor):
+    W = W_cpu.cuda()
+    packed, scales = tern.quantize_pack(W, EPS)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    return packed, scales
+
+
+def check_quantize(W_cpu, packed, scales, report):
+    N, K = W_cpu.shape
+    Wb = bits(W_cpu)
+    s_gpu = scales.cpu().double().numpy()
+    s_ref = oracle.absmean_scales(Wb, EPS)
+    rel = np.abs(s_gpu - s_ref) / s_ref
+    assert rel.max() <= SCALE_RTOL, f"scale rel err {rel.max():.3e}"
+    P = packed.cpu().numpy()
+    assert P.size == N * K // 4
+    T_gpu, bad = oracle.unpack_tiled(P, N, K)
+    assert bad == 0, "pattern 10 written"
+    T_ref = oracle.ternarize(Wb, s_gpu)
+    near_cnt, near = oracle.near_threshold(Wb, s_gpu, BAND)
+    diff = T_gpu != T_ref
+    assert not np.any(diff & ~near), f"{int(np.sum(diff & ~near))} codes differ off the threshold"
+    report["near_threshold"] = near_cnt
+    report["near_flips"] = int(np.sum(diff & near))
+    # end to end against the oracle's own quantisation: only threshold flips
+    T_own, _ = oracle.quantize(Wb, EPS)
+    near_own_cnt, near_own = oracle.near_threshold(Wb, s_ref, BAND)
+    d2 = T_gpu != T_own
+    assert not np.any(d2 & ~near_own)
+    return T_gpu, s_gpu
+
+
+def check_y(y_gpu: torch.Tensor, y_ref: np.ndarray):
+    y = y_gpu.detach().cpu().double().numpy()
+    assert y.shape == y_ref.shape
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    err = np.abs(y - y_ref)
+    bound = Y_RTOL * np.abs(y_ref) + Y_RMS * rms
+    bad = err > bound
+    assert not bad.any(), (f"{int(bad.sum())} of {bad.size} outputs out of tolerance; "
+                           f"worst err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}")
+    return float((err / (np.abs(y_ref) + rms)).max()) if y_ref.size else 0.0
+
+
+# ------------------------------------------------------------- quantise/pack
+@pytest.mark.parametrize("N,K", [(128, 64), (256, 256), (384, 320), (128, 1024), (1280, 3072)])
+def test_quantize_pack_small(N, K):
+    W = rand_bf16((N, K), 0.02, N * 7 + K)
+    packed, scales = quantize_on_gpu(W)
+    check_quantize(W, packed, scales, {})
+
+
+def test_quantize_pack_special_rows():
+    """Zero rows, equal magnitudes, exact threshold ties, large and tiny values."""
+    N, K = 128, 128
+    W = rand_bf16((N, K), 0.02, 99)
+    W[0] = 0
+    W[1] = 0.5
+    W[2, ::2] = -0.25
+    W[2, 1::2] = 0.25
+    W[3, :2] = torch.tensor([1.0, 3.0])  # mean 4/128, far above threshold
+    W[3, 2:] = 0
+    W[4] = torch.tensor([1e-30] * K)
+    W[5, 0] = 1e4
+    packed, scales = quantize_on_gpu(W)
+    check_quantize(W, packed, scales, {})
+    s = scales.cpu()
+    assert s[0].item() == pytest.approx(EPS, rel=1e-7)
+    T, _ = oracle.unpack_tiled(packed.cpu().numpy(), N, K)
+    assert not T[0].any()
+    assert (T[1] == 1).all()
+
+
+@pytest.mark.parametrize("N,K", [(9216, 3072), (12288, 3072), (3072, 12288), (21504, 3072), (3072, 15360),
+                                 (18432, 3072)])
+def test_quantize_pack_flux_shapes(N, K):
+    """Every weight shape of the FLUX linear stack, in full."""
+    W = rand_bf16((N, K), workloads.W_STD, 5000 + N + K)
+    packed, scales = quantize_on_gpu(W)
+    rep = {}
+    check_quantize(W, packed, scales, rep)
+    print(f"N={N} K={K}: near-threshold elements {rep['near_threshold']}, flips {rep['near_flips']}")
+
+
+# ---------------------------------------------------------------- linear
+def run_linear_case(M, N, K, seed, with_bias=True, x_std=1.0):
+    W = rand_bf16((N, K), 0.02, seed)
+    x = rand_bf16((M, K), x_std, seed + 1)
+    b = rand_bf16((N,), 0.01, seed + 2) if with_bias else None
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear(x.cuda(), packed, scales, None if b is None else b.cuda())
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    y_ref = oracle.linear(bits(x), T, s, None if b is None else bits(b))
+    return check_y(y, y_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 15, 16, 17, 31, 32, 33, 48, 63, 64, 65, 100, 127, 128, 129, 200, 300])
+def test_linear_token_counts(M):
+    run_linear_case(M, 384, 320, seed=M)
+
+
+@pytest.mark.parametrize("N,K", [(128, 64), (128, 128), (256, 448), (512, 1024), (1024, 3072)])
+@pytest.mark.parametrize("M", [1, 24, 64, 130])
+def test_linear_shapes(M, N, K):
+    run_linear_case(M, N, K, seed=N + K + M)
+
+
+def test_linear_no_bias():
+    run_linear_case(40, 256, 256, seed=3, with_bias=False)
+    run_linear_case(257, 256, 256, seed=4, with_bias=False)
+
+
+def test_linear_tiny_config():
+    L = workloads.CONFIGS["tiny"]
+    x, W, b = workloads.make_inputs(L)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear(x.cuda(), packed, scales, b.cuda())
+    y_ref = oracle.linear(bits(x), T, s, bits(b))
+    check_y(y, y_ref)
+    # end to end against the oracle's own quantisation
+    T_own, s_own = oracle.quantize(bits(W), EPS)
+    check_y(y, oracle.linear(bits(x), T_own, s_own, bits(b)))
+
+
+def test_linear_deterministic_and_canaries():
+    M, N, K = 33, 256, 512
+    W = rand_bf16((N, K), 0.02, 11)
+    x = rand_bf16((M, K), 1.0, 12).cuda()
+    packed, scales = quantize_on_gpu(W)
+    buf = torch.full((M * N + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    y1 = buf[2048:2048 + M * N].view(M, N)
+    tern.linear(x, packed, scales, None, out=y1)
+    y2 = tern.linear(x, packed, scales, None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2), "two runs differ"
+    assert (buf[:2048] == 7.0).all() and (buf[2048 + M * N:] == 7.0).all(), "wrote outside y"
+
+
+def test_linear_m_zero_is_noop():
+    W = rand_bf16((128, 64), 0.02, 1)
+    packed, scales = quantize_on_gpu(W)
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    y = tern.linear(x, packed, scales)
+    assert y.shape == (0, 128)
+
+
+def test_linear_rejects_misaligned_pointer():
+    W = rand_bf16((128, 64), 0.02, 1)
+    packed, scales = quantize_on_gpu(W)
+    xbuf = torch.zeros(4 * 64 + 8, dtype=torch.bfloat16, device="cuda")
+    x = xbuf[1:1 + 4 * 64].view(4, 64)  # 2-byte offset
+    with pytest.raises(tern.TernError) as e:
+        tern.linear(x, packed, scales)
+    assert e.value.status == -3
+
+
+# ---------------------------------------------------------------- batch
+def test_linear_batch_mixed_sizes():
+    cases = [(1, 256, 192), (16, 384, 256), (70, 128, 128), (300, 256, 320), (2, 512, 64), (130, 128, 576)]
+    probs, refs = [], []
+    for i, (M, N, K) in enumerate(cases):
+        W = rand_bf16((N, K), 0.02, 100 + i)
+        x = rand_bf16((M, K), 1.0, 200 + i)
+        b = rand_bf16((N,), 0.01, 300 + i) if i % 2 == 0 else None
+        packed, scales = quantize_on_gpu(W)
+        T, s = check_quantize(W, packed, scales, {})
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        probs.append(dict(x=x.cuda(), packed=packed, scales=scales, bias=None if b is None else b.cuda(), y=y))
+        refs.append(oracle.linear(bits(x), T, s, None if b is None else bits(b)))
+    tern.linear_batch(probs)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    for p, r in zip(probs, refs):
+        check_y(p["y"], r)
+    tern.linear_batch([])
+
+
+def test_linear_batch_rejects_bad_problem_before_launch():
+    W = rand_bf16((128, 64), 0.02, 1)
+    packed, scales = quantize_on_gpu(W)
+    x = rand_bf16((4, 64), 1.0, 2).cuda()
+    y = torch.full((4, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    bad_y = torch.empty(4, 128, dtype=torch.bfloat16, device="cuda")
+    probs = [dict(x=x, packed=packed, scales=scales, bias=None, y=y),
+             dict(x=x, packed=packed, scales=scales, bias=None, y=bad_y)]
+    probs[1]["y"] = x  # aliasing input and output
+    with pytest.raises(tern.TernError):
+        tern.linear_batch(probs)
+    torch.cuda.synchronize()
+    assert (y == 3.0).all(), "nothing may run when one problem is invalid"
+
+
+# ------------------------------------------------------------- full sizes
+def sampled_reference(L, x, T, s, b, rows):
+    return oracle.linear(bits(x[rows]), T, s, bits(b))
+
+
+@pytest.mark.parametrize("name", ["qkv", "mlp_up", "mlp_down"])
+def test_linear_flux_layers_sampled(name):
+    """Full-size layers in the launch configuration the benchmark times; the
+    oracle checks 48 seeded token rows against every output channel."""
+    L = workloads.CONFIGS[name]
+    x, W, b = workloads.make_inputs(L)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear(x.cuda(), packed, scales, b.cuda())
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    rows = np.sort(np.random.default_rng(L.seed).choice(L.M, 48, replace=False))
+    rows[-1] = L.M - 1  # include the last (ragged-free but boundary) row
+    check_y(y[torch.from_numpy(rows).cuda()], sampled_reference(L, x, T, s, b, rows))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 64])
+@pytest.mark.parametrize("mult", [6, 3])
+def test_linear_modulation_gemv_full(M, mult):
+    """adaLN modulation GEMV sweep, every output against the oracle."""
+    L = workloads.CONFIGS[f"mod{mult}_m{M}"]
+    x, W, b = workloads.make_inputs(L)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear(x.cuda(), packed, scales, b.cuda())
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    check_y(y, oracle.linear(bits(x), T, s, bits(b)))
+
+
+def test_dequantize_matches_codes_times_scales():
+    N, K = 256, 192
+    W = rand_bf16((N, K), 0.02, 77)
+    packed, scales = quantize_on_gpu(W)
+    Wd = tern.dequantize(packed, scales, K)
+    T, _ = oracle.unpack_tiled(packed.cpu().numpy(), N, K)
+    ref = (torch.from_numpy(T.astype(np.float32)) * scales.cpu()[:, None]).to(torch.bfloat16)
+    assert torch.equal(Wd.cpu(), ref)
+
+
+# ---------------------------------------------------------- failure detection
+def test_device_wait_timeout_is_reported_and_context_survives():
+    assert tern.device_status() == 0
+    tern.selftest_wait_timeout(5_000_000)  # 5 ms wait that nothing satisfies
+    assert tern.device_status() == -5
+    assert tern.device_status() == 0  # cleared by the read
+    run_linear_case(8, 128, 64, seed=5)  # the context is still usable
