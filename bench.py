@@ -1,0 +1,492 @@
+"""Benchmark of the ternary linear hot path of 1.58-bit FLUX on B200.
+
+One step = the whole path on the FLUX.1-dev double-block image-stream QKV
+layer (x [4096, 3072] bf16, W [9216, 3072] bf16 -> ternary codes, y [4096,
+9216] bf16): absmean quantise/pack of W, then the ternary linear y =
+(x . T^T) * s + b.  Inputs are seeded synthetic tensors of that shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is whole-job throughput in TFLOP/s
+(2*M*N*K per step per GPU); multi-GPU runs are independent replicas (each
+rank its own tokens and weights; weak scaling, no collective on the data
+path).  `--impl reference` times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ternary-linear TFLOP/s & packed-weight GB/s at FLUX shapes; % of roofline"
+WORKLOAD = "qkv"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "ternary_mma_qkv.md")
+KERNEL_SOURCE = os.path.join(ROOT, "bit_post_quantised_b200", "csrc", "ternary_mma.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tern", "reference"], default="tern")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-kernel side table")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU oracle sample budget (0 skips the CPU baseline, for profiling runs)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the linear kernel from the committed ncu
+    summary, or None if there is none or the kernel changed since."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_src or not m_tr or m_src.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if self.proc is None or not getattr(self, "out", ""):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        hi = max(sm)
+        loaded = [v for v in sm if v >= 0.5 * hi] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle leg
+def oracle_sample_step(layer, x, W, b, budget_s: float):
+    """Times the fp64 CPU oracle on a bounded sample of one step: the full
+    quantise + tiled pack of W, and the linear on as many leading token rows
+    as fit the time budget.  Returns (extrapolated full-step seconds, rows)."""
+    import oracle
+    from bit_post_quantised_b200 import workloads
+
+    Wb, xb, bb = workloads.bf16_bits(W), workloads.bf16_bits(x), workloads.bf16_bits(b)
+    t0 = time.perf_counter()
+    T, s = oracle.quantize(Wb, workloads.EPS)
+    oracle.pack_tiled(T)
+    t_quant = time.perf_counter() - t0
+    rows, t_lin = 0, 0.0
+    chunk = max(1, 2 * oracle.num_threads())
+    while rows < layer.M and t_lin < budget_s:
+        n = min(chunk, layer.M - rows)
+        t1 = time.perf_counter()
+        oracle.linear(xb[rows:rows + n], T, s, bb)
+        t_lin += time.perf_counter() - t1
+        rows += n
+        chunk = min(chunk * 2, 256)
+    return t_quant + t_lin * layer.M / rows, rows, t_quant, t_lin
+
+
+def cpu_baseline(layer, x, W, b, budget_s: float):
+    import oracle
+
+    est, rows, t_quant, t_lin = oracle_sample_step(layer, x, W, b, budget_s)
+    return {"value": layer.flop / est / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"full quantise+pack of W [{layer.N},{layer.K}] ({t_quant:.2f} s) and the fp64 "
+                       f"linear on {rows} of {layer.M} token rows ({t_lin:.2f} s), extrapolated "
+                       f"linearly in rows to the full step ({est:.1f} s)")}
+
+
+def run_reference(args):
+    """--impl reference: the oracle as it stands, on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    if rank != 0:
+        return 0
+    from bit_post_quantised_b200 import workloads
+
+    layer = workloads.CONFIGS[WORKLOAD]
+    x, W, b = workloads.make_inputs(layer)
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_step(layer, x, W, b, per_step)
+    ests, samples = [], []
+    for _ in range(args.steps):
+        est, rows, tq, tl = oracle_sample_step(layer, x, W, b, per_step)
+        ests.append(est)
+        samples.append(rows)
+    import oracle
+
+    step_s = statistics.mean(ests)
+    value = layer.flop / step_s / 1e12
+    sample = (f"each step: full quantise+pack of W and the fp64 linear on the leading "
+              f"{min(samples)}-{max(samples)} of {layer.M} token rows, extrapolated to the full step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, FLUX.1-dev QKV shapes)",
+        "config": workload_config(layer),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(layer):
+    return {"workload": f"FLUX.1-dev double-block image-stream QKV, 1024x1024 image: "
+                        f"x [{layer.M},{layer.K}] bf16, W [{layer.N},{layer.K}] ternary, bias bf16",
+            "M": layer.M, "K": layer.K, "N": layer.N, "eps": 1e-5,
+            "step": "tern_quantize_pack(W) + tern_linear(x)",
+            "accumulate": "fp32",
+            "l2": "two rotating input sets of 164 MB each (> 126 MB L2)"}
+
+
+# ------------------------------------------------------------ GPU arm
+def setup_dist(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    import torch
+
+    if world == 1:
+        return value
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def make_sets(layer, rank, n_sets, device):
+    """Per-rank input sets (rank-dependent seeds: independent replicas)."""
+    import dataclasses
+
+    import torch
+
+    from bit_post_quantised_b200 import workloads
+
+    sets = []
+    for i in range(n_sets):
+        L = dataclasses.replace(layer, seed=layer.seed + 7919 * rank + 104729 * i)
+        x, W, b = workloads.make_inputs(L)
+        sets.append({
+            "x": x.to(device), "W": W.to(device), "b": b.to(device),
+            "packed": torch.empty(layer.N * layer.K // 4, dtype=torch.uint8, device=device),
+            "scales": torch.empty(layer.N, dtype=torch.float32, device=device),
+            "y": torch.empty(layer.M, layer.N, dtype=torch.bfloat16, device=device),
+            "cpu": (x, W, b),
+        })
+    return sets
+
+
+def graph_time(calls, replays, stream):
+    """Device time per call of a list of launches captured in one CUDA graph
+    (removes host launch overhead from microsecond kernels)."""
+    import torch
+
+    for c in calls:  # warm-up outside capture (allocates any workspace)
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(replays):
+        g.replay()
+    e1.record(cur)
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e-3 / (replays * len(calls))
+
+
+def side_table(device, peaks, stream):
+    """Per-kernel figures for the other rows of the path (not the headline):
+    the adaLN modulation GEMV sweep, the MLP layers, quantise/pack, and bf16
+    cuBLAS on the dequantised weight as context.  Weights rotate over enough
+    copies that they do not stay in L2 between launches."""
+    import torch
+    import torch.nn.functional as F
+
+    from bit_post_quantised_b200 import tern, workloads
+
+    rows = {}
+    l2 = 126 * 2 ** 20
+    for name in ["mod6_m1", "mod6_m4", "mod6_m16", "mod6_m64", "mod3_m1", "mod3_m4", "mod3_m16",
+                 "mod3_m64", "mlp_up", "mlp_down"]:
+        L = workloads.CONFIGS[name]
+        x, W, b = (t.to(device) for t in workloads.make_inputs(L))
+        copies = max(2, min(24, int(3 * l2 // max(1, L.packed_bytes)) + 1))
+        packs = []
+        for _ in range(copies):
+            packs.append(tern.quantize_pack(W, workloads.EPS, stream=stream))
+        y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=device)
+        calls = [(lambda p=p, s=s: tern.linear(x, p, s, b, out=y)) for p, s in packs]
+        reps = max(2, 64 // copies)
+        t = graph_time(calls * reps, 5, stream)
+        flop_t = 2.0 * L.M * L.N * L.K / peaks["bf16_tflops"] / 1e12
+        byte_t = L.algorithmic_bytes / peaks["hbm_gbs"] / 1e9
+        entry = {"M": L.M, "N": L.N, "K": L.K, "us": t * 1e6, "tflops": L.flop / t / 1e12,
+                 "packed_gbs": L.packed_bytes / t / 1e9, "roofline_frac": max(flop_t, byte_t) / t,
+                 "bound": "tensor" if flop_t > byte_t else "hbm"}
+        if name in ("mlp_up", "mlp_down", "mod6_m64"):
+            Wd = tern.dequantize(packs[0][0], packs[0][1], L.K, stream=stream)
+            torch.cuda.synchronize()
+            tc = graph_time([lambda: F.linear(x, Wd, b)] * 10, 5, stream)
+            entry["cublas_bf16_us"] = tc * 1e6
+            del Wd
+        rows[name] = entry
+        del packs
+    # quantise/pack of the largest weight
+    N, K = 21504, 3072
+    W = (torch.randn(N, K, device=device) * 0.02).to(torch.bfloat16)
+    p = torch.empty(N * K // 4, dtype=torch.uint8, device=device)
+    s = torch.empty(N, dtype=torch.float32, device=device)
+    t = graph_time([lambda: tern.quantize_pack(W, packed=p, scales=s)] * 10, 5, stream)
+    nbytes = 2 * N * K + N * K // 4 + 4 * N
+    rows["quantize_pack_21504x3072"] = {"us": t * 1e6, "gbs": nbytes / t / 1e9,
+                                        "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    return rows
+
+
+def gpu_id_for_smi(local: int) -> str:
+    """nvidia-smi --id for the CUDA device (by UUID, so visible-device
+    remapping cannot point the sampler at another GPU)."""
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local)
+
+
+def run_tern(args):
+    import torch
+
+    from bit_post_quantised_b200 import tern, workloads
+
+    world, rank, local = setup_dist(args)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device)
+    peaks = load_peaks()
+    layer = workloads.CONFIGS[WORKLOAD]
+    sets = make_sets(layer, rank, 2, device)
+    K, Wm = args.steps, max(3, args.warmup)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(i, events=None):
+        st = sets[i % len(sets)]
+        if events:
+            events[0].record(stream)
+        tern.quantize_pack(st["W"], workloads.EPS, packed=st["packed"], scales=st["scales"], stream=stream)
+        if events:
+            events[1].record(stream)
+        tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        if events:
+            events[2].record(stream)
+
+    for i in range(Wm):
+        step(i)
+    barrier(world)
+    if tern.device_status(stream) != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id_for_smi(local)) as clocks:
+        barrier(world)
+        t0.record(stream)
+        for i in range(K):
+            step(i, ev[i])
+        t1.record(stream)
+        t1.synchronize()
+        barrier(world)
+    elapsed = max_over_ranks(t0.elapsed_time(t1) * 1e-3, world)
+    if tern.device_status(stream) != 0:
+        raise RuntimeError("device wait timed out during the timed steps")
+    t_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) * 1e-3
+    t_lin = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) * 1e-3
+    t_lin = max_over_ranks(t_lin, world)
+
+    # ---- end to end through the public API, from pinned host buffers
+    host = []
+    for st in sets:
+        x, W, b = st["cpu"]
+        host.append({"x": x.pin_memory(), "W": W.pin_memory(), "b": b.pin_memory(),
+                     "y": torch.empty(layer.M, layer.N, dtype=torch.bfloat16).pin_memory()})
+    h2d = sum(host[0][k].numel() * host[0][k].element_size() for k in ("x", "W", "b"))
+    d2h = host[0]["y"].numel() * host[0]["y"].element_size()
+
+    def e2e_step(i):
+        st, hs = sets[i % len(sets)], host[i % len(host)]
+        with torch.cuda.stream(stream):
+            st["W"].copy_(hs["W"], non_blocking=True)
+            st["x"].copy_(hs["x"], non_blocking=True)
+            st["b"].copy_(hs["b"], non_blocking=True)
+        tern.quantize_pack(st["W"], workloads.EPS, packed=st["packed"], scales=st["scales"], stream=stream)
+        tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        with torch.cuda.stream(stream):
+            hs["y"].copy_(st["y"], non_blocking=True)
+
+    for i in range(Wm):
+        e2e_step(i)
+    barrier(world)
+    t0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    t1.record(stream)
+    t1.synchronize()
+    barrier(world)
+    e2e_elapsed = max_over_ranks(t0.elapsed_time(t1) * 1e-3, world)
+
+    flop = layer.flop
+    value = world * K * flop / elapsed / 1e12
+    achieved = flop / t_lin / 1e12
+    traffic = profiled_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, FLUX.1-dev QKV shapes)",
+        "config": workload_config(layer),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "ternary_mma_kernel<128> (tern_linear)",
+                     "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"},
+        "linear_us": t_lin * 1e6, "quantize_pack_us": t_quant * 1e6,
+        "packed_weight_gbs": layer.packed_bytes / t_lin / 1e9,
+        "quantize_pack_gbs": (2 * layer.N * layer.K + layer.packed_bytes + 4 * layer.N) / t_quant / 1e9,
+        "e2e": {"value": world * K * flop / e2e_elapsed / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K * world,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        line["cpu_baseline"] = cpu_baseline(layer, *sets[0]["cpu"], budget_s=args.cpu_seconds)
+        if not args.no_extras:
+            line["side_table"] = side_table(device, peaks, stream)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_tern(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
