@@ -31,7 +31,7 @@ if ROOT not in sys.path:
 METRIC = "ternary-linear TFLOP/s & packed-weight GB/s at FLUX shapes; % of roofline"
 WORKLOAD = "qkv"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "ternary_mma_qkv.md")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCE = os.path.join(ROOT, "bit_post_quantised_b200", "csrc", "ternary_mma.cu")
 
 
@@ -41,6 +41,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tern", "reference"], default="tern")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="layer the step runs on (default: the QKV headline; others for profiling)")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-kernel side table")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU oracle sample budget (0 skips the CPU baseline, for profiling runs)")
@@ -64,11 +66,11 @@ def kernel_source_hash() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the linear kernel from the committed ncu
-    summary, or None if there is none or the kernel changed since."""
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the linear kernel on this workload from the
+    committed ncu summary, or None if there is none or the kernel changed since."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(os.path.join(PROFILE_DIR, f"ternary_mma_{workload}.md")).read()
     except OSError:
         return None
     m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
@@ -179,7 +181,7 @@ def run_reference(args):
         return 0
     from bit_post_quantised_b200 import workloads
 
-    layer = workloads.CONFIGS[WORKLOAD]
+    layer = workloads.CONFIGS[args.workload]
     x, W, b = workloads.make_inputs(layer)
     per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -209,9 +211,15 @@ def run_reference(args):
     return 0
 
 
+DESCRIPTIONS = {"qkv": "FLUX.1-dev double-block image-stream QKV, 1024x1024 image",
+                "mlp_up": "FLUX.1-dev MLP up projection, 4608 tokens",
+                "mlp_down": "FLUX.1-dev MLP down projection, 4608 tokens",
+                "tiny": "tiny ternary linear"}
+
+
 def workload_config(layer):
-    return {"workload": f"FLUX.1-dev double-block image-stream QKV, 1024x1024 image: "
-                        f"x [{layer.M},{layer.K}] bf16, W [{layer.N},{layer.K}] ternary, bias bf16",
+    what = DESCRIPTIONS.get(layer.name, f"FLUX.1-dev adaLN modulation GEMV ({layer.name})")
+    return {"workload": f"{what}: x [{layer.M},{layer.K}] bf16, W [{layer.N},{layer.K}] ternary, bias bf16",
             "M": layer.M, "K": layer.K, "N": layer.N, "eps": 1e-5,
             "step": "tern_quantize_pack(W) + tern_linear(x)",
             "accumulate": "fp32",
@@ -285,22 +293,25 @@ def graph_time(calls, replays, stream):
     (removes host launch overhead from microsecond kernels)."""
     import torch
 
-    for c in calls:  # warm-up outside capture (allocates any workspace)
-        c()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for c in calls:  # warm-up on the capture stream (allocates its workspace)
+            c()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    with torch.cuda.graph(g, stream=stream):
         for c in calls:
             c()
-    g.replay()
+    with torch.cuda.stream(stream):
+        g.replay()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    cur = torch.cuda.current_stream()
-    e0.record(cur)
-    for _ in range(replays):
-        g.replay()
-    e1.record(cur)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(replays):
+            g.replay()
+    e1.record(stream)
     e1.synchronize()
     del g
     return e0.elapsed_time(e1) * 1e-3 / (replays * len(calls))
@@ -376,7 +387,7 @@ def run_tern(args):
     device = torch.device("cuda", local)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
-    layer = workloads.CONFIGS[WORKLOAD]
+    layer = workloads.CONFIGS[args.workload]
     sets = make_sets(layer, rank, 2, device)
     K, Wm = args.steps, max(3, args.warmup)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -449,16 +460,23 @@ def run_tern(args):
     flop = layer.flop
     value = world * K * flop / elapsed / 1e12
     achieved = flop / t_lin / 1e12
-    traffic = profiled_traffic()
+    tensor_bound = flop / (peaks["bf16_tflops"] * 1e12) >= layer.algorithmic_bytes / (peaks["hbm_gbs"] * 1e9)
+    traffic = profiled_traffic(layer.name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, FLUX.1-dev QKV shapes)",
         "config": workload_config(layer),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                     "kernel": "ternary_mma_kernel<128> (tern_linear)",
-                     "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"},
+        "roofline": ({"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                      "kernel": "ternary_mma_kernel (tern_linear)",
+                      "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
+                     if tensor_bound else
+                     {"bound": "hbm", "achieved": layer.algorithmic_bytes / t_lin / 1e9,
+                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": layer.algorithmic_bytes / t_lin / 1e9 / peaks["hbm_gbs"], "traffic": traffic,
+                      "kernel": "ternary_mma_kernel (tern_linear)",
+                      "peak_source": f"{peaks['source']} HBM copy (MEASURED_PEAKS.json)"}),
         "linear_us": t_lin * 1e6, "quantize_pack_us": t_quant * 1e6,
         "packed_weight_gbs": layer.packed_bytes / t_lin / 1e9,
         "quantize_pack_gbs": (2 * layer.N * layer.K + layer.packed_bytes + 4 * layer.N) / t_quant / 1e9,
@@ -470,7 +488,10 @@ def run_tern(args):
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         line["cpu_baseline"] = cpu_baseline(layer, *sets[0]["cpu"], budget_s=args.cpu_seconds)
         if not args.no_extras:
-            line["side_table"] = side_table(device, peaks, stream)
+            try:
+                line["side_table"] = side_table(device, peaks, stream)
+            except Exception as e:  # the side table is context; never lose the main line
+                line["side_table"] = {"error": f"{type(e).__name__}: {e}"}
     if world > 1:
         import torch.distributed as dist
 

@@ -20,7 +20,7 @@ struct alignas(64) Problem {
   int M, N, K;
   int n_tiles, m_tiles, splits;
   int chunks_per_split;     // 64-wide k chunks per split
-  int cta_begin;            // first CTA of this problem in the grid
+  int unit_begin;            // first work unit (CTA, or 2-SM tile) of this problem
 };
 
 constexpr int kMaxProblems = 15;  // keeps the kernel parameter block under 4 KiB
@@ -28,7 +28,7 @@ constexpr int kMaxProblems = 15;  // keeps the kernel parameter block under 4 Ki
 struct Batch {
   Problem p[kMaxProblems];
   int count;
-  int total_ctas;
+  int total_units;
   unsigned long long wait_limit_ns;
   unsigned int* status;     // per-device status word (bounded waits report here)
 };
@@ -71,5 +71,12 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N,
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, unsigned int* status,
                                  cudaStream_t stream);
 int smem_bytes_for_tok(int tok);
+// Large-M kernel on CTA pairs (tcgen05 cta_group::2): 256-channel x
+// 256-token tiles, persistent over the tiles of a batch.  Problems use
+// n_tiles = N / 256, m_tiles = ceil(M / 256), splits = 1 and an x tensor map
+// whose box is 64 k x 128 rows.
+cudaError_t launch_ternary_mma2(const Batch& batch, int clusters, cudaStream_t stream);
+int max_active_clusters_2sm();
+int smem_bytes_2sm();
 
 }  // namespace tern

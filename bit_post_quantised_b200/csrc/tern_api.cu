@@ -51,6 +51,7 @@ struct DeviceState {
   bool checked = false;
   bool supported = false;
   int sms = 0;
+  int clusters_2sm = 0;  // CTA pairs of the 2-SM kernel resident at once
   unsigned int* status = nullptr;
 };
 
@@ -76,6 +77,7 @@ tern_status current_device(int* dev_out, DeviceState** st_out) {
     if (d.supported) {
       e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+      d.clusters_2sm = max_active_clusters_2sm();
     }
     d.checked = true;
   }
@@ -206,7 +208,7 @@ int pick_tok(int64_t M) {
   return 128;
 }
 
-// Fills everything of a Problem except cta_begin; returns its CTA count.
+// Fills everything of a Problem except unit_begin; returns its CTA count.
 tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, Problem* p,
                          int64_t* ctas) {
   std::memset(static_cast<void*>(p), 0, sizeof(Problem));
@@ -229,6 +231,59 @@ tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, 
   p->chunks_per_split = per;
   *ctas = int64_t(p->n_tiles) * p->m_tiles * splits;
   if (*ctas > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "too many tiles");
+  return TERN_OK;
+}
+
+// The 2-SM kernel takes M > 64 when N tiles into 256-channel pairs (every
+// FLUX linear does); it runs whenever the device can co-schedule CTA pairs.
+bool use_2sm(const tern_linear_args& a, const DeviceState* ds) {
+  return a.M > 64 && a.N % 256 == 0 && ds->clusters_2sm > 0;
+}
+
+// Fills a Problem for the 2-SM kernel except unit_begin; returns its tiles.
+tern_status fill_problem_2sm(const tern_linear_args& a, Problem* p, int64_t* tiles) {
+  std::memset(static_cast<void*>(p), 0, sizeof(Problem));
+  tern_status s = make_x_map(&p->tmap_x, a.x, a.M, a.K, 128);
+  if (s != TERN_OK) return s;
+  p->packed = static_cast<const uint8_t*>(a.packed);
+  p->scales = a.scales;
+  p->bias = static_cast<const __nv_bfloat16*>(a.bias);
+  p->y = static_cast<__nv_bfloat16*>(a.y);
+  p->M = int(a.M);
+  p->N = int(a.N);
+  p->K = int(a.K);
+  p->n_tiles = int(a.N / 256);
+  p->m_tiles = int((a.M + 255) / 256);
+  p->splits = 1;
+  p->chunks_per_split = int(a.K / 64);
+  *tiles = int64_t(p->n_tiles) * p->m_tiles;
+  if (*tiles > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "too many tiles");
+  return TERN_OK;
+}
+
+// Launches the problems `idx` of `args` on the 2-SM kernel, up to
+// kMaxProblems per launch.
+tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int>& idx, Batch& batch,
+                             const DeviceState* ds, cudaStream_t cs) {
+  for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
+    std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+    int64_t total = 0;
+    int n = 0;
+    for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
+      int64_t tiles = 0;
+      tern_status s = fill_problem_2sm(args[idx[g]], &batch.p[n], &tiles);
+      if (s != TERN_OK) return s;
+      batch.p[n].unit_begin = int(total);
+      total += tiles;
+      if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
+    }
+    batch.count = n;
+    batch.total_units = int(total);
+    batch.wait_limit_ns = g_wait_limit_ns.load();
+    batch.status = ds->status;
+    cudaError_t e = launch_ternary_mma2(batch, int(std::min<int64_t>(total, ds->clusters_2sm)), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "ternary_mma2 launch");
+  }
   return TERN_OK;
 }
 
@@ -284,6 +339,12 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
   if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
+  if (use_2sm(a, ds)) {
+    static Batch batch2;  // built under the lock below; ~4 KiB, copied into the launch
+    static std::mutex batch2_mu;
+    std::lock_guard<std::mutex> lock(batch2_mu);
+    return launch_2sm_group(&a, std::vector<int>{0}, batch2, ds, cs);
+  }
   const int tok = pick_tok(M);
   int splits = 1;
   const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
@@ -304,9 +365,9 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
     const size_t ws_bytes = size_t(p.splits) * size_t(tiles) * tok * 128 * sizeof(float);
     if ((s = get_workspace(dev, cs, ws_bytes, size_t(tiles), &p.ws, &p.counters)) != TERN_OK) return s;
   }
-  p.cta_begin = 0;
+  p.unit_begin = 0;
   batch.count = 1;
-  batch.total_ctas = int(ctas);
+  batch.total_units = int(ctas);
   batch.wait_limit_ns = g_wait_limit_ns.load();
   batch.status = ds->status;
   cudaError_t e = launch_ternary_mma(tok, batch, cs);
@@ -333,10 +394,16 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
   static Batch batch;
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
+  {
+    std::vector<int> group;
+    for (int i = 0; i < count; ++i)
+      if (args[i].M > 0 && use_2sm(args[i], ds)) group.push_back(i);
+    if ((s = launch_2sm_group(args, group, batch, ds, cs)) != TERN_OK) return s;
+  }
   for (int tok : kTokTiles) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
-      if (args[i].M > 0 && pick_tok(args[i].M) == tok) group.push_back(i);
+      if (args[i].M > 0 && !use_2sm(args[i], ds) && pick_tok(args[i].M) == tok) group.push_back(i);
     for (size_t g0 = 0; g0 < group.size(); g0 += kMaxProblems) {
       std::memset(static_cast<void*>(&batch), 0, sizeof batch);
       int64_t total = 0;
@@ -344,12 +411,12 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
       for (size_t g = g0; g < group.size() && n < kMaxProblems; ++g, ++n) {
         int64_t ctas = 0;
         if ((s = fill_problem(args[group[g]], tok, 1, &batch.p[n], &ctas)) != TERN_OK) return s;
-        batch.p[n].cta_begin = int(total);
+        batch.p[n].unit_begin = int(total);
         total += ctas;
         if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
       }
       batch.count = n;
-      batch.total_ctas = int(total);
+      batch.total_units = int(total);
       batch.wait_limit_ns = g_wait_limit_ns.load();
       batch.status = ds->status;
       cudaError_t e = launch_ternary_mma(tok, batch, cs);

@@ -145,6 +145,15 @@ def test_linear_shapes(M, N, K):
     run_linear_case(M, N, K, seed=N + K + M)
 
 
+@pytest.mark.parametrize("M,N,K", [(65, 256, 64), (129, 512, 320), (255, 256, 128), (256, 512, 192),
+                                   (257, 768, 320), (511, 256, 576), (513, 512, 64), (777, 1280, 448),
+                                   (2048, 2560, 192)])
+def test_linear_pair_tiles(M, N, K):
+    """Large M with N % 256 == 0 runs on CTA pairs (256 x 256 tiles): ragged
+    token tails, single-stage and many-stage K, more tiles than SM pairs."""
+    run_linear_case(M, N, K, seed=M + N + K)
+
+
 def test_linear_no_bias():
     run_linear_case(40, 256, 256, seed=3, with_bias=False)
     run_linear_case(257, 256, 256, seed=4, with_bias=False)
