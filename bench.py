@@ -32,7 +32,7 @@ METRIC = "ternary-linear TFLOP/s & packed-weight GB/s at FLUX shapes; % of roofl
 WORKLOAD = "qkv"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-KERNEL_SOURCE = os.path.join(ROOT, "bit_post_quantised_b200", "csrc", "ternary_mma.cu")
+CSRC = os.path.join(ROOT, "bit_post_quantised_b200", "csrc")
 
 
 def parse_args():
@@ -61,21 +61,29 @@ def load_peaks():
         return {**FALLBACK_PEAKS, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
+def linear_kernel(layer):
+    """(kernel name, source file stem) of the tern_linear launch for this shape:
+    M > 64 with N % 256 == 0 runs on SM pairs, everything else on single SMs."""
+    if layer.M > 64 and layer.N % 256 == 0:
+        return "ternary_mma2_kernel", "ternary_mma2"
+    return "ternary_mma_kernel", "ternary_mma"
+
+
+def kernel_source_hash(stem: str) -> str:
+    with open(os.path.join(CSRC, stem + ".cu"), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(stem: str, workload: str):
     """DRAM bytes per launch of the linear kernel on this workload from the
     committed ncu summary, or None if there is none or the kernel changed since."""
     try:
-        text = open(os.path.join(PROFILE_DIR, f"ternary_mma_{workload}.md")).read()
+        text = open(os.path.join(PROFILE_DIR, f"{stem}_{workload}.md")).read()
     except OSError:
         return None
     m_src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_src or not m_tr or m_src.group(1) != kernel_source_hash():
+    if not m_src or not m_tr or m_src.group(1) != kernel_source_hash(stem):
         return None
     return float(m_tr.group(1))
 
@@ -461,7 +469,8 @@ def run_tern(args):
     value = world * K * flop / elapsed / 1e12
     achieved = flop / t_lin / 1e12
     tensor_bound = flop / (peaks["bf16_tflops"] * 1e12) >= layer.algorithmic_bytes / (peaks["hbm_gbs"] * 1e9)
-    traffic = profiled_traffic(layer.name)
+    kname, kstem = linear_kernel(layer)
+    traffic = profiled_traffic(kstem, layer.name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -469,13 +478,13 @@ def run_tern(args):
         "config": workload_config(layer),
         "roofline": ({"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                       "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                      "kernel": "ternary_mma_kernel (tern_linear)",
+                      "kernel": f"{kname} (tern_linear)",
                       "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
                      if tensor_bound else
                      {"bound": "hbm", "achieved": layer.algorithmic_bytes / t_lin / 1e9,
                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
                       "frac": layer.algorithmic_bytes / t_lin / 1e9 / peaks["hbm_gbs"], "traffic": traffic,
-                      "kernel": "ternary_mma_kernel (tern_linear)",
+                      "kernel": f"{kname} (tern_linear)",
                       "peak_source": f"{peaks['source']} HBM copy (MEASURED_PEAKS.json)"}),
         "linear_us": t_lin * 1e6, "quantize_pack_us": t_quant * 1e6,
         "packed_weight_gbs": layer.packed_bytes / t_lin / 1e9,
