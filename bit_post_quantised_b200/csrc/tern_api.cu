@@ -504,3 +504,98 @@ const char* tern_status_string(tern_status status) {
 const char* tern_last_error(void) { return t_last_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// tern_linear_noalloc: the same ternary linear with its scratch in a fixed
+// device array of this library, for callers that must not allocate device
+// memory (see include/tern.h).  Only the split-K path of small M needs
+// scratch (fp32 partial sums and per-tile arrival counters); here they live
+// in g_noalloc_scratch instead of the per-(device, stream) workspace that
+// tern_linear allocates on first use.
+namespace tern {
+namespace {
+
+constexpr size_t kNoAllocPartialBytes = size_t(10) << 20;  // fp32 split-K partials
+constexpr size_t kNoAllocCounters = 1024;                  // arrival counters (int)
+constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocCounters * sizeof(int);
+
+// One copy per GPU that loads the library, kept until the process exits.
+// Host code must not use this name as a device address: the address comes
+// from cudaGetSymbolAddress below, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+unsigned char* g_noalloc_ptr[kMaxDevices] = {};  // device address of the array, per device
+
+// The device address of g_noalloc_scratch on `dev` (the current device),
+// looked up on the first call for that device.
+tern_status noalloc_scratch(int dev, unsigned char** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return TERN_OK;
+}
+
+}  // namespace
+}  // namespace tern
+
+extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                                           const float* scales, const void* bias_bf16, int64_t N,
+                                           void* y_bf16, tern_stream_t stream) {
+  const tern_linear_args a{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K};
+  tern_status s = check_linear(a);
+  if (s != TERN_OK) return s;
+  if (M == 0) return TERN_OK;
+  int dev;
+  DeviceState* ds;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  unsigned char* scratch = nullptr;
+  if ((s = noalloc_scratch(dev, &scratch)) != TERN_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  static Batch batch;  // built under the lock below, copied into the launch
+  static std::mutex batch_mu;
+  std::lock_guard<std::mutex> lock(batch_mu);
+  if (use_2sm(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, batch, ds, cs);  // no scratch
+
+  // Same tile and split choice as tern_linear, so the two give identical y.
+  const int tok = pick_tok(M);
+  int splits = 1;
+  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  if (tok <= 64) {
+    const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
+    if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
+    splits = std::max(1, std::min(splits, 16));
+  }
+  std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+  int64_t ctas = 0;
+  if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;
+  Problem& p = batch.p[0];
+  if (p.splits > 1) {
+    const size_t need = size_t(p.splits) * size_t(tiles) * tok * 128 * sizeof(float);
+    if (need > kNoAllocPartialBytes || size_t(tiles) > kNoAllocCounters)
+      return fail(TERN_ERR_UNSUPPORTED_SHAPE,
+                  "M=%lld N=%lld K=%lld needs %zu bytes of split-K partials and %lld counters; the "
+                  "static scratch holds %zu bytes and %zu counters",
+                  (long long)M, (long long)N, (long long)K, need, (long long)tiles, kNoAllocPartialBytes,
+                  kNoAllocCounters);
+    p.ws = reinterpret_cast<float*>(scratch);
+    p.counters = reinterpret_cast<int*>(scratch + kNoAllocPartialBytes);
+    // The array keeps whatever the previous call (or a timed-out one) left:
+    // the arrival counters must start at zero.
+    cudaError_t e = cudaMemsetAsync(p.counters, 0, size_t(tiles) * sizeof(int), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "no-alloc counter clear");
+  }
+  p.unit_begin = 0;
+  batch.count = 1;
+  batch.total_units = int(ctas);
+  batch.wait_limit_ns = g_wait_limit_ns.load();
+  batch.status = ds->status;
+  cudaError_t e = launch_ternary_mma(tok, batch, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "ternary_mma launch (no-alloc)");
+  return TERN_OK;
+}

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
                 -3: "TERN_ERR_MISALIGNED", -4: "TERN_ERR_CUDA", -5: "TERN_ERR_TIMEOUT",
                 -6: "TERN_ERR_NO_DEVICE"}
 
-EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_batch",
+EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
+            "tern_linear_batch",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.tern_quantize_pack.restype = st
         L.tern_linear.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
         L.tern_linear.restype = st
+        L.tern_linear_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
+        L.tern_linear_noalloc.restype = st
         L.tern_linear_batch.argtypes = [ctypes.POINTER(LinearArgs), ctypes.c_int, vp]
         L.tern_linear_batch.restype = st
         L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
@@ -117,6 +120,21 @@ def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     _check(lib().tern_linear(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
                              _stream(stream)))
+    return out
+
+
+def linear_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                   bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   stream=None):
+    """tern_linear_noalloc: tern_linear with its split-K scratch in the library's
+    static device array (no device allocation by the library; `out` must be
+    given by callers that cannot allocate)."""
+    M, K = x.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().tern_linear_noalloc(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N,
+                                     _ptr(out), _stream(stream)))
     return out
 
 

@@ -105,6 +105,34 @@ TERN_API tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const
                         const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
                         tern_stream_t stream);
 
+/*
+ * tern_linear without any device allocation, for callers that cannot call
+ * cudaMalloc: code that runs while a CUDA graph is being captured in global
+ * mode, engines that own all device memory in a preplanned arena or a
+ * memory budget, and latency-critical loops where an allocation (which may
+ * synchronise the device) is not allowed.  The paper has no counterpart: this
+ * is an interface choice of this library.
+ *   Arguments, layouts and results are those of tern_linear, and the tile and
+ *   split choice is the same, so y matches tern_linear's bit for bit.
+ *   Scratch: the small-M path (M <= 64) splits K across CTAs and keeps its
+ *   fp32 partial sums and per-tile counters in one static device array of
+ *   10 MiB + 4 KiB inside this library (held on every GPU that loads the
+ *   library until the process exits).  That covers every shape on a 148-SM
+ *   B200; a shape that would need more returns TERN_ERR_UNSUPPORTED_SHAPE
+ *   with the sizes in tern_last_error().  M > 64 needs no scratch.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents (the counters are cleared on the stream before each
+ *   launch).  Calls whose kernels may overlap on the GPU -- on different
+ *   streams, or from different host threads -- race on it: order them on one
+ *   stream, or use tern_linear.
+ */
+TERN_API tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                                const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                                tern_stream_t stream);
+
 /* One independent linear problem of a batch (same meaning as tern_linear). */
 typedef struct {
   const void* x;      /* [M, K] bf16 */
