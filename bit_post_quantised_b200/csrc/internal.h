@@ -34,7 +34,7 @@ struct Batch {
 };
 
 // Token-tile sizes (UMMA N) with a compiled kernel.
-constexpr int kTokTiles[] = {16, 32, 64, 128};
+constexpr int kTokTiles[] = {32, 64, 128};
 
 // Per-tile geometry, shared by host (launch) and device (kernel).
 template <int TOK>
@@ -76,6 +76,11 @@ int smem_bytes_for_tok(int tok);
 // n_tiles = N / 256, m_tiles = ceil(M / 256), splits = 1 and an x tensor map
 // whose box is 64 k x 128 rows.
 cudaError_t launch_ternary_mma2(const Batch& batch, int clusters, cudaStream_t stream);
+// Small-M kernel (M <= 8 nt tokens, nt in {1, 2}): grid (splits, slabs) with
+// clusters of `splits` CTAs along k; problems use n_tiles = N / 128 slabs,
+// unit_begin = first slab in the launch, chunks_per_split 64-k chunks per CTA
+// and a 3-D x tensor map {64 k, M, K / 64} whose box is {64, min(M, 8 nt), 8}.
+cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int slabs, cudaStream_t stream);
 int max_active_clusters_2sm();
 int smem_bytes_2sm();
 

@@ -122,6 +122,23 @@ tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, in
   return TERN_OK;
 }
 
+// x [M, K] bf16 row-major viewed as 3-D {64 k, M tokens, K / 64 chunks} for
+// the GEMV kernel: box {64, rows, 8} lands as [chunk][token][64 k] with
+// 128-byte swizzle; chunks past K read as zero.
+tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_t K, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {64, cuuint64_t(M), cuuint64_t(K / 64)};
+  const cuuint64_t strides[2] = {cuuint64_t(K) * 2, 128};
+  const cuuint32_t box[3] = {64, cuuint32_t(rows), 8};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled (3-D x) failed (%d)", int(r));
+  return TERN_OK;
+}
+
 // ------------------------------------------------------------ workspace
 struct Workspace {
   float* ws = nullptr;
@@ -201,8 +218,12 @@ tern_status check_linear(const tern_linear_args& a) {
   return TERN_OK;
 }
 
+// Up to 16 tokens run on the register-fed GEMV kernel, in n8 blocks.
+constexpr int64_t kGemvMaxM = 16;
+int gemv_nt(int64_t M) { return M <= 8 ? 1 : 2; }
+
+// Token tile of the single-SM tcgen05 kernel for 16 < M (or N % 256 != 0).
 int pick_tok(int64_t M) {
-  if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   return 128;
@@ -287,6 +308,50 @@ tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int
   return TERN_OK;
 }
 
+// Launches the problems `idx` of `args` (all with M <= 8 nt) on the GEMV
+// kernel, up to kMaxProblems per launch.  K is split over a cluster of up to
+// eight CTAs when the launch has fewer 128-channel slabs than the GPU has SMs.
+tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<int>& idx, int nt, Batch& batch,
+                              const DeviceState* ds, cudaStream_t cs) {
+  for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
+    std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+    int64_t slabs = 0;
+    int64_t min_chunks = int64_t(1) << 40;
+    int n = 0;
+    for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
+      const tern_linear_args& a = args[idx[g]];
+      Problem* p = &batch.p[n];
+      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, int(std::min<int64_t>(a.M, 8 * nt)));
+      if (s != TERN_OK) return s;
+      p->packed = static_cast<const uint8_t*>(a.packed);
+      p->scales = a.scales;
+      p->bias = static_cast<const __nv_bfloat16*>(a.bias);
+      p->y = static_cast<__nv_bfloat16*>(a.y);
+      p->M = int(a.M);
+      p->N = int(a.N);
+      p->K = int(a.K);
+      p->n_tiles = int(a.N / 128);
+      p->m_tiles = 1;
+      p->unit_begin = int(slabs);
+      slabs += a.N / 128;
+      min_chunks = std::min<int64_t>(min_chunks, a.K / 64);
+    }
+    if (slabs > 65535) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "more than 65535 slabs of 128 channels in one launch");
+    const int splits = int(std::max<int64_t>(1, std::min<int64_t>({8, ds->sms / slabs, min_chunks})));
+    for (int i = 0; i < n; ++i) {
+      batch.p[i].splits = splits;
+      batch.p[i].chunks_per_split = (batch.p[i].K / 64 + splits - 1) / splits;
+    }
+    batch.count = n;
+    batch.total_units = int(slabs);
+    batch.wait_limit_ns = g_wait_limit_ns.load();
+    batch.status = ds->status;
+    cudaError_t e = launch_ternary_gemv(nt, batch, splits, int(slabs), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "ternary_gemv launch");
+  }
+  return TERN_OK;
+}
+
 int ctas_per_sm(int tok) {
   const int smem = smem_bytes_for_tok(tok);
   const int by_smem = (228 * 1024) / (smem + 1024);
@@ -339,6 +404,12 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
   if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
+  if (M <= kGemvMaxM) {
+    static Batch batch_g;  // built under the lock below; ~4 KiB, copied into the launch
+    static std::mutex batch_g_mu;
+    std::lock_guard<std::mutex> lock(batch_g_mu);
+    return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
+  }
   if (use_2sm(a, ds)) {
     static Batch batch2;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch2_mu;
@@ -394,16 +465,22 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
   static Batch batch;
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
+  for (int nt : {1, 2}) {
+    std::vector<int> group;
+    for (int i = 0; i < count; ++i)
+      if (args[i].M > 0 && args[i].M <= kGemvMaxM && gemv_nt(args[i].M) == nt) group.push_back(i);
+    if ((s = launch_gemv_group(args, group, nt, batch, ds, cs)) != TERN_OK) return s;
+  }
   {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
-      if (args[i].M > 0 && use_2sm(args[i], ds)) group.push_back(i);
+      if (args[i].M > kGemvMaxM && use_2sm(args[i], ds)) group.push_back(i);
     if ((s = launch_2sm_group(args, group, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int tok : kTokTiles) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
-      if (args[i].M > 0 && !use_2sm(args[i], ds) && pick_tok(args[i].M) == tok) group.push_back(i);
+      if (args[i].M > kGemvMaxM && !use_2sm(args[i], ds) && pick_tok(args[i].M) == tok) group.push_back(i);
     for (size_t g0 = 0; g0 < group.size(); g0 += kMaxProblems) {
       std::memset(static_cast<void*>(&batch), 0, sizeof batch);
       int64_t total = 0;
@@ -560,7 +637,9 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
   static Batch batch;  // built under the lock below, copied into the launch
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
-  if (use_2sm(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, batch, ds, cs);  // no scratch
+  // Neither the small-M GEMV nor the pair-tile kernel needs scratch.
+  if (M <= kGemvMaxM) return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch, ds, cs);
+  if (use_2sm(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, batch, ds, cs);
 
   // Same tile and split choice as tern_linear, so the two give identical y.
   const int tok = pick_tok(M);

@@ -1,0 +1,325 @@
+// ternary_gemv.cu -- the small-M (M <= 16) ternary linear y = (x . T^T) * s + b,
+// bound by the HBM stream of packed codes.
+//
+// Page "1.58-bit FLUX" (arXiv 2412.18653): Section 1 (weights in {-1,0,+1},
+// stored as 2-bit signed integers), Section 4 (activations stay 16-bit); the
+// adaLN modulation layers of every block are such products with one token
+// row per image.
+//
+// With a handful of tokens every code byte is used by at most 16 multiply-
+// adds, so the kernel's job is to stream the N*K/4 code bytes at HBM speed and
+// spend as few instructions per weight as possible.  The tensor cores of
+// tcgen05 read their operands as bf16 from shared memory or TMEM, which caps
+// them at about 64 weights per SM clock -- below the ~90 weights per clock
+// that HBM delivers as 2-bit codes.  So this kernel expands codes in
+// registers and feeds the warp-level tensor-core instruction (mma.sync
+// m16n8k16, bf16 in, fp32 accumulate), whose A operand comes from registers:
+//   * A = 16 channels x 16 k of weights.  A code (two's complement: +1 = 01,
+//     -1 = 11, 0 = 00) shifted so that its two bits land on bits 14 and 15 of
+//     a bf16 is the bf16 value 2t exactly (0x4000 = 2, 0xC000 = -2, 0 = 0),
+//     so one shift and one AND expand a (k, k+1) pair; the sum is halved at
+//     the end (exact).
+//   * The k order inside each 64-k chunk is permuted so that the lane that
+//     loads code word c of a row (one 32-bit shared-memory load, the 32 lanes
+//     of a warp reading 128 contiguous bytes) holds exactly its A-fragment
+//     pairs: MMA q (q = 0..3) of the chunk takes pairs 2q and 2q+1 of every
+//     word, i.e. k = 16c + 4q .. 16c + 4q + 3 for the lane with c = lane % 4,
+//     and B = x is read in the same permuted order (8 contiguous bytes).
+//   * B = x^T for 8 tokens per n8 block (NT blocks: M <= 8 NT).
+// One CTA owns 128 channels (one tile-interleaved slab: each 64-k chunk is a
+// contiguous 2 KiB block) over a range of k.  Its sixteen consumer warps own
+// 16 channels each, two warps per channel group splitting every stage's
+// chunks (even / odd).  A producer lane streams stages of eight chunks into a
+// six-stage ring with two copies per stage: one 16 KiB bulk copy of codes and
+// one 3-D TMA box of the matching x rows (k-in-chunk x token x chunk, 128-byte
+// swizzle; only min(M, 8 NT) token rows are fetched -- the MMA columns of
+// absent tokens read stale shared memory and are never stored).  When there
+// are too few slabs to fill the SMs, the k range is split over a cluster of
+// CTAs, whose partial sums are added in rank order through distributed shared
+// memory (deterministic, no global scratch).  No TMA multicast is used.
+#include "internal.h"
+#include "kernel_common.cuh"
+#include "ptx.cuh"
+
+namespace tern {
+
+namespace {
+
+template <int NT>
+struct GemvCfg {
+  static constexpr int kGroups = 8;                  // 16-channel groups per 128-channel slab
+  static constexpr int kWarps = 2 * kGroups;         // consumer warps: two per group
+  static constexpr int kThreads = (kWarps + 1) * 32;  // + one producer warp
+  static constexpr int kChunks = 8;                  // 64-k chunks per stage
+  static constexpr int kStages = 6;
+  static constexpr int kCodeBytes = kChunks * 2048;
+  static constexpr int kXBytes = kChunks * 8 * NT * 128;  // up to 8 NT token rows x 64 bf16 per chunk
+  static constexpr int kStageBytes = kCodeBytes + kXBytes + 1024;  // + slack: rows >= R read past the box
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static_assert(kStageBytes % 1024 == 0 && kCodeBytes % 1024 == 0, "swizzled x boxes stay 1024-aligned");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+// bf16x2 of 2t for the code pair j (k and k + 1) of a code word.
+template <int J>
+__device__ __forceinline__ uint32_t pm2_pair(uint32_t w) {
+  return (w << (14 - 2 * J)) & 0xC000C000u;
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace
+
+// Grid (splits, total slabs), cluster (splits, 1, 1): blockIdx.y picks the
+// problem and its 128-channel slab, blockIdx.x (the rank in the cluster) the
+// k range (chunks_per_split 64-k chunks).  The x tensor map is 3-D
+// {64 k, M tokens, K / 64 chunks} with box {64, min(M, 8 NT), 8}.
+template <int NT>
+__global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
+    ternary_gemv_kernel(const __grid_constant__ Batch batch) {
+  using C = GemvCfg<NT>;
+  constexpr int S = C::kStages;
+  constexpr int kConsumerThreads = C::kWarps * 32;
+
+  __shared__ __align__(8) uint64_t full_bar[S];   // codes and x of stage s landed
+  __shared__ __align__(8) uint64_t empty_bar[S];  // all consumer warps are done with stage s
+  __shared__ __align__(16) float part[C::kGroups * 32 * NT * 4];  // odd-chunk warps' sums, then the CTA's
+  extern __shared__ uint8_t dyn_smem[];
+
+  const uint64_t lim = batch.wait_limit_ns;
+  unsigned int* const st = batch.status;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const uint8_t* const smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
+
+  const int unit = blockIdx.y;
+  int pi = 0;
+  while (pi + 1 < batch.count && unit >= batch.p[pi + 1].unit_begin) ++pi;
+  const Problem& P = batch.p[pi];
+  const int slab = unit - P.unit_begin;
+  const int splits = gridDim.x, rank = blockIdx.x;
+  const int kc_total = P.K >> 6;
+  const int kc0 = rank * P.chunks_per_split;
+  const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
+  const int nstages = (nk + C::kChunks - 1) / C::kChunks;
+  const int rows = min(P.M, 8 * NT);  // token rows the x box fetches
+  const uint8_t* codes = P.packed + (size_t(slab) * kc_total + kc0) * 2048;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), C::kWarps);
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+
+  float d[NT][4];  // D fragments: channels (g, g + 8) x tokens (2c, 2c + 1) of each n8 block
+#pragma unroll
+  for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d[nb][e] = 0.f;
+  const int grp = warp & (C::kGroups - 1), half = warp / C::kGroups;
+  // Scale and bias of this lane's two output channels, fetched before the
+  // stream starts so their latency is hidden (only rank 0's first warps store).
+  const int n_out = slab * 128 + grp * 16 + (lane >> 2);
+  float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
+  if (warp < C::kGroups && rank == 0) {
+    s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
+    s1 = 0.5f * P.scales[n_out + 8];
+    const uint16_t* bias = reinterpret_cast<const uint16_t*>(P.bias);
+    if (bias) {
+      b0 = bf16_bits_to_float(bias[n_out]);
+      b1 = bf16_bits_to_float(bias[n_out + 8]);
+    }
+  }
+
+  if (warp == C::kWarps) {
+    // ------------------------------------------------------ producer
+    if (lane == 0) prefetch_tensormap(&P.tmap_x);
+    int issued = 0;
+    for (int i = 0; i < nstages; ++i) {
+      const int s = i % S;
+      if (i >= S &&
+          !__shfl_sync(0xffffffffu, mbar_wait(smem_u32(&empty_bar[s]), ((i / S) & 1) ^ 1, lim, st), 0))
+        break;
+      if (lane == 0) {
+        const int nch = min(C::kChunks, nk - i * C::kChunks);
+        const uint32_t stage = smem_base + s * C::kStageBytes;
+        const uint32_t fb = smem_u32(&full_bar[s]);
+        mbar_arrive_expect_tx(fb, nch * 2048 + C::kChunks * rows * 128);
+        tma_load_bulk(stage, codes + size_t(i) * C::kCodeBytes, nch * 2048, fb);
+        tma_load_3d(stage + C::kCodeBytes, &P.tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
+      }
+      __syncwarp();
+      issued = i + 1;
+    }
+    // No copy may still be landing in shared memory when the CTA exits.
+    for (int i = max(0, issued - S); i < issued; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
+  } else {
+    // ------------------------------------------------------ consumers
+    const int g = lane >> 2, c = lane & 3;
+    // Shared-memory offsets of this lane's two 16-byte x pieces in each of
+    // its chunks (line j * rows + g of the stage's x box, XOR-swizzled by
+    // the line index; the second n8 block is 8 lines = 1 KiB further).
+    uint32_t xoff_a[C::kChunks / 2], xoff_b[C::kChunks / 2];
+#pragma unroll
+    for (int t = 0; t < C::kChunks / 2; ++t) {
+      const uint32_t line = uint32_t((half + 2 * t) * rows + g);
+      xoff_a[t] = line * 128 + ((uint32_t(2 * c) ^ (line & 7)) << 4);
+      xoff_b[t] = line * 128 + ((uint32_t(2 * c + 1) ^ (line & 7)) << 4);
+    }
+    float acc[4][NT][4];  // one accumulator per MMA position q: four independent chains
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[q][nb][e] = 0.f;
+    for (int i = 0; i < nstages; ++i) {
+      const int s = i % S;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (i / S) & 1, lim, st))) break;
+      const int nch = min(C::kChunks, nk - i * C::kChunks);
+      const uint8_t* stage = smem_gen + s * C::kStageBytes;
+      const uint32_t xstage = smem_base + s * C::kStageBytes + C::kCodeBytes;
+      // Code words first (word c of rows 16 grp + g and 16 grp + g + 8 of
+      // chunks half, half + 2, ...), for all of this warp's chunks at once.
+      uint32_t w0[C::kChunks / 2], w1[C::kChunks / 2];
+#pragma unroll
+      for (int t = 0; t < C::kChunks / 2; ++t) {
+        const int j = half + 2 * t;
+        if (j < nch) {
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + j * 2048) + grp * 64 + lane;
+          w0[t] = cw[0];
+          w1[t] = cw[32];
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < C::kChunks / 2; ++t) {
+        const int j = half + 2 * t;
+        if (j < nch) {
+#pragma unroll
+          for (int nb = 0; nb < NT; ++nb) {
+            // x row 8 nb + g of chunk j, k = 16c .. 16c + 15: 16-byte pieces
+            // 2c and 2c + 1 of its 128-byte line, XOR-swizzled by line index.
+            const uint4 xa = ld_shared_v4(xstage + xoff_a[t] + nb * 1024);
+            const uint4 xb = ld_shared_v4(xstage + xoff_b[t] + nb * 1024);
+            const uint32_t a = w0[t], b = w1[t];
+            mma_16816(acc[0][nb], pm2_pair<0>(a), pm2_pair<0>(b), pm2_pair<1>(a), pm2_pair<1>(b), xa.x, xa.y);
+            mma_16816(acc[1][nb], pm2_pair<2>(a), pm2_pair<2>(b), pm2_pair<3>(a), pm2_pair<3>(b), xa.z, xa.w);
+            mma_16816(acc[2][nb], pm2_pair<4>(a), pm2_pair<4>(b), pm2_pair<5>(a), pm2_pair<5>(b), xb.x, xb.y);
+            mma_16816(acc[3][nb], pm2_pair<6>(a), pm2_pair<6>(b), pm2_pair<7>(a), pm2_pair<7>(b), xb.z, xb.w);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
+    }
+#pragma unroll
+    for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        d[nb][e] = (acc[0][nb][e] + acc[1][nb][e]) + (acc[2][nb][e] + acc[3][nb][e]);
+    // Even-chunk warps add the odd-chunk warps' sums (fixed order).
+    float* mine = &part[(grp * 32 + lane) * NT * 4];
+    if (half == 1) {
+#pragma unroll
+      for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = d[nb][e];
+    }
+    named_barrier_sync(1, kConsumerThreads);
+    if (half == 0) {
+#pragma unroll
+      for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          d[nb][e] += mine[nb * 4 + e];
+          if (splits > 1) mine[nb * 4 + e] = d[nb][e];  // this CTA's total, for rank 0
+        }
+    }
+  }
+
+  // ------------------------------------------------------ reduce and store
+  if (splits > 1) cluster_sync();  // every rank's partial sums are in its shared memory
+  if (warp < C::kGroups && rank == 0) {
+    if (splits > 1) {
+      const uint32_t mine = smem_u32(&part[(warp * 32 + lane) * NT * 4]);
+      for (int r = 1; r < splits; ++r)  // rank order: deterministic
+#pragma unroll
+        for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d[nb][e] += ld_shared_cluster_f32(mapa_shared(mine + uint32_t(nb * 4 + e) * 4, uint32_t(r)));
+    }
+    const int c = lane & 3;
+    const int n = n_out;
+#pragma unroll
+    for (int nb = 0; nb < NT; ++nb) {
+      const int t0 = 8 * nb + 2 * c;
+      if (t0 < P.M) {
+        P.y[size_t(t0) * P.N + n] = __float2bfloat16_rn(fmaf(d[nb][0], s0, b0));
+        P.y[size_t(t0) * P.N + n + 8] = __float2bfloat16_rn(fmaf(d[nb][2], s1, b1));
+      }
+      if (t0 + 1 < P.M) {
+        P.y[size_t(t0 + 1) * P.N + n] = __float2bfloat16_rn(fmaf(d[nb][1], s0, b0));
+        P.y[size_t(t0 + 1) * P.N + n + 8] = __float2bfloat16_rn(fmaf(d[nb][3], s1, b1));
+      }
+    }
+  }
+  if (splits > 1) cluster_sync_relaxed();  // rank 0 has read every partial before any CTA exits
+}
+
+template <int NT>
+static cudaError_t launch_nt(const Batch& batch, int splits, int slabs, cudaStream_t stream) {
+  using C = GemvCfg<NT>;
+  static unsigned long long configured = 0;  // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & (1ull << dev))) {
+    e = cudaFuncSetAttribute(ternary_gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(splits), unsigned(slabs), 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<NT>, batch);
+}
+
+cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int slabs, cudaStream_t stream) {
+  if (splits < 1 || splits > 8 || slabs < 1 || slabs > 65535) return cudaErrorInvalidValue;
+  switch (nt) {
+    case 1: return launch_nt<1>(batch, splits, slabs, stream);
+    case 2: return launch_nt<2>(batch, splits, slabs, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tern

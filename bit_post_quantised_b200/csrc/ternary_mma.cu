@@ -255,7 +255,6 @@ static cudaError_t launch_tok(const Batch& batch, cudaStream_t stream) {
 
 int smem_bytes_for_tok(int tok) {
   switch (tok) {
-    case 16: return TileCfg<16>::kSmemBytes;
     case 32: return TileCfg<32>::kSmemBytes;
     case 64: return TileCfg<64>::kSmemBytes;
     case 128: return TileCfg<128>::kSmemBytes;
@@ -265,7 +264,6 @@ int smem_bytes_for_tok(int tok) {
 
 cudaError_t launch_ternary_mma(int tok, const Batch& batch, cudaStream_t stream) {
   switch (tok) {
-    case 16: return launch_tok<16>(batch, stream);
     case 32: return launch_tok<32>(batch, stream);
     case 64: return launch_tok<64>(batch, stream);
     case 128: return launch_tok<128>(batch, stream);

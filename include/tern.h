@@ -96,10 +96,11 @@ TERN_API tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K
  *   bias    [N] bf16, or NULL for no bias.
  *   y_bf16  [M, N] bf16 output, overwritten (round to nearest even).
  * Products are exact (T is +-1/0), sums are fp32, then y = fp32 sum * s + b.
- * Small M (<= 64) splits K across CTAs and uses a library-owned fp32
- * workspace per (device, stream), allocated on the first such call; make that
- * first call outside CUDA stream capture.  Calls on the same stream are
- * ordered; calls on different streams use different workspaces.
+ * M <= 16 runs on a register-fed GEMV kernel that needs no scratch.
+ * 16 < M <= 64 splits K across CTAs and uses a library-owned fp32 workspace
+ * per (device, stream), allocated on the first such call; make that first
+ * call outside CUDA stream capture.  Calls on the same stream are ordered;
+ * calls on different streams use different workspaces.
  */
 TERN_API tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
                         const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
@@ -114,12 +115,12 @@ TERN_API tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const
  * is an interface choice of this library.
  *   Arguments, layouts and results are those of tern_linear, and the tile and
  *   split choice is the same, so y matches tern_linear's bit for bit.
- *   Scratch: the small-M path (M <= 64) splits K across CTAs and keeps its
+ *   Scratch: the path for 16 < M <= 64 splits K across CTAs and keeps its
  *   fp32 partial sums and per-tile counters in one static device array of
  *   10 MiB + 4 KiB inside this library (held on every GPU that loads the
  *   library until the process exits).  That covers every shape on a 148-SM
  *   B200; a shape that would need more returns TERN_ERR_UNSUPPORTED_SHAPE
- *   with the sizes in tern_last_error().  M > 64 needs no scratch.
+ *   with the sizes in tern_last_error().  Other M need no scratch.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
@@ -146,10 +147,11 @@ typedef struct {
 /*
  * Several independent ternary linears (for instance the per-stream adaLN
  * modulation GEMVs and projections of one FLUX block) with as few launches as
- * possible: problems with similar M share one grouped launch.  `args` is host
- * memory, read before the call returns.  Every problem is validated before
- * anything is launched; on an error nothing runs.  count == 0 is a no-op.
- * Batched problems do not split K, so they need no workspace.
+ * possible: problems with similar M share one grouped launch (M <= 8, M <= 16,
+ * then the tcgen05 kernels).  `args` is host memory, read before the call
+ * returns.  Every problem is validated before anything is launched; on an
+ * error nothing runs.  count == 0 is a no-op.  Batched problems need no
+ * workspace (only the single-call path for 16 < M <= 64 splits K into one).
  */
 TERN_API tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream);
 
