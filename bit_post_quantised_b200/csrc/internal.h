@@ -71,11 +71,14 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N,
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, unsigned int* status,
                                  cudaStream_t stream);
 int smem_bytes_for_tok(int tok);
-// Large-M kernel on CTA pairs (tcgen05 cta_group::2): 256-channel x
-// 256-token tiles, persistent over the tiles of a batch.  Problems use
-// n_tiles = N / 256, m_tiles = ceil(M / 256), splits = 1 and an x tensor map
-// whose box is 64 k x 128 rows.
-cudaError_t launch_ternary_mma2(const Batch& batch, int clusters, cudaStream_t stream);
+// Persistent tcgen05 tile kernel: tok-token tiles of 256 channels on CTA pairs
+// (pair, cta_group::2; tok 256 for M > 64) or of 128 channels on single CTAs
+// (!pair; tok 64 for 16 < M <= 64).  Problems use n_tiles = N / (256 or 128),
+// m_tiles = ceil(M / tok), splits = 1 and a 3-D x tensor map {64 k, M,
+// K / 64} whose box is {64, tok / 2 or tok rows, 2 chunks}; ctas_or_pairs
+// work units run at once.
+cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream);
+int max_active_clusters_2sm();
 // Small-M kernel (M <= 8 nt tokens, nt in {1, 2}): grid (splits, slabs) with
 // clusters of `splits` CTAs along k; problems use n_tiles = N / 128 slabs,
 // unit_begin = first slab in the launch, chunks_per_split 64-k chunks per CTA

@@ -122,15 +122,16 @@ tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, in
   return TERN_OK;
 }
 
-// x [M, K] bf16 row-major viewed as 3-D {64 k, M tokens, K / 64 chunks} for
-// the GEMV kernel: box {64, rows, 8} lands as [chunk][token][64 k] with
-// 128-byte swizzle; chunks past K read as zero.
-tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_t K, int rows) {
+// x [M, K] bf16 row-major viewed as 3-D {64 k, M tokens, K / 64 chunks}: box
+// {64, rows, chunks} lands as [chunk][token][64 k] with 128-byte swizzle, so
+// one copy brings several 64-k chunks; tokens past M and chunks past K read
+// as zero.
+tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_t K, int rows, int chunks) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[3] = {64, cuuint64_t(M), cuuint64_t(K / 64)};
   const cuuint64_t strides[2] = {cuuint64_t(K) * 2, 128};
-  const cuuint32_t box[3] = {64, cuuint32_t(rows), 8};
+  const cuuint32_t box[3] = {64, cuuint32_t(rows), cuuint32_t(chunks)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -255,16 +256,23 @@ tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, 
   return TERN_OK;
 }
 
-// The 2-SM kernel takes M > 64 when N tiles into 256-channel pairs (every
-// FLUX linear does); it runs whenever the device can co-schedule CTA pairs.
-bool use_2sm(const tern_linear_args& a, const DeviceState* ds) {
-  return a.M > 64 && a.N % 256 == 0 && ds->clusters_2sm > 0;
+// Token tile of the persistent tcgen05 tile kernel for this problem, or 0
+// when it does not apply: N must tile into 256-channel pairs (every FLUX
+// linear does), and M <= 16 goes to the GEMV kernel.  M > 64 runs 256-token
+// tiles on CTA pairs (needs the device to co-schedule pairs), 16 < M <= 64
+// 64-token tiles on single CTAs.
+int pair_tok(const tern_linear_args& a, const DeviceState* ds) {
+  if (a.N % 256 != 0 || a.M <= 16) return 0;
+  if (a.M <= 64) return 64;
+  return ds->clusters_2sm > 0 ? 256 : 0;
 }
+bool tok_is_pair(int tok) { return tok == 256; }
 
-// Fills a Problem for the 2-SM kernel except unit_begin; returns its tiles.
-tern_status fill_problem_2sm(const tern_linear_args& a, Problem* p, int64_t* tiles) {
+// Fills a Problem for the pair-tile kernel except unit_begin; returns its tiles.
+tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int64_t* tiles) {
   std::memset(static_cast<void*>(p), 0, sizeof(Problem));
-  tern_status s = make_x_map(&p->tmap_x, a.x, a.M, a.K, 128);
+  const bool pair = tok_is_pair(tok);
+  tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, pair ? tok / 2 : tok, 2);
   if (s != TERN_OK) return s;
   p->packed = static_cast<const uint8_t*>(a.packed);
   p->scales = a.scales;
@@ -273,8 +281,8 @@ tern_status fill_problem_2sm(const tern_linear_args& a, Problem* p, int64_t* til
   p->M = int(a.M);
   p->N = int(a.N);
   p->K = int(a.K);
-  p->n_tiles = int(a.N / 256);
-  p->m_tiles = int((a.M + 255) / 256);
+  p->n_tiles = int(a.N / (pair ? 256 : 128));
+  p->m_tiles = int((a.M + tok - 1) / tok);
   p->splits = 1;
   p->chunks_per_split = int(a.K / 64);
   *tiles = int64_t(p->n_tiles) * p->m_tiles;
@@ -282,9 +290,9 @@ tern_status fill_problem_2sm(const tern_linear_args& a, Problem* p, int64_t* til
   return TERN_OK;
 }
 
-// Launches the problems `idx` of `args` on the 2-SM kernel, up to
-// kMaxProblems per launch.
-tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int>& idx, Batch& batch,
+// Launches the problems `idx` of `args` (all with pair_tok == tok) on the
+// pair-tile kernel, up to kMaxProblems per launch.
+tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int>& idx, int tok, Batch& batch,
                              const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
@@ -292,7 +300,7 @@ tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int
     int n = 0;
     for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
       int64_t tiles = 0;
-      tern_status s = fill_problem_2sm(args[idx[g]], &batch.p[n], &tiles);
+      tern_status s = fill_problem_2sm(args[idx[g]], tok, &batch.p[n], &tiles);
       if (s != TERN_OK) return s;
       batch.p[n].unit_begin = int(total);
       total += tiles;
@@ -302,7 +310,9 @@ tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int
     batch.total_units = int(total);
     batch.wait_limit_ns = g_wait_limit_ns.load();
     batch.status = ds->status;
-    cudaError_t e = launch_ternary_mma2(batch, int(std::min<int64_t>(total, ds->clusters_2sm)), cs);
+    const bool pair = tok_is_pair(tok);
+    const int64_t resident = pair ? ds->clusters_2sm : ds->sms;
+    cudaError_t e = launch_ternary_mma2(tok, pair, batch, int(std::min<int64_t>(total, resident)), cs);
     if (e != cudaSuccess) return cuda_fail(e, "ternary_mma2 launch");
   }
   return TERN_OK;
@@ -321,7 +331,7 @@ tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<in
     for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
       const tern_linear_args& a = args[idx[g]];
       Problem* p = &batch.p[n];
-      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, int(std::min<int64_t>(a.M, 8 * nt)));
+      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, int(std::min<int64_t>(a.M, 8 * nt)), 8);
       if (s != TERN_OK) return s;
       p->packed = static_cast<const uint8_t*>(a.packed);
       p->scales = a.scales;
@@ -410,11 +420,11 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
     std::lock_guard<std::mutex> lock(batch_g_mu);
     return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
   }
-  if (use_2sm(a, ds)) {
+  if (const int ptok = pair_tok(a, ds)) {
     static Batch batch2;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch2_mu;
     std::lock_guard<std::mutex> lock(batch2_mu);
-    return launch_2sm_group(&a, std::vector<int>{0}, batch2, ds, cs);
+    return launch_2sm_group(&a, std::vector<int>{0}, ptok, batch2, ds, cs);
   }
   const int tok = pick_tok(M);
   int splits = 1;
@@ -471,16 +481,16 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
       if (args[i].M > 0 && args[i].M <= kGemvMaxM && gemv_nt(args[i].M) == nt) group.push_back(i);
     if ((s = launch_gemv_group(args, group, nt, batch, ds, cs)) != TERN_OK) return s;
   }
-  {
+  for (int ptok : {64, 256}) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
-      if (args[i].M > kGemvMaxM && use_2sm(args[i], ds)) group.push_back(i);
-    if ((s = launch_2sm_group(args, group, batch, ds, cs)) != TERN_OK) return s;
+      if (args[i].M > 0 && pair_tok(args[i], ds) == ptok) group.push_back(i);
+    if ((s = launch_2sm_group(args, group, ptok, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int tok : kTokTiles) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
-      if (args[i].M > kGemvMaxM && !use_2sm(args[i], ds) && pick_tok(args[i].M) == tok) group.push_back(i);
+      if (args[i].M > kGemvMaxM && !pair_tok(args[i], ds) && pick_tok(args[i].M) == tok) group.push_back(i);
     for (size_t g0 = 0; g0 < group.size(); g0 += kMaxProblems) {
       std::memset(static_cast<void*>(&batch), 0, sizeof batch);
       int64_t total = 0;
@@ -639,7 +649,7 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
   std::lock_guard<std::mutex> lock(batch_mu);
   // Neither the small-M GEMV nor the pair-tile kernel needs scratch.
   if (M <= kGemvMaxM) return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch, ds, cs);
-  if (use_2sm(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, batch, ds, cs);
+  if (const int ptok = pair_tok(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, ptok, batch, ds, cs);
 
   // Same tile and split choice as tern_linear, so the two give identical y.
   const int tok = pick_tok(M);

@@ -14,9 +14,9 @@
 //
 // Per CTA, per 128-wide k stage (36 KiB of shared memory, 6 stages; the last
 // stage of a row holds 64 k when K % 128 == 64):
-//   * warp 0 (producer): tiled TMA copies of its 128 x-rows (one 64 k x 128
-//     row box per 64 k, 128-byte swizzle) and one bulk copy of its codes
-//     (128 channels x 128 k, contiguous in the tile-interleaved layout), all
+//   * warp 0 (producer): one 3-D TMA copy of its 128 x-rows x 128 k (two
+//     64-k chunks, 128-byte swizzle) and one bulk copy of its codes (128
+//     channels x 128 k, contiguous in the tile-interleaved layout), both
 //     completing on full[s].
 //   * warps 2-5 (decoders): one thread per channel row waits for the stage
 //     and for TMEM slot a (4 slots of 64 columns) to be free, expands its
@@ -35,6 +35,8 @@
 // Work is persistent: cluster c takes tiles c, c + #clusters, ...  No TMA
 // multicast is used: every copy reads this GPU's global memory into the
 // issuing CTA's own shared memory.
+#include <algorithm>
+
 #include "internal.h"
 #include "kernel_common.cuh"
 #include "ptx.cuh"
@@ -43,29 +45,45 @@ namespace tern {
 
 namespace {
 
+// TOK = UMMA N = tokens per tile.  PAIR: a cluster of two CTAs shares each
+// MMA (cta_group::2, M = 256 channels, each CTA loads TOK / 2 x rows) -- used
+// for TOK = 256, where one instruction is long enough to hide its issue cost.
+// !PAIR: one CTA per tile (cta_group::1, M = 128 channels, all TOK x rows),
+// used for TOK = 64, where a pair instruction would take as long as at
+// N = 256 but do a quarter of the work.
+template <int TOK, bool PAIR>
 struct Cfg2 {
-  static constexpr int kTokPair = 256;            // UMMA N: tokens per tile
-  static constexpr int kTokCta = 128;             // x rows each CTA loads
+  static constexpr int kTokPair = TOK;
+  static constexpr int kTokCta = PAIR ? TOK / 2 : TOK;  // x rows each CTA loads
+  static constexpr int kChCta = 128;              // channels (TMEM lanes) per CTA
+  static constexpr int kChTile = PAIR ? 256 : 128;  // channels per tile
   static constexpr int kBK = 128;                 // k per stage
-  static constexpr int kXBox = kTokCta * 128;     // one 64 k x 128 row box, 128-byte swizzle
+  static constexpr int kXBox = kTokCta * 128;     // one 64 k x kTokCta row box, 128-byte swizzle
   static constexpr int kXBytes = 2 * kXBox;
   static constexpr int kCSub = 128 * 16;          // codes of 128 channels x 64 k
   static constexpr int kCBytes = 2 * kCSub;
   static constexpr int kStageBytes = kXBytes + kCBytes;
-  static constexpr int kStages = 6;
+  static constexpr int kStages = kStageBytes > 24 * 1024 ? 6 : 8;
   static constexpr int kASlots = 4;               // decoded-weight slots in TMEM
   static constexpr int kACols = kBK / 2;          // 32-bit TMEM columns per slot (bf16x2)
-  static constexpr int kDCols = kTokPair;         // the accumulator
-  static constexpr int kACol0 = kDCols;
+  static constexpr int kDCols = TOK;              // one accumulator
+  // Two accumulators (the epilogue of a tile overlaps the next tile's MMAs)
+  // where TMEM has room next to the A slots; one at N = 256.
+  static constexpr int kAccBufs = TOK >= 256 ? 1 : 2;
+  static constexpr int kACol0 = kAccBufs * kDCols;
   static constexpr int kTmemCols = 512;
-  static constexpr int kDecWarps = 4;
-  static constexpr int kEpiWarps = 8;             // two per TMEM lane quarter, 128 columns each
+  // A narrow tile makes the MMAs of a stage short, so decoding needs more warps.
+  static constexpr int kDecWarps = TOK >= 256 ? 4 : 8;
+  static constexpr int kEpiWarps = 8;             // two per TMEM lane quarter, half the columns each
+  static constexpr int kEpiCols = TOK / 2;
   static constexpr int kEpiWarp0 = 2 + kDecWarps;
   static constexpr int kThreads = (2 + kDecWarps + kEpiWarps) * 32;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-  // kind::f16, D fp32, A/B bf16 K-major, N = 256, M = 256 (the pair).
+  static constexpr int kCtas = PAIR ? 2 : 1;      // CTAs sharing one MMA
+  // kind::f16, D fp32, A/B bf16 K-major, N = TOK, M = 128 per CTA of the MMA.
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                     (uint32_t(kTokPair >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+                                     (uint32_t(TOK >> 3) << 17) | (uint32_t((128 * kCtas) >> 4) << 24);
+  static_assert(TOK % 64 == 0 && TOK >= 64 && TOK <= 256, "UMMA N; 32-column epilogue loads per half");
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
   static_assert(kACol0 + kASlots * kACols <= kTmemCols, "TMEM columns");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -96,19 +114,55 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 }  // namespace
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
-    ternary_mma2_kernel(const __grid_constant__ Batch batch) {
-  using C = Cfg2;
+// The tcgen05 forms of a one-CTA tile (cta_group::1) or a CTA-pair tile
+// (cta_group::2: the leader's commits arrive in both CTAs, the other CTA's
+// warps arrive on the leader's barriers).
+template <bool PAIR>
+struct Tc;
+template <>
+struct Tc<true> {
+  static __device__ __forceinline__ void alloc(uint32_t dst, uint32_t n) { tmem_alloc_2sm(dst, n); }
+  static __device__ __forceinline__ void relinquish() { tmem_relinquish_2sm(); }
+  static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc_2sm(t, n); }
+  static __device__ __forceinline__ void mma(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    mma_bf16_ts_2sm(d, a, b, idesc, acc);
+  }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit_2sm_multicast(bar, 0x3); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit_2sm(bar); }
+  static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return mapa_shared(bar, 0); }
+  static __device__ __forceinline__ void arrive_leader(uint32_t addr) { mbar_arrive_cluster(addr); }
+  static __device__ __forceinline__ void sync_all() { cluster_sync(); }
+};
+template <>
+struct Tc<false> {
+  static __device__ __forceinline__ void alloc(uint32_t dst, uint32_t n) { tmem_alloc(dst, n); }
+  static __device__ __forceinline__ void relinquish() { tmem_relinquish(); }
+  static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc(t, n); }
+  static __device__ __forceinline__ void mma(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    mma_bf16_ts(d, a, b, idesc, acc);
+  }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit(bar); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit(bar); }
+  static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return bar; }
+  static __device__ __forceinline__ void arrive_leader(uint32_t addr) { mbar_arrive(addr); }
+  static __device__ __forceinline__ void sync_all() { __syncthreads(); }
+};
+
+template <int TOK, bool PAIR>
+__device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
+  using C = Cfg2<TOK, PAIR>;
+  using T = Tc<PAIR>;
   constexpr int S = C::kStages;
   constexpr int A = C::kASlots;
+  constexpr int AB = C::kAccBufs;
 
-  __shared__ __align__(8) uint64_t full_bar[S];   // TMA of stage s landed (this CTA)
-  __shared__ __align__(8) uint64_t empty_bar[S];  // MMAs reading stage s done (both CTAs)
-  __shared__ __align__(8) uint64_t afull_bar[A];  // leader: slot a decoded in both CTAs
-  __shared__ __align__(8) uint64_t aempty_bar[A]; // MMAs reading slot a done (both CTAs)
-  __shared__ __align__(8) uint64_t accfull_bar;   // the tile's last MMA is done (both CTAs)
-  __shared__ __align__(8) uint64_t accempty_bar;  // leader: both epilogues drained TMEM
-  __shared__ __align__(8) uint64_t drain_bar;     // leader: every MMA issued is done
+  __shared__ __align__(8) uint64_t full_bar[S];      // TMA of stage s landed (this CTA)
+  __shared__ __align__(8) uint64_t empty_bar[S];     // MMAs reading stage s done (both CTAs)
+  __shared__ __align__(8) uint64_t afull_bar[A];     // leader: slot a decoded in both CTAs
+  __shared__ __align__(8) uint64_t aempty_bar[A];    // MMAs reading slot a done (both CTAs)
+  __shared__ __align__(8) uint64_t accfull_bar[AB];  // a tile's last MMA is done (both CTAs)
+  __shared__ __align__(8) uint64_t accempty_bar[AB]; // leader: both epilogues drained TMEM
+  __shared__ __align__(8) uint64_t drain_bar;        // leader: every MMA issued is done
   __shared__ uint32_t tmem_base_sh;
   extern __shared__ uint8_t dyn_smem[];
 
@@ -116,10 +170,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
   unsigned int* const st = batch.status;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   uint8_t* const smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
-  const int u0 = int(cluster_id_x()), ustep = int(nclusters_x()), units = batch.total_units;
+  const int u0 = PAIR ? int(cluster_id_x()) : int(blockIdx.x);
+  const int ustep = PAIR ? int(nclusters_x()) : int(gridDim.x);
+  const int units = batch.total_units;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -127,21 +183,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int a = 0; a < A; ++a) {
-      mbar_init(smem_u32(&afull_bar[a]), 2 * C::kDecWarps);
+      mbar_init(smem_u32(&afull_bar[a]), C::kCtas * C::kDecWarps);
       mbar_init(smem_u32(&aempty_bar[a]), 1);
     }
-    mbar_init(smem_u32(&accfull_bar), 1);
-    mbar_init(smem_u32(&accempty_bar), 2 * C::kEpiWarps);
+    for (int b = 0; b < AB; ++b) {
+      mbar_init(smem_u32(&accfull_bar[b]), 1);
+      mbar_init(smem_u32(&accempty_bar[b]), C::kCtas * C::kEpiWarps);
+    }
     mbar_init(smem_u32(&drain_bar), 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc_2sm(smem_u32(&tmem_base_sh), C::kTmemCols);
-    tmem_relinquish_2sm();
+    T::alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
+    T::relinquish();
   }
   tc_fence_before();
-  cluster_sync();  // both CTAs' barriers exist and TMEM is allocated
+  T::sync_all();  // (both CTAs') barriers exist and TMEM is allocated
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
@@ -154,7 +212,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
     for (int u = u0; u < units && ok; u += ustep) {
       const Tile2 t = tile_of(batch, u);
       const int kc_total = t.P->K >> 6;  // 64-wide k chunks
-      const uint8_t* codes = t.P->packed + size_t(t.n_tile * 2 + int(rank)) * kc_total * C::kCSub;
+      const uint8_t* codes =
+          t.P->packed + size_t(t.n_tile * C::kCtas + int(rank)) * kc_total * C::kCSub;
       const int row = t.m_tile * C::kTokPair + int(rank) * C::kTokCta;
       for (int kc = 0; kc < kc_total; kc += 2, ++it) {
         const int s = it % S;
@@ -164,9 +223,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
         if (lane == 0) {
           const uint32_t stage = smem_base + s * C::kStageBytes;
           const uint32_t fb = smem_u32(&full_bar[s]);
-          mbar_arrive_expect_tx(fb, nsub * (C::kXBox + C::kCSub));
-          tma_load_2d(stage, &t.P->tmap_x, kc * 64, row, fb);
-          if (nsub == 2) tma_load_2d(stage + C::kXBox, &t.P->tmap_x, kc * 64 + 64, row, fb);
+          // One 3-D box brings both 64-k chunks of x (the second reads as
+          // zero past K); the codes of the stage are one contiguous block.
+          mbar_arrive_expect_tx(fb, C::kXBytes + nsub * C::kCSub);
+          tma_load_3d(stage, &t.P->tmap_x, 0, row, kc, fb);
           tma_load_bulk(stage + C::kXBytes, codes + size_t(kc) * C::kCSub, nsub * C::kCSub, fb);
         }
         __syncwarp();
@@ -177,14 +237,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
       mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer (leader)
-    if (rank == 0) {
+    if (rank == 0) {  // the leader issues for the pair
       int it = 0, lt = 0;
       bool ok = true;
       for (int u = u0; u < units && ok; u += ustep, ++lt) {
         const int kc_total = tile_of(batch, u).P->K >> 6;
-        ok = __shfl_sync(0xffffffffu, mbar_wait(smem_u32(&accempty_bar), (lt & 1) ^ 1, lim, st), 0);
+        const int ab = lt % AB;
+        ok = __shfl_sync(0xffffffffu, mbar_wait(smem_u32(&accempty_bar[ab]), ((lt / AB) & 1) ^ 1, lim, st), 0);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem + ab * C::kDCols;
         for (int kc = 0; kc < kc_total; kc += 2, ++it) {
           const int s = it % S, a = it % A;
           const int nmma = kc + 1 < kc_total ? 8 : 4;
@@ -197,27 +259,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               if (j < nmma)
-                mma_bf16_ts_2sm(tmem, a_tmem + j * 8,
-                                sw128_kmajor_desc(stage + (j >> 2) * C::kXBox + (j & 3) * 32), C::kIdesc,
-                                (kc | j) != 0);
-            mma_commit_2sm_multicast(smem_u32(&empty_bar[s]), 0x3);
-            mma_commit_2sm_multicast(smem_u32(&aempty_bar[a]), 0x3);
+                T::mma(d_tmem, a_tmem + j * 8, sw128_kmajor_desc(stage + (j >> 2) * C::kXBox + (j & 3) * 32),
+                       C::kIdesc, (kc | j) != 0);
+            T::commit_all(smem_u32(&empty_bar[s]));
+            T::commit_all(smem_u32(&aempty_bar[a]));
           }
           __syncwarp();
         }
-        if (ok && lane == 0) mma_commit_2sm_multicast(smem_u32(&accfull_bar), 0x3);
+        if (ok && lane == 0) T::commit_all(smem_u32(&accfull_bar[ab]));
         __syncwarp();
       }
-      if (lane == 0) mma_commit_2sm(smem_u32(&drain_bar));
+      if (lane == 0) T::commit_local(smem_u32(&drain_bar));
       __syncwarp();
       mbar_wait(smem_u32(&drain_bar), 0, lim, st);
     }
   } else if (warp < C::kEpiWarp0) {
     // ------------------------------------------------------ decoders
+    // With four decoder warps each thread expands both 64-k halves of its
+    // row; with eight, warps 2-5 take the first half and warps 6-9 the second.
+    constexpr int kSubs = 8 / C::kDecWarps;  // 64-k halves per decoder warp
     const int quarter = warp & 3;  // TMEM lanes this warp may touch
+    const int sub0 = kSubs == 2 ? 0 : (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t afull_leader0 = mapa_shared(smem_u32(&afull_bar[0]), 0);
+    const uint32_t afull_leader0 = T::leader_addr(smem_u32(&afull_bar[0]));
     int it = 0;
     bool ok = true;
     for (int u = u0; u < units && ok; u += ustep) {
@@ -231,49 +296,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
         tc_fence_after();
         const uint8_t* cp = smem_gen + s * C::kStageBytes + C::kXBytes + r * 16;
         const uint32_t dst = tmem + lane_off + C::kACol0 + a * C::kACols;
-        uint32_t t[32];
-        const uint4 v0 = *reinterpret_cast<const uint4*>(cp);
-        decode_word(v0.x, t + 0);
-        decode_word(v0.y, t + 8);
-        decode_word(v0.z, t + 16);
-        decode_word(v0.w, t + 24);
-        tmem_st32(dst, t);
-        if (kc + 1 < kc_total) {
-          const uint4 v1 = *reinterpret_cast<const uint4*>(cp + C::kCSub);
-          decode_word(v1.x, t + 0);
-          decode_word(v1.y, t + 8);
-          decode_word(v1.z, t + 16);
-          decode_word(v1.w, t + 24);
-          tmem_st32(dst + 32, t);
+#pragma unroll
+        for (int h = 0; h < kSubs; ++h) {
+          const int sub = sub0 + h;
+          if (kc + sub < kc_total) {
+            uint32_t t[32];
+            const uint4 v = *reinterpret_cast<const uint4*>(cp + sub * C::kCSub);
+            decode_word(v.x, t + 0);
+            decode_word(v.y, t + 8);
+            decode_word(v.z, t + 16);
+            decode_word(v.w, t + 24);
+            tmem_st32(dst + sub * 32, t);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(afull_leader0 + a * 8);
+        if (lane == 0) T::arrive_leader(afull_leader0 + a * 8);
       }
     }
   } else {
     // ------------------------------------------------------ epilogue
+    constexpr int kCols = C::kEpiCols;
     const int ew = warp - C::kEpiWarp0;
     const int quarter = warp & 3;
-    const int half = ew >> 2;  // token columns [128 * half, 128 * half + 128)
+    const int half = ew >> 2;  // token columns [kCols * half, kCols * half + kCols)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t accempty_leader = mapa_shared(smem_u32(&accempty_bar), 0);
+    const uint32_t accempty_leader0 = T::leader_addr(smem_u32(&accempty_bar[0]));
     int lt = 0;
     for (int u = u0; u < units; u += ustep, ++lt) {
       const Tile2 t = tile_of(batch, u);
       const Problem& P = *t.P;
-      const int n = t.n_tile * 256 + int(rank) * 128 + r;
+      const int ab = lt % AB;
+      const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
       const float sc = P.scales[n];
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar), lt & 1, lim, st))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
       tc_fence_after();
-      uint32_t out[64];  // bf16x2: tokens (2c, 2c + 1) of this half
+      uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < kCols; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + half * 128 + c0, v);
+        tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -282,12 +347,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(accempty_leader);
-      const int row0 = t.m_tile * C::kTokPair + half * 128;
-      const int rows = min(128, P.M - row0);
+      if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+      const int row0 = t.m_tile * C::kTokPair + half * kCols;
+      const int rows = min(kCols, P.M - row0);
       uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
 #pragma unroll
-      for (int c = 0; c < 128; ++c)
+      for (int c = 0; c < kCols; ++c)
         if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
     }
   }
@@ -295,45 +360,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2::kThreads, 1)
   // ------------------------------------------------------ teardown
   // No CTA may leave while the pair's MMAs or remote arrivals still touch it.
   tc_fence_before();
-  cluster_sync();
+  T::sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_2sm(tmem, C::kTmemCols);
+    T::dealloc(tmem, C::kTmemCols);
   }
 }
 
-int smem_bytes_2sm() { return Cfg2::kSmemBytes; }
+// Pair tiles run as clusters of two CTAs; single-CTA tiles without clusters.
+template <int TOK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<TOK, true>::kThreads, 1)
+    ternary_pair_kernel(const __grid_constant__ Batch batch) {
+  tile_kernel_body<TOK, true>(batch);
+}
+template <int TOK>
+__global__ void __launch_bounds__(Cfg2<TOK, false>::kThreads, 1)
+    ternary_tile_kernel(const __grid_constant__ Batch batch) {
+  tile_kernel_body<TOK, false>(batch);
+}
+template <int TOK, bool PAIR>
+constexpr auto tile_kernel() {
+  if constexpr (PAIR) return ternary_pair_kernel<TOK>;
+  else return ternary_tile_kernel<TOK>;
+}
 
-static cudaError_t configure_2sm() {
+template <int TOK, bool PAIR>
+static cudaError_t configure_tile() {
   static unsigned long long configured = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
   if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & (1ull << dev))) {
-    e = cudaFuncSetAttribute(ternary_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg2::kSmemBytes);
+    e = cudaFuncSetAttribute(tile_kernel<TOK, PAIR>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg2<TOK, PAIR>::kSmemBytes);
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
   return cudaSuccess;
 }
 
-cudaError_t launch_ternary_mma2(const Batch& batch, int clusters, cudaStream_t stream) {
-  cudaError_t e = configure_2sm();
+// `ctas_or_pairs` CTAs (one-CTA tiles) or clusters of two (pair tiles).
+template <int TOK, bool PAIR>
+static cudaError_t launch_tile(const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
+  using C = Cfg2<TOK, PAIR>;
+  cudaError_t e = configure_tile<TOK, PAIR>();
   if (e != cudaSuccess) return e;
-  ternary_mma2_kernel<<<2 * clusters, Cfg2::kThreads, Cfg2::kSmemBytes, stream>>>(batch);
+  tile_kernel<TOK, PAIR>()<<<C::kCtas * ctas_or_pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
   return cudaGetLastError();
 }
 
+cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
+  if (pair && tok == 256) return launch_tile<256, true>(batch, ctas_or_pairs, stream);
+  if (!pair && tok == 64) return launch_tile<64, false>(batch, ctas_or_pairs, stream);
+  return cudaErrorInvalidValue;
+}
+
 int max_active_clusters_2sm() {
-  if (configure_2sm() != cudaSuccess) return 0;
+  if (configure_tile<256, true>() != cudaSuccess || configure_tile<64, false>() != cudaSuccess) return 0;
   int n = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 148);
-  cfg.blockDim = dim3(Cfg2::kThreads);
-  cfg.dynamicSmemBytes = Cfg2::kSmemBytes;
-  if (cudaOccupancyMaxActiveClusters(&n, ternary_mma2_kernel, &cfg) != cudaSuccess) return 0;
+  cfg.blockDim = dim3(Cfg2<256, true>::kThreads);
+  cfg.dynamicSmemBytes = Cfg2<256, true>::kSmemBytes;
+  if (cudaOccupancyMaxActiveClusters(&n, ternary_pair_kernel<256>, &cfg) != cudaSuccess) return 0;
   return n;
 }
 

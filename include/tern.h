@@ -96,8 +96,9 @@ TERN_API tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K
  *   bias    [N] bf16, or NULL for no bias.
  *   y_bf16  [M, N] bf16 output, overwritten (round to nearest even).
  * Products are exact (T is +-1/0), sums are fp32, then y = fp32 sum * s + b.
- * M <= 16 runs on a register-fed GEMV kernel that needs no scratch.
- * 16 < M <= 64 splits K across CTAs and uses a library-owned fp32 workspace
+ * M <= 16 runs on a register-fed GEMV kernel; N % 256 == 0 with M > 16 on
+ * CTA pairs; neither needs scratch.  The remaining case, 16 < M <= 64 with
+ * N % 256 != 0, splits K across CTAs and uses a library-owned fp32 workspace
  * per (device, stream), allocated on the first such call; make that first
  * call outside CUDA stream capture.  Calls on the same stream are ordered;
  * calls on different streams use different workspaces.
@@ -115,7 +116,7 @@ TERN_API tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const
  * is an interface choice of this library.
  *   Arguments, layouts and results are those of tern_linear, and the tile and
  *   split choice is the same, so y matches tern_linear's bit for bit.
- *   Scratch: the path for 16 < M <= 64 splits K across CTAs and keeps its
+ *   Scratch: the path for 16 < M <= 64 with N % 256 != 0 splits K and keeps its
  *   fp32 partial sums and per-tile counters in one static device array of
  *   10 MiB + 4 KiB inside this library (held on every GPU that loads the
  *   library until the process exits).  That covers every shape on a 148-SM

@@ -154,6 +154,14 @@ def test_linear_pair_tiles(M, N, K):
     run_linear_case(M, N, K, seed=M + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(17, 256, 64), (24, 768, 192), (31, 512, 3072), (32, 256, 448),
+                                   (33, 1280, 320), (48, 256, 128), (64, 2560, 576)])
+def test_linear_pair_tiles_narrow(M, N, K):
+    """16 < M <= 64 with N % 256 == 0 runs on CTA pairs with 64-token tiles
+    (double-buffered accumulators, eight decoder warps)."""
+    run_linear_case(M, N, K, seed=3 * M + N + K)
+
+
 def test_linear_no_bias():
     run_linear_case(40, 256, 256, seed=3, with_bias=False)
     run_linear_case(257, 256, 256, seed=4, with_bias=False)
