@@ -9,12 +9,14 @@
 // |W[n,k]| / s_n > 1/2, i.e. |W[n,k]| > s_n / 2; s_n / 2 is exact in fp32, so
 // the kernel decides every code exactly for the fp32 s_n it stores.
 //
-// One warp owns one row.  Pass 1 streams the row with 16-byte loads and sums
-// |w|: eight values in fp32 (a pairwise tree, error <= 3 ulp of the group),
-// the groups in fp64, then s_n = fp32(sum / K + eps) is rounded once.  Pass 2
-// re-reads the row (now in L1/L2), forms the 2-bit codes and writes them in
-// the tile-interleaved layout: the lane that read k = 8L..8L+7 builds half
-// of the 32-bit word for 16 consecutive k, its neighbour lane the other half.
+// One warp owns one row.  It sums |w| over 16-byte loads: eight values in
+// fp32 (a pairwise tree, error <= 3 ulp of the group), the groups in fp64,
+// then s_n = fp32(sum / K + eps) is rounded once.  It then forms the 2-bit
+// codes and writes them in the tile-interleaved layout: the lane that read
+// k = 8L..8L+7 builds half of the 32-bit word for 16 consecutive k, its
+// neighbour lane the other half.  Rows of up to 4096 values stay in
+// registers between the two steps; longer rows are read twice (the second
+// time from L2).
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -35,55 +37,115 @@ __device__ __forceinline__ float abs_sum8(const uint4& v) {
   return (a + b) + (c + d);
 }
 
-// 2-bit two's-complement code of one bf16 value given the fp32 threshold
-// s/2 (as bits, non-negative): 01 for +1, 11 for -1, 00 for 0.  Magnitudes of
-// non-negative floats order like their bit patterns.
-__device__ __forceinline__ uint32_t code_of(uint32_t b16, uint32_t half_s_bits) {
-  const uint32_t nz = ((b16 & 0x7FFFu) << 16) > half_s_bits ? 1u : 0u;
-  const uint32_t neg = b16 >> 15;
+
+// Codes of the two bf16 values of a 32-bit word (k in the low half, k + 1 in
+// the high half) at bits 0-1 and 16-17, given the bf16 threshold thr16 =
+// the top 16 bits of the fp32 s/2.  For a bf16 magnitude m (15 bits),
+// m > thr16 exactly when |w| > s/2 (|w| is a bf16; thr16 is s/2 rounded
+// down to bf16).  Per half, 0x8000 + thr16 - m stays in [1, 0xFFFF], so its
+// bit 15 is clear exactly when m > thr16, with no borrow into the other half.
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, uint32_t thr_pair) {
+  const uint32_t mag = w & 0x7FFF7FFFu;
+  const uint32_t nz = (~((thr_pair | 0x80008000u) - mag) >> 15) & 0x00010001u;
+  const uint32_t neg = (w >> 15) & 0x00010001u;
   return nz | ((nz & neg) << 1);
 }
 
+// Same computation with the row held in registers, so W is read from HBM
+// once: a lane keeps its NV 16-byte groups (k = 8i .. 8i + 7, i = lane +
+// 32 t) from the mean through the codes.  All NV loads are issued before the
+// first is used.  For K <= 256 NV.
+template <int NV>
 __global__ void __launch_bounds__(kRowsPerCta * 32)
-    quantize_pack_kernel(const uint16_t* __restrict__ W, int N, int K, float eps,
-                         uint8_t* __restrict__ packed, float* __restrict__ scales) {
+    quantize_pack_regs_kernel(const uint16_t* __restrict__ W, int N, int K, float eps,
+                              uint8_t* __restrict__ packed, float* __restrict__ scales) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kRowsPerCta + warp;
   if (n >= N) return;
   const uint4* row = reinterpret_cast<const uint4*>(W + size_t(n) * K);
-  const int n8 = K >> 3;  // 16-byte groups of 8 values; K % 64 == 0 -> n8 % 8 == 0
-
-  // ---- pass 1: mean magnitude
+  const int n8 = K >> 3;
+  uint4 v[NV];
+#pragma unroll
+  for (int t = 0; t < NV; ++t) {
+    const int i = lane + 32 * t;
+    v[t] = i < n8 ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // ---- mean magnitude: groups of eight in fp32, groups summed in fp64
   double acc = 0.0;
-#pragma unroll 4
-  for (int i = lane; i < n8; i += 32) acc += double(abs_sum8(__ldg(row + i)));
+#pragma unroll
+  for (int t = 0; t < NV; ++t) acc += double(abs_sum8(v[t]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   const float s = float(acc / double(K) + double(eps));
   if (lane == 0) scales[n] = s;
-  const uint32_t half_s = __float_as_uint(0.5f * s);
+  const uint32_t thr16 = __float_as_uint(0.5f * s) >> 16;
+  const uint32_t thr_pair = thr16 | (thr16 << 16);
 
-  // ---- pass 2: codes
+  // ---- codes
   uint8_t* slab = packed + size_t(n >> 7) * size_t(K >> 6) * 2048 + size_t(n & 127) * 16;
-  for (int base = 0; base < n8; base += 32) {
-    const int i = base + lane;  // this lane's 8 values are k = 8i .. 8i+7
-    uint32_t word = 0;
-    if (i < n8) {
-      const uint4 v = __ldg(row + i);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-      const int j0 = (i & 1) * 4;  // pair index of k = 8i inside its 16-k word
+  const int j0 = (lane & 1) * 4;  // pair index of k = 8i inside its 16-k word (i has lane's parity)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // k = 8i + 2e (even) and 8i + 2e + 1 (odd): pair j0 + e
-        word |= code_of(w4[e] & 0xFFFFu, half_s) << (2 * (j0 + e));
-        word |= code_of(w4[e] >> 16, half_s) << (16 + 2 * (j0 + e));
-      }
-    }
+  for (int t = 0; t < NV; ++t) {
+    const int i = lane + 32 * t;
+    const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) word |= code_pair(w4[e], thr_pair) << (2 * (j0 + e));
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    if (i < n8 && (i & 1) == 0) {
-      const int chunk = i >> 3;          // 64-wide k chunk
-      const int wsel = (i & 7) >> 1;     // word inside the 16-byte group
-      *reinterpret_cast<uint32_t*>(slab + size_t(chunk) * 2048 + wsel * 4) = word;
+    if (i < n8 && (i & 1) == 0)
+      *reinterpret_cast<uint32_t*>(slab + size_t(i >> 3) * 2048 + ((i & 7) >> 1) * 4) = word;
+  }
+}
+
+// Rows longer than 4096 values: the same steps over segments of 4096 values
+// (16 groups of eight per lane, all loads of a segment in flight), the mean
+// over every segment first, then the codes segment by segment, re-reading
+// the row (from L2: a warp's row is at most 2 MiB / 64 = 32 KiB here).
+__global__ void __launch_bounds__(kRowsPerCta * 32)
+    quantize_pack_long_kernel(const uint16_t* __restrict__ W, int N, int K, float eps,
+                              uint8_t* __restrict__ packed, float* __restrict__ scales) {
+  constexpr int NV = 16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * kRowsPerCta + warp;
+  if (n >= N) return;
+  const uint4* row = reinterpret_cast<const uint4*>(W + size_t(n) * K);
+  const int n8 = K >> 3;
+  double acc = 0.0;
+  for (int base = 0; base < n8; base += 32 * NV) {
+    uint4 v[NV];
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+      const int i = base + lane + 32 * t;
+      v[t] = i < n8 ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < NV; ++t) acc += double(abs_sum8(v[t]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  const float s = float(acc / double(K) + double(eps));
+  if (lane == 0) scales[n] = s;
+  const uint32_t thr16 = __float_as_uint(0.5f * s) >> 16;
+  const uint32_t thr_pair = thr16 | (thr16 << 16);
+  uint8_t* slab = packed + size_t(n >> 7) * size_t(K >> 6) * 2048 + size_t(n & 127) * 16;
+  const int j0 = (lane & 1) * 4;
+  for (int base = 0; base < n8; base += 32 * NV) {
+    uint4 v[NV];
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+      const int i = base + lane + 32 * t;
+      v[t] = i < n8 ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+      const int i = base + lane + 32 * t;
+      const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) word |= code_pair(w4[e], thr_pair) << (2 * (j0 + e));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      if (i < n8 && (i & 1) == 0)
+        *reinterpret_cast<uint32_t*>(slab + size_t(i >> 3) * 2048 + ((i & 7) >> 1) * 4) = word;
     }
   }
 }
@@ -137,8 +199,19 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns, unsigned int* 
 cudaError_t launch_quantize_pack(const __nv_bfloat16* W, int N, int K, float eps, uint8_t* packed,
                                  float* scales, cudaStream_t stream) {
   const int grid = (N + kRowsPerCta - 1) / kRowsPerCta;
-  quantize_pack_kernel<<<grid, kRowsPerCta * 32, 0, stream>>>(reinterpret_cast<const uint16_t*>(W), N,
-                                                             K, eps, packed, scales);
+  const uint16_t* w = reinterpret_cast<const uint16_t*>(W);
+  // Rows of up to 4096 values stay in registers (one read of W); longer rows
+  // are read twice, the second time mostly from L2.
+  if (K <= 32 * 8 * 4)
+    quantize_pack_regs_kernel<4><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+  else if (K <= 32 * 8 * 8)
+    quantize_pack_regs_kernel<8><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+  else if (K <= 32 * 8 * 12)
+    quantize_pack_regs_kernel<12><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+  else if (K <= 32 * 8 * 16)
+    quantize_pack_regs_kernel<16><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+  else
+    quantize_pack_long_kernel<<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
   return cudaGetLastError();
 }
 
