@@ -38,7 +38,7 @@ CSRC = os.path.join(ROOT, "bit_post_quantised_b200", "csrc")
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tern", "reference"], default="tern")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -62,10 +62,13 @@ def load_peaks():
 
 
 def linear_kernel(layer):
-    """(kernel name, source file stem) of the tern_linear launch for this shape:
-    M > 64 with N % 256 == 0 runs on SM pairs, everything else on single SMs."""
-    if layer.M > 64 and layer.N % 256 == 0:
-        return "ternary_mma2_kernel", "ternary_mma2"
+    """(kernel name, source file stem) of the tern_linear launch for this shape
+    (the routing of the library's host code)."""
+    if layer.M <= 16:
+        return "ternary_gemv_kernel", "ternary_gemv"
+    if layer.N % 256 == 0:
+        return ("ternary_pair_kernel<256>", "ternary_mma2") if layer.M > 64 else \
+            ("ternary_tile_kernel<64>", "ternary_mma2")
     return "ternary_mma_kernel", "ternary_mma"
 
 
@@ -89,60 +92,93 @@ def profiled_traffic(stem: str, workload: str):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and clock-event (throttle) reasons while the timed
+    region runs: NVML every 2 ms from a thread (reads only), else nvidia-smi
+    every 100 ms."""
 
+    # NVML clock-event reason bits
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.samples = []  # (sm_mhz, max_mhz, reasons set)
         self.proc = None
+        self.thread = None
+        self.stop = False
+
+    def _nvml_loop(self, handle, nv):
+        mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+            except Exception:
+                break
+            self.samples.append((float(sm), float(mx), {k for k, b in self.REASONS.items() if bits & b}))
+            time.sleep(0.002)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.25)
+            import pynvml as nv
+
+            nv.nvmlInit()
+            handle = (nv.nvmlDeviceGetHandleByUUID(self.gpu) if self.gpu.startswith("GPU-")
+                      else nv.nvmlDeviceGetHandleByIndex(int(self.gpu)))
+            import threading
+
+            self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+            time.sleep(0.25)
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc is not None:
             time.sleep(0.15)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                out, _ = self.proc.communicate()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in out.strip().splitlines():
+                f = [v.strip() for v in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    self.samples.append((float(f[1]), float(f[2]),
+                                         {n for n, v in zip(names, f[5:9]) if v.lower() == "active"}))
+                except ValueError:
+                    continue
 
     def summary(self):
-        if self.proc is None or not getattr(self, "out", ""):
+        if not self.samples:
             return None
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.strip().splitlines():
-            f = [v.strip() for v in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return None
+        sm = [a for a, _, _ in self.samples]
         hi = max(sm)
         loaded = [v for v in sm if v >= 0.5 * hi] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(b for _, b, _ in self.samples),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvml 2 ms" if self.thread is not None else "nvidia-smi 100 ms"}
 
 
 # ------------------------------------------------------------ CPU oracle leg
