@@ -227,7 +227,7 @@ def run_reference(args):
 
     layer = workloads.CONFIGS[args.workload]
     x, W, b = workloads.make_inputs(layer)
-    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.3, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample_step(layer, x, W, b, per_step)
     ests, samples = [], []
