@@ -407,7 +407,71 @@ def side_table(device, peaks, stream):
     nbytes = 2 * N * K + N * K // 4 + 4 * N
     rows["quantize_pack_21504x3072"] = {"us": t * 1e6, "gbs": nbytes / t / 1e9,
                                         "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    del W, p, s
+    rows.update(stack_rows(device, peaks, stream))
     return rows
+
+
+def stack_rows(device, peaks, stream):
+    """The whole ternary linear stack of one FLUX.1-dev forward at 1024x1024
+    (19 double + 38 single blocks; weights drawn on the device from N(0, 0.02)
+    per layer seed and quantised, only the codes kept), run block by block
+    through tern_linear_batch with synthetic activations, and the 76 adaLN
+    modulation GEMVs of a forward alone: batched versus one call each."""
+    import torch
+
+    from bit_post_quantised_b200 import tern, workloads
+
+    layers = workloads.flux_stack()
+    packs = []
+    for L in layers:
+        g = torch.Generator(device=device).manual_seed(L.seed)
+        W = (torch.randn(L.N, L.K, generator=g, device=device) * L.w_std).to(torch.bfloat16)
+        packs.append(tern.quantize_pack(W, workloads.EPS, stream=stream))
+        del W
+    bias = {}
+    xs, ys = {}, {}
+
+    def buf(d, key, shape):
+        if key not in d:
+            d[key] = (torch.randn(*shape, device=device) * 0.5).to(torch.bfloat16)
+        return d[key]
+
+    blocks = {}
+    for i, L in enumerate(layers):
+        blocks.setdefault(L.name.split(".")[0], []).append(i)
+    problems = []  # per block: list of dicts for tern_linear_batch
+    for name, idx in blocks.items():
+        probs = []
+        for j, i in enumerate(idx):
+            L = layers[i]
+            if L.N not in bias:
+                bias[L.N] = (torch.randn(L.N, device=device) * 0.01).to(torch.bfloat16)
+            probs.append(dict(x=buf(xs, (L.M, L.K), (L.M, L.K)), packed=packs[i][0], scales=packs[i][1],
+                              bias=bias[L.N], y=buf(ys, (j, L.M, L.N), (L.M, L.N))))
+        problems.append(probs)
+    flop = sum(L.flop for L in layers)
+
+    def forward():
+        for probs in problems:
+            tern.linear_batch(probs, stream=stream)
+
+    t = graph_time([forward], 3, stream)
+    out = {"flux_stack": {"layers": len(layers), "launch_groups": "one tern_linear_batch per block",
+                          "ms_per_forward": t * 1e3, "tflops": flop / t / 1e12,
+                          "tensor_roofline_ms": flop / (peaks["bf16_tflops"] * 1e12) * 1e3,
+                          "packed_weight_gb": sum(L.packed_bytes for L in layers) / 1e9}}
+    mods = [dict(x=buf(xs, (1, L.K), (1, L.K)), packed=packs[i][0], scales=packs[i][1], bias=bias[L.N],
+                 y=buf(ys, ("mod", i), (1, L.N))) for i, L in enumerate(layers) if L.name.endswith(".mod")]
+    mod_bytes = sum(p["packed"].numel() for p in mods)
+    t_batch = graph_time([lambda: tern.linear_batch(mods, stream=stream)], 5, stream)
+    t_each = graph_time([lambda: [tern.linear(p["x"], p["packed"], p["scales"], p["bias"], out=p["y"],
+                                              stream=stream) for p in mods]], 5, stream)
+    out["modulation_gemvs_per_forward"] = {
+        "count": len(mods), "packed_mb": mod_bytes / 1e6,
+        "batched_us": t_batch * 1e6, "batched_packed_gbs": mod_bytes / t_batch / 1e9,
+        "one_call_each_us": t_each * 1e6, "hbm_frac_batched": mod_bytes / t_batch / 1e9 / peaks["hbm_gbs"]}
+    return out
 
 
 def gpu_id_for_smi(local: int) -> str:

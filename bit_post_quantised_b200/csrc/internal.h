@@ -79,11 +79,13 @@ int smem_bytes_for_tok(int tok);
 // work units run at once.
 cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream);
 int max_active_clusters_2sm();
-// Small-M kernel (M <= 8 nt tokens, nt in {1, 2}): grid (splits, slabs) with
-// clusters of `splits` CTAs along k; problems use n_tiles = N / 128 slabs,
-// unit_begin = first slab in the launch, chunks_per_split 64-k chunks per CTA
-// and a 3-D x tensor map {64 k, M, K / 64} whose box is {64, min(M, 8 nt), 8}.
-cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int slabs, cudaStream_t stream);
+// Small-M kernel (M <= 8 nt tokens, nt in {1, 2}), persistent over work
+// units (problem, 128-channel slab): grid (splits, ctas) with clusters of
+// `splits` CTAs along k (splits > 1 needs ctas == total_units); problems use
+// n_tiles = N / 128 slabs, unit_begin = first slab in the launch,
+// chunks_per_split 64-k chunks per CTA and a 3-D x tensor map {64 k, M,
+// K / 64} whose box is {64, min(M, 8 nt), 8}.
+cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream);
 int max_active_clusters_2sm();
 int smem_bytes_2sm();
 

@@ -356,7 +356,9 @@ tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<in
     batch.total_units = int(slabs);
     batch.wait_limit_ns = g_wait_limit_ns.load();
     batch.status = ds->status;
-    cudaError_t e = launch_ternary_gemv(nt, batch, splits, int(slabs), cs);
+    // splits > 1: one CTA per slab; otherwise persistent CTAs, one per SM at most.
+    const int ctas = splits > 1 ? int(slabs) : int(std::min<int64_t>(slabs, ds->sms));
+    cudaError_t e = launch_ternary_gemv(nt, batch, splits, ctas, cs);
     if (e != cudaSuccess) return cuda_fail(e, "ternary_gemv launch");
   }
   return TERN_OK;

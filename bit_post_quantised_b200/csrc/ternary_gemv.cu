@@ -48,7 +48,12 @@ namespace {
 template <int NT>
 struct GemvCfg {
   static constexpr int kGroups = 8;                  // 16-channel groups per 128-channel slab
-  static constexpr int kWarps = 2 * kGroups;         // consumer warps: two per group
+  // Consumer warps per group, splitting every stage's chunks round-robin.
+  // More warps hide more of the expansion's dependency latency; NT = 2 keeps
+  // two because its accumulators need the registers.
+  static constexpr int kSplit = 2;
+  static constexpr int kWarps = kSplit * kGroups;
+  static constexpr int kPerWarp = (8 + kSplit - 1) / kSplit;  // chunks per warp per stage (at most)
   static constexpr int kThreads = (kWarps + 1) * 32;  // + one producer warp
   static constexpr int kChunks = 8;                  // 64-k chunks per stage
   static constexpr int kStages = 6;
@@ -83,10 +88,21 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 
 }  // namespace
 
-// Grid (splits, total slabs), cluster (splits, 1, 1): blockIdx.y picks the
-// problem and its 128-channel slab, blockIdx.x (the rank in the cluster) the
-// k range (chunks_per_split 64-k chunks).  The x tensor map is 3-D
-// {64 k, M tokens, K / 64 chunks} with box {64, min(M, 8 NT), 8}.
+// Grid (splits, G), cluster (splits, 1, 1).  Work unit u = one 128-channel
+// slab of one problem of the batch (u < total_units); the CTAs with
+// blockIdx.y = g take units g, g + G, ...  (persistent: the producer streams
+// the next unit's codes while the consumers finish the current one).
+// blockIdx.x, the rank in the cluster, picks the k range of every unit
+// (chunks_per_split 64-k chunks).  The x tensor map is 3-D {64 k, M tokens,
+// K / 64 chunks} with box {64, min(M, 8 NT), 8}.
+template <int NT>
+__device__ __forceinline__ const Problem& unit_problem(const Batch& batch, int u, int* slab) {
+  int pi = 0;
+  while (pi + 1 < batch.count && u >= batch.p[pi + 1].unit_begin) ++pi;
+  *slab = u - batch.p[pi].unit_begin;
+  return batch.p[pi];
+}
+
 template <int NT>
 __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     ternary_gemv_kernel(const __grid_constant__ Batch batch) {
@@ -96,7 +112,8 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
 
   __shared__ __align__(8) uint64_t full_bar[S];   // codes and x of stage s landed
   __shared__ __align__(8) uint64_t empty_bar[S];  // all consumer warps are done with stage s
-  __shared__ __align__(16) float part[C::kGroups * 32 * NT * 4];  // odd-chunk warps' sums, then the CTA's
+  // Sums of the warps with half > 0 (one slot each), then the CTA's total.
+  __shared__ __align__(16) float part[(C::kSplit - 1) * C::kGroups * 32 * NT * 4];
   extern __shared__ uint8_t dyn_smem[];
 
   const uint64_t lim = batch.wait_limit_ns;
@@ -105,19 +122,14 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   const uint8_t* const smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
-
-  const int unit = blockIdx.y;
-  int pi = 0;
-  while (pi + 1 < batch.count && unit >= batch.p[pi + 1].unit_begin) ++pi;
-  const Problem& P = batch.p[pi];
-  const int slab = unit - P.unit_begin;
   const int splits = gridDim.x, rank = blockIdx.x;
-  const int kc_total = P.K >> 6;
-  const int kc0 = rank * P.chunks_per_split;
-  const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
-  const int nstages = (nk + C::kChunks - 1) / C::kChunks;
-  const int rows = min(P.M, 8 * NT);  // token rows the x box fetches
-  const uint8_t* codes = P.packed + (size_t(slab) * kc_total + kc0) * 2048;
+  const int u0 = blockIdx.y, ustep = gridDim.y, units = batch.total_units;
+  // With K split over a cluster the producer only joins the per-unit cluster
+  // rendezvous after its whole stream, so each CTA must own a single unit.
+  if (splits > 1 && ustep < units) {
+    if (threadIdx.x == 0) atomicOr(st, kStatusTimeout);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -128,165 +140,194 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     fence_proxy_async_smem();
   }
   __syncthreads();
-
-  float d[NT][4];  // D fragments: channels (g, g + 8) x tokens (2c, 2c + 1) of each n8 block
-#pragma unroll
-  for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) d[nb][e] = 0.f;
   const int grp = warp & (C::kGroups - 1), half = warp / C::kGroups;
-  // Scale and bias of this lane's two output channels, fetched before the
-  // stream starts so their latency is hidden (only rank 0's first warps store).
-  const int n_out = slab * 128 + grp * 16 + (lane >> 2);
-  float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
-  if (warp < C::kGroups && rank == 0) {
-    s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
-    s1 = 0.5f * P.scales[n_out + 8];
-    const uint16_t* bias = reinterpret_cast<const uint16_t*>(P.bias);
-    if (bias) {
-      b0 = bf16_bits_to_float(bias[n_out]);
-      b1 = bf16_bits_to_float(bias[n_out + 8]);
-    }
-  }
 
   if (warp == C::kWarps) {
     // ------------------------------------------------------ producer
-    if (lane == 0) prefetch_tensormap(&P.tmap_x);
-    int issued = 0;
-    for (int i = 0; i < nstages; ++i) {
-      const int s = i % S;
-      if (i >= S &&
-          !__shfl_sync(0xffffffffu, mbar_wait(smem_u32(&empty_bar[s]), ((i / S) & 1) ^ 1, lim, st), 0))
-        break;
-      if (lane == 0) {
-        const int nch = min(C::kChunks, nk - i * C::kChunks);
-        const uint32_t stage = smem_base + s * C::kStageBytes;
-        const uint32_t fb = smem_u32(&full_bar[s]);
-        mbar_arrive_expect_tx(fb, nch * 2048 + C::kChunks * rows * 128);
-        tma_load_bulk(stage, codes + size_t(i) * C::kCodeBytes, nch * 2048, fb);
-        tma_load_3d(stage + C::kCodeBytes, &P.tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
+    if (lane == 0)
+      for (int pi = 0; pi < batch.count; ++pi) prefetch_tensormap(&batch.p[pi].tmap_x);
+    int it = 0;
+    bool ok = true;
+    for (int u = u0; u < units && ok; u += ustep) {
+      int slab;
+      const Problem& P = unit_problem<NT>(batch, u, &slab);
+      const int kc_total = P.K >> 6;
+      const int kc0 = rank * P.chunks_per_split;
+      const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
+      const int rows = min(P.M, 8 * NT);
+      const uint8_t* codes = P.packed + (size_t(slab) * kc_total + kc0) * 2048;
+      for (int i = 0; i * C::kChunks < nk; ++i, ++it) {
+        const int s = it % S;
+        if (it >= S &&
+            !__shfl_sync(0xffffffffu, mbar_wait(smem_u32(&empty_bar[s]), ((it / S) & 1) ^ 1, lim, st), 0)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const int nch = min(C::kChunks, nk - i * C::kChunks);
+          const uint32_t stage = smem_base + s * C::kStageBytes;
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          mbar_arrive_expect_tx(fb, nch * 2048 + C::kChunks * rows * 128);
+          tma_load_bulk(stage, codes + size_t(i) * C::kCodeBytes, nch * 2048, fb);
+          tma_load_3d(stage + C::kCodeBytes, &P.tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      issued = i + 1;
     }
     // No copy may still be landing in shared memory when the CTA exits.
-    for (int i = max(0, issued - S); i < issued; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
-  } else {
-    // ------------------------------------------------------ consumers
-    const int g = lane >> 2, c = lane & 3;
-    // Shared-memory offsets of this lane's two 16-byte x pieces in each of
-    // its chunks (line j * rows + g of the stage's x box, XOR-swizzled by
-    // the line index; the second n8 block is 8 lines = 1 KiB further).
-    uint32_t xoff_a[C::kChunks / 2], xoff_b[C::kChunks / 2];
+    for (int i = max(0, it - S); i < it; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
+  }
+
+  // Consumers walk the same units; all threads (producer included) meet at
+  // the per-unit cluster rendezvous when K is split.
+  const int g = lane >> 2, c = lane & 3;
+  int it = 0;
+  bool ok = true;
+  for (int u = u0; u < units; u += ustep) {
+    int slab;
+    const Problem& P = unit_problem<NT>(batch, u, &slab);
+    float d[NT][4];  // D fragments: channels (g, g + 8) x tokens (2c, 2c + 1) of each n8 block
 #pragma unroll
-    for (int t = 0; t < C::kChunks / 2; ++t) {
-      const uint32_t line = uint32_t((half + 2 * t) * rows + g);
-      xoff_a[t] = line * 128 + ((uint32_t(2 * c) ^ (line & 7)) << 4);
-      xoff_b[t] = line * 128 + ((uint32_t(2 * c + 1) ^ (line & 7)) << 4);
-    }
-    float acc[4][NT][4];  // one accumulator per MMA position q: four independent chains
+    for (int nb = 0; nb < NT; ++nb)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[q][nb][e] = 0.f;
-    for (int i = 0; i < nstages; ++i) {
-      const int s = i % S;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (i / S) & 1, lim, st))) break;
-      const int nch = min(C::kChunks, nk - i * C::kChunks);
-      const uint8_t* stage = smem_gen + s * C::kStageBytes;
-      const uint32_t xstage = smem_base + s * C::kStageBytes + C::kCodeBytes;
-      // Code words first (word c of rows 16 grp + g and 16 grp + g + 8 of
-      // chunks half, half + 2, ...), for all of this warp's chunks at once.
-      uint32_t w0[C::kChunks / 2], w1[C::kChunks / 2];
-#pragma unroll
-      for (int t = 0; t < C::kChunks / 2; ++t) {
-        const int j = half + 2 * t;
-        if (j < nch) {
-          const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + j * 2048) + grp * 64 + lane;
-          w0[t] = cw[0];
-          w1[t] = cw[32];
+      for (int e = 0; e < 4; ++e) d[nb][e] = 0.f;
+    const int n_out = slab * 128 + grp * 16 + g;
+    if (warp < C::kWarps) {
+      // Scale and bias of this lane's two output channels, loaded now and used
+      // after the stream (only rank 0's first warps store).
+      float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
+      if (half == 0 && rank == 0) {
+        s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
+        s1 = 0.5f * P.scales[n_out + 8];
+        const uint16_t* bias = reinterpret_cast<const uint16_t*>(P.bias);
+        if (bias) {
+          b0 = bf16_bits_to_float(bias[n_out]);
+          b1 = bf16_bits_to_float(bias[n_out + 8]);
         }
       }
+      const int kc_total = P.K >> 6;
+      const int nk = max(0, min(kc_total, (rank + 1) * P.chunks_per_split) - rank * P.chunks_per_split);
+      const int rows = min(P.M, 8 * NT);
+      // Shared-memory offsets of this lane's two 16-byte x pieces in each of
+      // its chunks (line j * rows + g of the stage's x box, XOR-swizzled by
+      // the line index; the second n8 block is 8 lines = 1 KiB further).
+      uint32_t xoff_a[C::kPerWarp], xoff_b[C::kPerWarp];
 #pragma unroll
-      for (int t = 0; t < C::kChunks / 2; ++t) {
-        const int j = half + 2 * t;
-        if (j < nch) {
+      for (int t = 0; t < C::kPerWarp; ++t) {
+        const uint32_t line = uint32_t((half + C::kSplit * t) * rows + g);
+        xoff_a[t] = line * 128 + ((uint32_t(2 * c) ^ (line & 7)) << 4);
+        xoff_b[t] = line * 128 + ((uint32_t(2 * c + 1) ^ (line & 7)) << 4);
+      }
+      float acc[4][NT][4];  // one accumulator per MMA position q: four independent chains
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][nb][e] = 0.f;
+      for (int i = 0; ok && i * C::kChunks < nk; ++i, ++it) {
+        const int s = it % S;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (it / S) & 1, lim, st))) {
+          ok = false;
+          break;
+        }
+        const int nch = min(C::kChunks, nk - i * C::kChunks);
+        const uint8_t* stage = smem_gen + s * C::kStageBytes;
+        const uint32_t xstage = smem_base + s * C::kStageBytes + C::kCodeBytes;
+        // Word c of rows 16 grp + g and 16 grp + g + 8 of chunks half,
+        // half + kSplit, ...: 128 contiguous bytes per warp load.
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + half * 2048) + grp * 64 + lane;
+        const uint32_t xh = xstage;
+        auto chunk = [&](int t) {
+          const uint32_t a = cw[t * C::kSplit * 512], b = cw[t * C::kSplit * 512 + 32];
 #pragma unroll
           for (int nb = 0; nb < NT; ++nb) {
-            // x row 8 nb + g of chunk j, k = 16c .. 16c + 15: 16-byte pieces
-            // 2c and 2c + 1 of its 128-byte line, XOR-swizzled by line index.
-            const uint4 xa = ld_shared_v4(xstage + xoff_a[t] + nb * 1024);
-            const uint4 xb = ld_shared_v4(xstage + xoff_b[t] + nb * 1024);
-            const uint32_t a = w0[t], b = w1[t];
+            const uint4 xa = ld_shared_v4(xh + xoff_a[t] + nb * 1024);
+            const uint4 xb = ld_shared_v4(xh + xoff_b[t] + nb * 1024);
             mma_16816(acc[0][nb], pm2_pair<0>(a), pm2_pair<0>(b), pm2_pair<1>(a), pm2_pair<1>(b), xa.x, xa.y);
             mma_16816(acc[1][nb], pm2_pair<2>(a), pm2_pair<2>(b), pm2_pair<3>(a), pm2_pair<3>(b), xa.z, xa.w);
             mma_16816(acc[2][nb], pm2_pair<4>(a), pm2_pair<4>(b), pm2_pair<5>(a), pm2_pair<5>(b), xb.x, xb.y);
             mma_16816(acc[3][nb], pm2_pair<6>(a), pm2_pair<6>(b), pm2_pair<7>(a), pm2_pair<7>(b), xb.z, xb.w);
           }
+        };
+        if (nch == C::kChunks) {  // every stage but a row's last: no bounds tests
+#pragma unroll
+          for (int t = 0; t < C::kPerWarp; ++t) chunk(t);
+        } else {
+#pragma unroll
+          for (int t = 0; t < C::kPerWarp; ++t)
+            if (half + C::kSplit * t < nch) chunk(t);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
-    }
-#pragma unroll
-    for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        d[nb][e] = (acc[0][nb][e] + acc[1][nb][e]) + (acc[2][nb][e] + acc[3][nb][e]);
-    // Even-chunk warps add the odd-chunk warps' sums (fixed order).
-    float* mine = &part[(grp * 32 + lane) * NT * 4];
-    if (half == 1) {
 #pragma unroll
       for (int nb = 0; nb < NT; ++nb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = d[nb][e];
-    }
-    named_barrier_sync(1, kConsumerThreads);
-    if (half == 0) {
-#pragma unroll
-      for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          d[nb][e] += mine[nb * 4 + e];
-          if (splits > 1) mine[nb * 4 + e] = d[nb][e];  // this CTA's total, for rank 0
-        }
-    }
-  }
-
-  // ------------------------------------------------------ reduce and store
-  if (splits > 1) cluster_sync();  // every rank's partial sums are in its shared memory
-  if (warp < C::kGroups && rank == 0) {
-    if (splits > 1) {
-      const uint32_t mine = smem_u32(&part[(warp * 32 + lane) * NT * 4]);
-      for (int r = 1; r < splits; ++r)  // rank order: deterministic
+        for (int e = 0; e < 4; ++e)
+          d[nb][e] = (acc[0][nb][e] + acc[1][nb][e]) + (acc[2][nb][e] + acc[3][nb][e]);
+      // The first warp of each group adds the others' sums in warp order.
+      if (half > 0) {
+        float* slot = &part[(((half - 1) * C::kGroups + grp) * 32 + lane) * NT * 4];
 #pragma unroll
         for (int nb = 0; nb < NT; ++nb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d[nb][e] += ld_shared_cluster_f32(mapa_shared(mine + uint32_t(nb * 4 + e) * 4, uint32_t(r)));
-    }
-    const int c = lane & 3;
-    const int n = n_out;
+          for (int e = 0; e < 4; ++e) slot[nb * 4 + e] = d[nb][e];
+      }
+      named_barrier_sync(1, kConsumerThreads);
+      if (half == 0) {
+        for (int h = 1; h < C::kSplit; ++h) {
+          const float* slot = &part[(((h - 1) * C::kGroups + grp) * 32 + lane) * NT * 4];
 #pragma unroll
-    for (int nb = 0; nb < NT; ++nb) {
-      const int t0 = 8 * nb + 2 * c;
-      if (t0 < P.M) {
-        P.y[size_t(t0) * P.N + n] = __float2bfloat16_rn(fmaf(d[nb][0], s0, b0));
-        P.y[size_t(t0) * P.N + n + 8] = __float2bfloat16_rn(fmaf(d[nb][2], s1, b1));
+          for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[nb][e] += slot[nb * 4 + e];
+        }
+        if (splits > 1) {  // this CTA's total, for rank 0 (the slot read above was this thread's own)
+          float* mine = &part[(grp * 32 + lane) * NT * 4];
+#pragma unroll
+          for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = d[nb][e];
+        }
       }
-      if (t0 + 1 < P.M) {
-        P.y[size_t(t0 + 1) * P.N + n] = __float2bfloat16_rn(fmaf(d[nb][1], s0, b0));
-        P.y[size_t(t0 + 1) * P.N + n + 8] = __float2bfloat16_rn(fmaf(d[nb][3], s1, b1));
+      if (splits > 1) cluster_sync();  // every rank's partial sums are in its shared memory
+      if (half == 0 && rank == 0) {
+        if (splits > 1) {
+          const uint32_t mine = smem_u32(&part[(grp * 32 + lane) * NT * 4]);
+          for (int r = 1; r < splits; ++r)  // rank order: deterministic
+#pragma unroll
+            for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                d[nb][e] += ld_shared_cluster_f32(mapa_shared(mine + uint32_t(nb * 4 + e) * 4, uint32_t(r)));
+        }
+#pragma unroll
+        for (int nb = 0; nb < NT; ++nb) {
+          const int t0 = 8 * nb + 2 * c;
+          if (t0 < P.M) {
+            P.y[size_t(t0) * P.N + n_out] = __float2bfloat16_rn(fmaf(d[nb][0], s0, b0));
+            P.y[size_t(t0) * P.N + n_out + 8] = __float2bfloat16_rn(fmaf(d[nb][2], s1, b1));
+          }
+          if (t0 + 1 < P.M) {
+            P.y[size_t(t0 + 1) * P.N + n_out] = __float2bfloat16_rn(fmaf(d[nb][1], s0, b0));
+            P.y[size_t(t0 + 1) * P.N + n_out + 8] = __float2bfloat16_rn(fmaf(d[nb][3], s1, b1));
+          }
+        }
       }
+      if (splits > 1) cluster_sync_relaxed();  // rank 0 has read every partial before they change
+      // The slots are rewritten by the next unit only after this barrier.
+      named_barrier_sync(1, kConsumerThreads);
+    } else if (splits > 1) {
+      cluster_sync();  // the producer warp takes part in every cluster rendezvous
+      cluster_sync_relaxed();
     }
   }
-  if (splits > 1) cluster_sync_relaxed();  // rank 0 has read every partial before any CTA exits
 }
 
+// Grid (splits, ctas): with splits > 1 one CTA per unit (ctas = units).
 template <int NT>
-static cudaError_t launch_nt(const Batch& batch, int splits, int slabs, cudaStream_t stream) {
+static cudaError_t launch_nt(const Batch& batch, int splits, int ctas, cudaStream_t stream) {
   using C = GemvCfg<NT>;
   static unsigned long long configured = 0;  // one bit per device ordinal
   int dev = 0;
@@ -299,7 +340,7 @@ static cudaError_t launch_nt(const Batch& batch, int splits, int slabs, cudaStre
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(splits), unsigned(slabs), 1);
+  cfg.gridDim = dim3(unsigned(splits), unsigned(ctas), 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
@@ -313,11 +354,12 @@ static cudaError_t launch_nt(const Batch& batch, int splits, int slabs, cudaStre
   return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<NT>, batch);
 }
 
-cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int slabs, cudaStream_t stream) {
-  if (splits < 1 || splits > 8 || slabs < 1 || slabs > 65535) return cudaErrorInvalidValue;
+cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream) {
+  if (splits < 1 || splits > 8 || ctas < 1 || ctas > 65535 || (splits > 1 && ctas < batch.total_units))
+    return cudaErrorInvalidValue;
   switch (nt) {
-    case 1: return launch_nt<1>(batch, splits, slabs, stream);
-    case 2: return launch_nt<2>(batch, splits, slabs, stream);
+    case 1: return launch_nt<1>(batch, splits, ctas, stream);
+    case 2: return launch_nt<2>(batch, splits, ctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }
