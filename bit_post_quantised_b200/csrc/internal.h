@@ -84,7 +84,7 @@ int max_active_clusters_2sm();
 // `splits` CTAs along k (splits > 1 needs ctas == total_units); problems use
 // n_tiles = N / 128 slabs, unit_begin = first slab in the launch,
 // chunks_per_split 64-k chunks per CTA and a 3-D x tensor map {64 k, M,
-// K / 64} whose box is {64, min(M, 8 nt), 8}.
+// K / 64} whose box is {64, min(M, 8 nt), 16 (nt = 1) or 8 chunks}.
 cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream);
 int max_active_clusters_2sm();
 int smem_bytes_2sm();

@@ -331,7 +331,7 @@ tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<in
     for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
       const tern_linear_args& a = args[idx[g]];
       Problem* p = &batch.p[n];
-      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, int(std::min<int64_t>(a.M, 8 * nt)), 8);
+      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, 8 * nt, nt == 1 ? 16 : 8);
       if (s != TERN_OK) return s;
       p->packed = static_cast<const uint8_t*>(a.packed);
       p->scales = a.scales;

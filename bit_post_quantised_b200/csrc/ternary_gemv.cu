@@ -48,18 +48,19 @@ namespace {
 template <int NT>
 struct GemvCfg {
   static constexpr int kGroups = 8;                  // 16-channel groups per 128-channel slab
-  // Consumer warps per group, splitting every stage's chunks round-robin.
-  // More warps hide more of the expansion's dependency latency; NT = 2 keeps
-  // two because its accumulators need the registers.
-  static constexpr int kSplit = 2;
-  static constexpr int kWarps = kSplit * kGroups;
-  static constexpr int kPerWarp = (8 + kSplit - 1) / kSplit;  // chunks per warp per stage (at most)
+  // One consumer warp per group: it takes every chunk of its 16 rows, so no
+  // warp ever waits for another (two warps per SM sub-partition already keep
+  // the expansion and the MMAs at full rate).
+  static constexpr int kWarps = kGroups;
   static constexpr int kThreads = (kWarps + 1) * 32;  // + one producer warp
-  static constexpr int kChunks = 8;                  // 64-k chunks per stage
-  static constexpr int kStages = 6;
+  // 64-k chunks per stage: 16 (32 KiB of codes) where shared memory allows,
+  // so the per-stage handshake is paid half as often.
+  static constexpr int kChunks = NT == 1 ? 16 : 8;
+  static constexpr int kStages = NT == 1 ? 4 : 6;
   static constexpr int kCodeBytes = kChunks * 2048;
-  static constexpr int kXBytes = kChunks * 8 * NT * 128;  // up to 8 NT token rows x 64 bf16 per chunk
-  static constexpr int kStageBytes = kCodeBytes + kXBytes + 1024;  // + slack: rows >= R read past the box
+  static constexpr int kXChunk = 8 * NT * 128;          // 8 NT token rows x 64 bf16 (rows >= M read as 0)
+  static constexpr int kXBytes = kChunks * kXChunk;
+  static constexpr int kStageBytes = kCodeBytes + kXBytes;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
   static_assert(kStageBytes % 1024 == 0 && kCodeBytes % 1024 == 0, "swizzled x boxes stay 1024-aligned");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -94,7 +95,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 // the next unit's codes while the consumers finish the current one).
 // blockIdx.x, the rank in the cluster, picks the k range of every unit
 // (chunks_per_split 64-k chunks).  The x tensor map is 3-D {64 k, M tokens,
-// K / 64 chunks} with box {64, min(M, 8 NT), 8}.
+// K / 64 chunks} with box {64, min(M, 8 NT), kChunks}.
 template <int NT>
 __device__ __forceinline__ const Problem& unit_problem(const Batch& batch, int u, int* slab) {
   int pi = 0;
@@ -108,12 +109,10 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     ternary_gemv_kernel(const __grid_constant__ Batch batch) {
   using C = GemvCfg<NT>;
   constexpr int S = C::kStages;
-  constexpr int kConsumerThreads = C::kWarps * 32;
 
   __shared__ __align__(8) uint64_t full_bar[S];   // codes and x of stage s landed
   __shared__ __align__(8) uint64_t empty_bar[S];  // all consumer warps are done with stage s
-  // Sums of the warps with half > 0 (one slot each), then the CTA's total.
-  __shared__ __align__(16) float part[(C::kSplit - 1) * C::kGroups * 32 * NT * 4];
+  __shared__ __align__(16) float part[C::kWarps * 32 * NT * 4];  // this CTA's sums, for rank 0
   extern __shared__ uint8_t dyn_smem[];
 
   const uint64_t lim = batch.wait_limit_ns;
@@ -140,7 +139,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     fence_proxy_async_smem();
   }
   __syncthreads();
-  const int grp = warp & (C::kGroups - 1), half = warp / C::kGroups;
+  const int grp = warp;  // 16-channel group of a consumer warp
 
   if (warp == C::kWarps) {
     // ------------------------------------------------------ producer
@@ -154,7 +153,6 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
       const int kc_total = P.K >> 6;
       const int kc0 = rank * P.chunks_per_split;
       const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
-      const int rows = min(P.M, 8 * NT);
       const uint8_t* codes = P.packed + (size_t(slab) * kc_total + kc0) * 2048;
       for (int i = 0; i * C::kChunks < nk; ++i, ++it) {
         const int s = it % S;
@@ -167,7 +165,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           const int nch = min(C::kChunks, nk - i * C::kChunks);
           const uint32_t stage = smem_base + s * C::kStageBytes;
           const uint32_t fb = smem_u32(&full_bar[s]);
-          mbar_arrive_expect_tx(fb, nch * 2048 + C::kChunks * rows * 128);
+          mbar_arrive_expect_tx(fb, nch * 2048 + C::kXBytes);
           tma_load_bulk(stage, codes + size_t(i) * C::kCodeBytes, nch * 2048, fb);
           tma_load_3d(stage + C::kCodeBytes, &P.tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
         }
@@ -181,6 +179,11 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   // Consumers walk the same units; all threads (producer included) meet at
   // the per-unit cluster rendezvous when K is split.
   const int g = lane >> 2, c = lane & 3;
+  // This lane's two 16-byte x pieces of a chunk: row g (and 8 + g, ... for
+  // the next n8 blocks), k = 16c .. 16c + 15, XOR-swizzled by the row (each
+  // chunk of the box is 8 NT rows of 128 bytes, so the swizzle row is g).
+  const uint32_t xoff_a = uint32_t(g * 128) + ((uint32_t(2 * c) ^ uint32_t(g)) << 4);
+  const uint32_t xoff_b = uint32_t(g * 128) + ((uint32_t(2 * c + 1) ^ uint32_t(g)) << 4);
   int it = 0;
   bool ok = true;
   for (int u = u0; u < units; u += ustep) {
@@ -194,9 +197,9 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     const int n_out = slab * 128 + grp * 16 + g;
     if (warp < C::kWarps) {
       // Scale and bias of this lane's two output channels, loaded now and used
-      // after the stream (only rank 0's first warps store).
+      // after the stream (only rank 0 stores).
       float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
-      if (half == 0 && rank == 0) {
+      if (rank == 0) {
         s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
         s1 = 0.5f * P.scales[n_out + 8];
         const uint16_t* bias = reinterpret_cast<const uint16_t*>(P.bias);
@@ -207,17 +210,9 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
       }
       const int kc_total = P.K >> 6;
       const int nk = max(0, min(kc_total, (rank + 1) * P.chunks_per_split) - rank * P.chunks_per_split);
-      const int rows = min(P.M, 8 * NT);
-      // Shared-memory offsets of this lane's two 16-byte x pieces in each of
-      // its chunks (line j * rows + g of the stage's x box, XOR-swizzled by
-      // the line index; the second n8 block is 8 lines = 1 KiB further).
-      uint32_t xoff_a[C::kPerWarp], xoff_b[C::kPerWarp];
+      bool xrow[NT];
 #pragma unroll
-      for (int t = 0; t < C::kPerWarp; ++t) {
-        const uint32_t line = uint32_t((half + C::kSplit * t) * rows + g);
-        xoff_a[t] = line * 128 + ((uint32_t(2 * c) ^ (line & 7)) << 4);
-        xoff_b[t] = line * 128 + ((uint32_t(2 * c + 1) ^ (line & 7)) << 4);
-      }
+      for (int nb = 0; nb < NT; ++nb) xrow[nb] = 8 * nb + g < P.M;
       float acc[4][NT][4];  // one accumulator per MMA position q: four independent chains
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -232,18 +227,23 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           break;
         }
         const int nch = min(C::kChunks, nk - i * C::kChunks);
-        const uint8_t* stage = smem_gen + s * C::kStageBytes;
-        const uint32_t xstage = smem_base + s * C::kStageBytes + C::kCodeBytes;
-        // Word c of rows 16 grp + g and 16 grp + g + 8 of chunks half,
-        // half + kSplit, ...: 128 contiguous bytes per warp load.
-        const uint32_t* cw = reinterpret_cast<const uint32_t*>(stage + half * 2048) + grp * 64 + lane;
-        const uint32_t xh = xstage;
-        auto chunk = [&](int t) {
-          const uint32_t a = cw[t * C::kSplit * 512], b = cw[t * C::kSplit * 512 + 32];
+        // Word c of rows 16 grp + g and 16 grp + g + 8 of each chunk: 128
+        // contiguous bytes per warp load.
+        const uint32_t* cw =
+            reinterpret_cast<const uint32_t*>(smem_gen + s * C::kStageBytes) + grp * 64 + lane;
+        const uint32_t xs = smem_base + s * C::kStageBytes + C::kCodeBytes;
+        auto chunk = [&](int j) {
+          const uint32_t a = cw[j * 512], b = cw[j * 512 + 32];
 #pragma unroll
           for (int nb = 0; nb < NT; ++nb) {
-            const uint4 xa = ld_shared_v4(xh + xoff_a[t] + nb * 1024);
-            const uint4 xb = ld_shared_v4(xh + xoff_b[t] + nb * 1024);
+            // Lanes of absent tokens skip their x loads (their MMA columns are
+            // never stored): at M = 1 this cuts the shared-memory reads of x,
+            // the largest ones of the loop, eightfold.
+            uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
+            if (xrow[nb]) {
+              xa = ld_shared_v4(xs + j * C::kXChunk + nb * 1024 + xoff_a);
+              xb = ld_shared_v4(xs + j * C::kXChunk + nb * 1024 + xoff_b);
+            }
             mma_16816(acc[0][nb], pm2_pair<0>(a), pm2_pair<0>(b), pm2_pair<1>(a), pm2_pair<1>(b), xa.x, xa.y);
             mma_16816(acc[1][nb], pm2_pair<2>(a), pm2_pair<2>(b), pm2_pair<3>(a), pm2_pair<3>(b), xa.z, xa.w);
             mma_16816(acc[2][nb], pm2_pair<4>(a), pm2_pair<4>(b), pm2_pair<5>(a), pm2_pair<5>(b), xb.x, xb.y);
@@ -252,11 +252,10 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
         };
         if (nch == C::kChunks) {  // every stage but a row's last: no bounds tests
 #pragma unroll
-          for (int t = 0; t < C::kPerWarp; ++t) chunk(t);
+          for (int j = 0; j < C::kChunks; ++j) chunk(j);
         } else {
-#pragma unroll
-          for (int t = 0; t < C::kPerWarp; ++t)
-            if (half + C::kSplit * t < nch) chunk(t);
+#pragma unroll 1
+          for (int j = 0; j < nch; ++j) chunk(j);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
@@ -266,33 +265,15 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           d[nb][e] = (acc[0][nb][e] + acc[1][nb][e]) + (acc[2][nb][e] + acc[3][nb][e]);
-      // The first warp of each group adds the others' sums in warp order.
-      if (half > 0) {
-        float* slot = &part[(((half - 1) * C::kGroups + grp) * 32 + lane) * NT * 4];
+      if (splits > 1) {
+        float* mine = &part[(grp * 32 + lane) * NT * 4];
 #pragma unroll
         for (int nb = 0; nb < NT; ++nb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) slot[nb * 4 + e] = d[nb][e];
-      }
-      named_barrier_sync(1, kConsumerThreads);
-      if (half == 0) {
-        for (int h = 1; h < C::kSplit; ++h) {
-          const float* slot = &part[(((h - 1) * C::kGroups + grp) * 32 + lane) * NT * 4];
-#pragma unroll
-          for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[nb][e] += slot[nb * 4 + e];
-        }
-        if (splits > 1) {  // this CTA's total, for rank 0 (the slot read above was this thread's own)
-          float* mine = &part[(grp * 32 + lane) * NT * 4];
-#pragma unroll
-          for (int nb = 0; nb < NT; ++nb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = d[nb][e];
-        }
+          for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = d[nb][e];  // this CTA's sums, for rank 0
       }
       if (splits > 1) cluster_sync();  // every rank's partial sums are in its shared memory
-      if (half == 0 && rank == 0) {
+      if (rank == 0) {
         if (splits > 1) {
           const uint32_t mine = smem_u32(&part[(grp * 32 + lane) * NT * 4]);
           for (int r = 1; r < splits; ++r)  // rank order: deterministic
@@ -316,8 +297,6 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
         }
       }
       if (splits > 1) cluster_sync_relaxed();  // rank 0 has read every partial before they change
-      // The slots are rewritten by the next unit only after this barrier.
-      named_barrier_sync(1, kConsumerThreads);
     } else if (splits > 1) {
       cluster_sync();  // the producer warp takes part in every cluster rendezvous
       cluster_sync_relaxed();
