@@ -74,8 +74,11 @@ struct Cfg2 {
   static constexpr int kTmemCols = 512;
   // A narrow tile makes the MMAs of a stage short, so decoding needs more warps.
   static constexpr int kDecWarps = TOK >= 256 ? 4 : 8;
-  static constexpr int kEpiWarps = 8;             // two per TMEM lane quarter, half the columns each
-  static constexpr int kEpiCols = TOK / 2;
+  // Epilogue warps: kEpiWarps / 4 per TMEM lane quarter, each draining
+  // kEpiCols accumulator columns.  The single accumulator of the 256-token
+  // tile is released sooner with more of them.
+  static constexpr int kEpiWarps = TOK >= 256 ? 16 : 8;
+  static constexpr int kEpiCols = TOK / (kEpiWarps / 4);
   static constexpr int kEpiWarp0 = 2 + kDecWarps;
   static constexpr int kThreads = (2 + kDecWarps + kEpiWarps) * 32;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
@@ -320,7 +323,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     constexpr int kCols = C::kEpiCols;
     const int ew = warp - C::kEpiWarp0;
     const int quarter = warp & 3;
-    const int half = ew >> 2;  // token columns [kCols * half, kCols * half + kCols)
+    const int half = ew >> 2;  // token columns [kCols * half, kCols * half + kCols) ("half" of 2 or 4)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t accempty_leader0 = T::leader_addr(smem_u32(&accempty_bar[0]));
