@@ -271,21 +271,33 @@ def workload_config(layer):
 
 
 # ------------------------------------------------------------ GPU arm
-def setup_dist(args):
+def setup_dist(backend: str = "nccl"):
+    """Rank layout from the torchrun environment; one process per GPU.  The
+    process group (NCCL on GPUs, gloo for the CPU tests of this logic) carries
+    only the barriers and the max-over-ranks of the timings: ranks are
+    independent replicas with no collective on the data path."""
     import torch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
 
         import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
+
+
+def _collective_device():
+    import torch
+    import torch.distributed as dist
+
+    return torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
 
 
 def barrier(world):
@@ -295,19 +307,28 @@ def barrier(world):
         import torch.distributed as dist
 
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(value: float, world: int) -> float:
+    """Largest of the ranks' values (every rank gets it): a multi-GPU time is
+    the slowest rank's."""
     import torch
 
     if world == 1:
         return value
     import torch.distributed as dist
 
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=_collective_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, steps: int, flop_per_step: float, elapsed_s: float) -> float:
+    """Whole-job TFLOP/s: every rank ran `steps` steps of `flop_per_step`
+    within `elapsed_s` (the max over ranks)."""
+    return world * steps * flop_per_step / elapsed_s / 1e12
 
 
 def make_sets(layer, rank, n_sets, device):
@@ -491,7 +512,7 @@ def run_tern(args):
 
     from bit_post_quantised_b200 import tern, workloads
 
-    world, rank, local = setup_dist(args)
+    world, rank, local = setup_dist("nccl")
     device = torch.device("cuda", local)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
@@ -566,7 +587,7 @@ def run_tern(args):
     e2e_elapsed = max_over_ranks(t0.elapsed_time(t1) * 1e-3, world)
 
     flop = layer.flop
-    value = world * K * flop / elapsed / 1e12
+    value = job_throughput(world, K, flop, elapsed)
     achieved = flop / t_lin / 1e12
     tensor_bound = flop / (peaks["bf16_tflops"] * 1e12) >= layer.algorithmic_bytes / (peaks["hbm_gbs"] * 1e9)
     kname, kstem = linear_kernel(layer)
@@ -589,7 +610,7 @@ def run_tern(args):
         "linear_us": t_lin * 1e6, "quantize_pack_us": t_quant * 1e6,
         "packed_weight_gbs": layer.packed_bytes / t_lin / 1e9,
         "quantize_pack_gbs": (2 * layer.N * layer.K + layer.packed_bytes + 4 * layer.N) / t_quant / 1e9,
-        "e2e": {"value": world * K * flop / e2e_elapsed / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_throughput(world, K, flop, e2e_elapsed), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K * world,
         "clocks": clocks.summary(),

@@ -162,6 +162,13 @@ def test_linear_pair_tiles_narrow(M, N, K):
     run_linear_case(M, N, K, seed=3 * M + N + K)
 
 
+def test_linear_pair_tiles_many_token_tiles():
+    """Token rows far past 2^16 with a single 256-wide channel slab: 128 token
+    tiles queued on fewer CTA pairs, each pair looping over several."""
+    run_linear_case(32768, 256, 128, seed=91)
+    run_linear_case(20001, 512, 64, seed=92)
+
+
 def test_linear_no_bias():
     run_linear_case(40, 256, 256, seed=3, with_bias=False)
     run_linear_case(257, 256, 256, seed=4, with_bias=False)
@@ -214,7 +221,12 @@ def test_linear_rejects_misaligned_pointer():
 
 # ---------------------------------------------------------------- batch
 def test_linear_batch_mixed_sizes():
-    cases = [(1, 256, 192), (16, 384, 256), (70, 128, 128), (300, 256, 320), (2, 512, 64), (130, 128, 576)]
+    # one or more problems of each launch group: GEMV M <= 8 and M <= 16,
+    # 64-token and 256-token CTA-pair tiles, and the single-CTA kernel for
+    # N % 256 != 0
+    cases = [(1, 256, 192), (16, 384, 256), (70, 128, 128), (300, 256, 320), (2, 512, 64), (130, 128, 576),
+             (40, 512, 256), (9, 256, 128), (64, 256, 3072), (600, 512, 192), (257, 768, 320),
+             (33, 384, 448)]
     probs, refs = [], []
     for i, (M, N, K) in enumerate(cases):
         W = rand_bf16((N, K), 0.02, 100 + i)
