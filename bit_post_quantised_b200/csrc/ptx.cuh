@@ -292,28 +292,98 @@ __device__ __forceinline__ void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols)
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-__device__ __forceinline__ void mma_bf16_ts_2sm(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
+// Commits issued, like mma_stage, by the lane elect.sync picks in a
+// converged warp (all 32 lanes call them): the mbarrier gets one arrival when
+// every tcgen05 op that lane issued so far is done.  The 2-SM multicast form
+// arrives at the same shared-memory offset in every CTA of `cta_mask`.
+__device__ __forceinline__ void mma_commit_elected(uint32_t bar) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
 }
-// Arrive once on the mbarrier at this shared-memory offset in every CTA of
-// `cta_mask` when all tcgen05 ops issued so far by this thread are done.
-__device__ __forceinline__ void mma_commit_2sm_multicast(uint32_t bar, uint16_t cta_mask) {
+__device__ __forceinline__ void mma_commit_2sm_multicast_elected(uint32_t bar, uint16_t cta_mask) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          bar),
-      "h"(cta_mask)
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}"
+      ::"r"(bar), "h"(cta_mask)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit_2sm(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+__device__ __forceinline__ void mma_commit_2sm_elected(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+      "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
 }
+
+// One 128-k stage of the tile kernels issued at once: NMMA k16 MMAs (8, or 4
+// for a 64-k tail) followed by two commits, all from the lane that elect.sync
+// picks in a converged warp (later commits covering these MMAs go through the
+// *_elected forms below, called by the same converged warp, so they come from
+// that lane too).  Every lane computes the same operands, so they stay
+// warp-uniform; issuing the same instructions from a single-lane branch with
+// per-MMA descriptor arithmetic was measured to take several times the MMA's
+// own duration at N = 64, and a lane-0 predicate instead of elect.sync ~13 %
+// longer per tile at N = 64.
+//   d        accumulator TMEM address
+//   a        TMEM column address of k16 step 0 of A; step j reads a + 8 j
+//   desc     shared-memory descriptor of B's step 0; step j adds 32 bytes
+//            (2 in the address field) inside a 64-k chunk, and `chunk2` (the
+//            second chunk's byte offset >> 4) for j >= 4
+//   acc      0 for the first stage of a tile (D = A B), else D += A B
+//   bar0/1   mbarriers the commits arrive on (PAIR: in both CTAs of the pair)
+#define TERN_STAGE_PROLOGUE                                            \
+  "{\n\t.reg .pred p, q, t;\n\t"                                      \
+  ".reg .b64 e1, e2, e3, e4, e5, e6, e7;\n\t"                         \
+  ".reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"                         \
+  "elect.sync _|p, 0xffffffff;\n\t"                                   \
+  "setp.ne.b32 q, %4, 0;\n\t"                                         \
+  "setp.eq.b32 t, 0, 0;\n\t"                                          \
+  "add.s64 e1, %2, 2;\n\t add.s64 e2, %2, 4;\n\t add.s64 e3, %2, 6;\n\t" \
+  "add.s64 e4, %2, %7;\n\t add.s64 e5, e4, 2;\n\t"                    \
+  "add.s64 e6, e4, 4;\n\t add.s64 e7, e4, 6;\n\t"                     \
+  "add.u32 a1, %1, 8;\n\t add.u32 a2, %1, 16;\n\t add.u32 a3, %1, 24;\n\t" \
+  "add.u32 a4, %1, 32;\n\t add.u32 a5, %1, 40;\n\t"                   \
+  "add.u32 a6, %1, 48;\n\t add.u32 a7, %1, 56;\n\t"
+#define TERN_STAGE_MMA(G, A, E, P) "@p tcgen05.mma.cta_group::" #G ".kind::f16 [%0], [" A "], " E ", %3, " P ";\n\t"
+#define TERN_STAGE_LO(G) \
+  TERN_STAGE_MMA(G, "%1", "%2", "q") TERN_STAGE_MMA(G, "a1", "e1", "t") \
+  TERN_STAGE_MMA(G, "a2", "e2", "t") TERN_STAGE_MMA(G, "a3", "e3", "t")
+#define TERN_STAGE_HI(G) \
+  TERN_STAGE_MMA(G, "a4", "e4", "t") TERN_STAGE_MMA(G, "a5", "e5", "t") \
+  TERN_STAGE_MMA(G, "a6", "e6", "t") TERN_STAGE_MMA(G, "a7", "e7", "t")
+#define TERN_COMMIT1(BAR) "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [" BAR "];\n\t"
+#define TERN_COMMIT2(BAR) \
+  "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [" BAR "], %8;\n\t"
+
+template <int NMMA, bool PAIR>
+__device__ __forceinline__ void mma_stage(uint32_t d, uint32_t a, uint64_t desc, uint32_t idesc, uint32_t acc,
+                                          uint32_t bar0, uint32_t bar1, uint64_t chunk2) {
+  static_assert(NMMA == 4 || NMMA == 8, "a stage is one or two 64-k chunks");
+  const uint16_t both = 0x3;  // commit multicast: both CTAs of the pair
+  if constexpr (!PAIR && NMMA == 8)
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(1) TERN_STAGE_HI(1) TERN_COMMIT1("%5") TERN_COMMIT1("%6") "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "l"(chunk2), "h"(both)
+                 : "memory");
+  else if constexpr (!PAIR)
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(1) TERN_COMMIT1("%5") TERN_COMMIT1("%6") "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "l"(chunk2), "h"(both)
+                 : "memory");
+  else if constexpr (NMMA == 8)
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(2) TERN_STAGE_HI(2) TERN_COMMIT2("%5") TERN_COMMIT2("%6") "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "l"(chunk2), "h"(both)
+                 : "memory");
+  else
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(2) TERN_COMMIT2("%5") TERN_COMMIT2("%6") "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "l"(chunk2), "h"(both)
+                 : "memory");
+}
+#undef TERN_STAGE_PROLOGUE
+#undef TERN_STAGE_MMA
+#undef TERN_STAGE_LO
+#undef TERN_STAGE_HI
+#undef TERN_COMMIT1
+#undef TERN_COMMIT2
 
 // Named barrier over a subset of the CTA's warps that also ANDs a predicate
 // across them (every participating thread gets the same answer).

@@ -26,7 +26,8 @@
 //   * warp 1 of the leader CTA (rank 0): waits afull[a] (eight arrivals, four
 //     from each CTA), issues the eight MMAs of the stage and commits, with
 //     one arrival in both CTAs, to empty[s] (shared-memory stage free) and
-//     aempty[a] (TMEM slot free).  Eight MMAs (1024 tensor cycles) between
+//     aempty[a] (TMEM slot free).  The whole warp computes the operands and
+//     lane 0 issues the stage as one block, so the operands stay uniform.  Eight MMAs (1024 tensor cycles) between
 //     two waits of the issuing thread keep the tensor pipe fed; a wait every
 //     four MMAs measurably starves it.
 //   * warps 6-13 (epilogue): after the tile's last MMA, tcgen05.ld of the
@@ -119,7 +120,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // The tcgen05 forms of a one-CTA tile (cta_group::1) or a CTA-pair tile
 // (cta_group::2: the leader's commits arrive in both CTAs, the other CTA's
-// warps arrive on the leader's barriers).
+// warps arrive on the leader's barriers).  The commits are called by the whole
+// converged MMA warp and issued by its elected lane, like the MMAs.
 template <bool PAIR>
 struct Tc;
 template <>
@@ -127,11 +129,8 @@ struct Tc<true> {
   static __device__ __forceinline__ void alloc(uint32_t dst, uint32_t n) { tmem_alloc_2sm(dst, n); }
   static __device__ __forceinline__ void relinquish() { tmem_relinquish_2sm(); }
   static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc_2sm(t, n); }
-  static __device__ __forceinline__ void mma(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    mma_bf16_ts_2sm(d, a, b, idesc, acc);
-  }
-  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit_2sm_multicast(bar, 0x3); }
-  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit_2sm(bar); }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit_2sm_multicast_elected(bar, 0x3); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit_2sm_elected(bar); }
   static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return mapa_shared(bar, 0); }
   static __device__ __forceinline__ void arrive_leader(uint32_t addr) { mbar_arrive_cluster(addr); }
   static __device__ __forceinline__ void sync_all() { cluster_sync(); }
@@ -141,11 +140,8 @@ struct Tc<false> {
   static __device__ __forceinline__ void alloc(uint32_t dst, uint32_t n) { tmem_alloc(dst, n); }
   static __device__ __forceinline__ void relinquish() { tmem_relinquish(); }
   static __device__ __forceinline__ void dealloc(uint32_t t, uint32_t n) { tmem_dealloc(t, n); }
-  static __device__ __forceinline__ void mma(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    mma_bf16_ts(d, a, b, idesc, acc);
-  }
-  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit(bar); }
-  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit(bar); }
+  static __device__ __forceinline__ void commit_all(uint32_t bar) { mma_commit_elected(bar); }
+  static __device__ __forceinline__ void commit_local(uint32_t bar) { mma_commit_elected(bar); }
   static __device__ __forceinline__ uint32_t leader_addr(uint32_t bar) { return bar; }
   static __device__ __forceinline__ void arrive_leader(uint32_t addr) { mbar_arrive(addr); }
   static __device__ __forceinline__ void sync_all() { __syncthreads(); }
@@ -240,6 +236,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer (leader)
+    const uint32_t tmem_u = __shfl_sync(0xffffffffu, tmem, 0);  // warp-uniform TMEM base
     if (rank == 0) {  // the leader issues for the pair
       int it = 0, lt = 0;
       bool ok = true;
@@ -249,30 +246,25 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         ok = __shfl_sync(0xffffffffu, mbar_wait(smem_u32(&accempty_bar[ab]), ((lt / AB) & 1) ^ 1, lim, st), 0);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + ab * C::kDCols;
+        const uint32_t d_tmem = tmem_u + ab * C::kDCols;
         for (int kc = 0; kc < kc_total; kc += 2, ++it) {
           const int s = it % S, a = it % A;
-          const int nmma = kc + 1 < kc_total ? 8 : 4;
           ok = __shfl_sync(0xffffffffu, mbar_wait(smem_u32(&afull_bar[a]), (it / A) & 1, lim, st), 0);
           if (!ok) break;
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t stage = smem_base + s * C::kStageBytes;
-            const uint32_t a_tmem = tmem + C::kACol0 + a * C::kACols;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (j < nmma)
-                T::mma(d_tmem, a_tmem + j * 8, sw128_kmajor_desc(stage + (j >> 2) * C::kXBox + (j & 3) * 32),
-                       C::kIdesc, (kc | j) != 0);
-            T::commit_all(smem_u32(&empty_bar[s]));
-            T::commit_all(smem_u32(&aempty_bar[a]));
-          }
-          __syncwarp();
+          // The whole warp computes the (uniform) operands; one lane issues.
+          const uint32_t a_tmem = tmem_u + C::kACol0 + a * C::kACols;
+          const uint64_t desc = sw128_kmajor_desc(smem_base + s * C::kStageBytes);
+          const uint32_t bar0 = smem_u32(&empty_bar[s]), bar1 = smem_u32(&aempty_bar[a]);
+          if (kc + 1 < kc_total)
+            mma_stage<8, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1, uint64_t(C::kXBox >> 4));
+          else
+            mma_stage<4, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1, uint64_t(C::kXBox >> 4));
         }
-        if (ok && lane == 0) T::commit_all(smem_u32(&accfull_bar[ab]));
+        if (ok) T::commit_all(smem_u32(&accfull_bar[ab]));  // converged warp: the issuing lane
         __syncwarp();
       }
-      if (lane == 0) T::commit_local(smem_u32(&drain_bar));
+      T::commit_local(smem_u32(&drain_bar));
       __syncwarp();
       mbar_wait(smem_u32(&drain_bar), 0, lim, st);
     }
