@@ -109,6 +109,7 @@ class ClockSampler:
         self.proc = None
         self.thread = None
         self.stop = False
+        self.ready = None
 
     def _nvml_loop(self, handle, nv):
         mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
@@ -119,6 +120,7 @@ class ClockSampler:
             except Exception:
                 break
             self.samples.append((float(sm), float(mx), {k for k, b in self.REASONS.items() if bits & b}))
+            self.ready.set()
             time.sleep(0.002)
 
     def __enter__(self):
@@ -130,8 +132,12 @@ class ClockSampler:
                       else nv.nvmlDeviceGetHandleByIndex(int(self.gpu)))
             import threading
 
+            self.ready = threading.Event()
             self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
             self.thread.start()
+            # a short timed region must not end before the sampler runs
+            self.ready.wait(2.0)
+            self.samples.clear()
         except Exception:
             self.thread = None
             try:
