@@ -96,12 +96,23 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 // blockIdx.x, the rank in the cluster, picks the k range of every unit
 // (chunks_per_split 64-k chunks).  The x tensor map is 3-D {64 k, M tokens,
 // K / 64 chunks} with box {64, min(M, 8 NT), kChunks}.
-template <int NT>
-__device__ __forceinline__ const Problem& unit_problem(const Batch& batch, int u, int* slab) {
+// The fields of a batch problem that the GEMV reads at every unit, copied
+// once to shared memory: reading them from the parameter block with a runtime
+// problem index measured ~0.5 us per unit boundary (each CTA walks several
+// units of a batch), shared-memory reads a few cycles.
+struct GemvProb {
+  const uint8_t* packed;
+  const float* scales;
+  const uint16_t* bias;
+  __nv_bfloat16* y;
+  int unit_begin, M, N, K, chunks_per_split;
+};
+
+__device__ __forceinline__ int unit_problem(const GemvProb* probs, int count, int u, int* slab) {
   int pi = 0;
-  while (pi + 1 < batch.count && u >= batch.p[pi + 1].unit_begin) ++pi;
-  *slab = u - batch.p[pi].unit_begin;
-  return batch.p[pi];
+  while (pi + 1 < count && u >= probs[pi + 1].unit_begin) ++pi;
+  *slab = u - probs[pi].unit_begin;
+  return pi;
 }
 
 template <int NT>
@@ -113,6 +124,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   __shared__ __align__(8) uint64_t full_bar[S];   // codes and x of stage s landed
   __shared__ __align__(8) uint64_t empty_bar[S];  // all consumer warps are done with stage s
   __shared__ __align__(16) float part[C::kWarps * 32 * NT * 4];  // this CTA's sums, for rank 0
+  __shared__ GemvProb probs[kMaxProblems];
   extern __shared__ uint8_t dyn_smem[];
 
   const uint64_t lim = batch.wait_limit_ns;
@@ -138,6 +150,20 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  if (threadIdx.x < batch.count) {
+    const Problem& q = batch.p[threadIdx.x];
+    GemvProb& g = probs[threadIdx.x];
+    g.packed = q.packed;
+    g.scales = q.scales;
+    g.bias = reinterpret_cast<const uint16_t*>(q.bias);
+    g.y = q.y;
+    g.unit_begin = q.unit_begin;
+    g.M = q.M;
+    g.N = q.N;
+    g.K = q.K;
+    g.chunks_per_split = q.chunks_per_split;
+  }
+  const int nprob = batch.count;
   __syncthreads();
   const int grp = warp;  // 16-channel group of a consumer warp
 
@@ -149,7 +175,8 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     bool ok = true;
     for (int u = u0; u < units && ok; u += ustep) {
       int slab;
-      const Problem& P = unit_problem<NT>(batch, u, &slab);
+      const int pi = unit_problem(probs, nprob, u, &slab);
+      const GemvProb& P = probs[pi];
       const int kc_total = P.K >> 6;
       const int kc0 = rank * P.chunks_per_split;
       const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
@@ -167,7 +194,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           const uint32_t fb = smem_u32(&full_bar[s]);
           mbar_arrive_expect_tx(fb, nch * 2048 + C::kXBytes);
           tma_load_bulk(stage, codes + size_t(i) * C::kCodeBytes, nch * 2048, fb);
-          tma_load_3d(stage + C::kCodeBytes, &P.tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
+          tma_load_3d(stage + C::kCodeBytes, &batch.p[pi].tmap_x, 0, 0, kc0 + i * C::kChunks, fb);
         }
         __syncwarp();
       }
@@ -188,7 +215,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   bool ok = true;
   for (int u = u0; u < units; u += ustep) {
     int slab;
-    const Problem& P = unit_problem<NT>(batch, u, &slab);
+    const GemvProb& P = probs[unit_problem(probs, nprob, u, &slab)];
     float d[NT][4];  // D fragments: channels (g, g + 8) x tokens (2c, 2c + 1) of each n8 block
 #pragma unroll
     for (int nb = 0; nb < NT; ++nb)
@@ -202,7 +229,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
       if (rank == 0) {
         s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
         s1 = 0.5f * P.scales[n_out + 8];
-        const uint16_t* bias = reinterpret_cast<const uint16_t*>(P.bias);
+        const uint16_t* bias = P.bias;
         if (bias) {
           b0 = bf16_bits_to_float(bias[n_out]);
           b1 = bf16_bits_to_float(bias[n_out + 8]);
