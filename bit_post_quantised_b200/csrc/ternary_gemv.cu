@@ -27,13 +27,13 @@
 //     and B = x is read in the same permuted order (8 contiguous bytes).
 //   * B = x^T for 8 tokens per n8 block (NT blocks: M <= 8 NT).
 // One CTA owns 128 channels (one tile-interleaved slab: each 64-k chunk is a
-// contiguous 2 KiB block) over a range of k.  Its sixteen consumer warps own
-// 16 channels each, two warps per channel group splitting every stage's
-// chunks (even / odd).  A producer lane streams stages of eight chunks into a
-// six-stage ring with two copies per stage: one 16 KiB bulk copy of codes and
-// one 3-D TMA box of the matching x rows (k-in-chunk x token x chunk, 128-byte
-// swizzle; only min(M, 8 NT) token rows are fetched -- the MMA columns of
-// absent tokens read stale shared memory and are never stored).  When there
+// contiguous 2 KiB block) over a range of k.  Its eight consumer warps own 16
+// channels each and take every chunk of their rows.  A producer lane streams
+// stages of sixteen chunks (M <= 8; eight for M <= 16) into a four- (six-)
+// stage ring with two copies per stage: one bulk copy of the codes (32 or 16
+// KiB) and one 3-D TMA box of the matching x rows (k-in-chunk x token x chunk,
+// 128-byte swizzle, 8 NT token rows; rows past M read as zero, and lanes of
+// absent tokens skip their x loads -- their MMA columns are never stored).  When there
 // are too few slabs to fill the SMs, the k range is split over a cluster of
 // CTAs, whose partial sums are added in rank order through distributed shared
 // memory (deterministic, no global scratch).  No TMA multicast is used.
