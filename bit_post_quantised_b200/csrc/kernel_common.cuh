@@ -36,6 +36,28 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t* out) {
   out[7] = bf16x2_sub((w2 & M1) ^ C1, C1);
 }
 
+// bf16x2 of 2t for the code pair J (k and k + 1) of a code word: shifted so
+// that the two bits of each half-word's code land on bits 15 and 14, a
+// two's-complement code is exactly the bf16 2t (0x4000 = 2, 0xC000 = -2,
+// 0 = 0), so a pair costs one shift and one AND (none for J = 7).  Sums of
+// 2t products are halved, exactly, with the scale.
+template <int J>
+__device__ __forceinline__ uint32_t code_pair_2t(uint32_t w) {
+  return (J == 7 ? w : (w << (14 - 2 * J))) & 0xC000C000u;
+}
+
+// The eight bf16x2 pairs of 2t of one code word, pair j = (k0 + 2j, k0 + 2j + 1).
+__device__ __forceinline__ void decode_word_2t(uint32_t w, uint32_t* out) {
+  out[0] = code_pair_2t<0>(w);
+  out[1] = code_pair_2t<1>(w);
+  out[2] = code_pair_2t<2>(w);
+  out[3] = code_pair_2t<3>(w);
+  out[4] = code_pair_2t<4>(w);
+  out[5] = code_pair_2t<5>(w);
+  out[6] = code_pair_2t<6>(w);
+  out[7] = code_pair_2t<7>(w);
+}
+
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
 // 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {

@@ -66,11 +66,6 @@ struct GemvCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-// bf16x2 of 2t for the code pair j (k and k + 1) of a code word.
-template <int J>
-__device__ __forceinline__ uint32_t pm2_pair(uint32_t w) {
-  return (w << (14 - 2 * J)) & 0xC000C000u;
-}
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -271,10 +266,14 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
               xa = ld_shared_v4(xs + j * C::kXChunk + nb * 1024 + xoff_a);
               xb = ld_shared_v4(xs + j * C::kXChunk + nb * 1024 + xoff_b);
             }
-            mma_16816(acc[0][nb], pm2_pair<0>(a), pm2_pair<0>(b), pm2_pair<1>(a), pm2_pair<1>(b), xa.x, xa.y);
-            mma_16816(acc[1][nb], pm2_pair<2>(a), pm2_pair<2>(b), pm2_pair<3>(a), pm2_pair<3>(b), xa.z, xa.w);
-            mma_16816(acc[2][nb], pm2_pair<4>(a), pm2_pair<4>(b), pm2_pair<5>(a), pm2_pair<5>(b), xb.x, xb.y);
-            mma_16816(acc[3][nb], pm2_pair<6>(a), pm2_pair<6>(b), pm2_pair<7>(a), pm2_pair<7>(b), xb.z, xb.w);
+            mma_16816(acc[0][nb], code_pair_2t<0>(a), code_pair_2t<0>(b), code_pair_2t<1>(a), code_pair_2t<1>(b),
+                      xa.x, xa.y);
+            mma_16816(acc[1][nb], code_pair_2t<2>(a), code_pair_2t<2>(b), code_pair_2t<3>(a), code_pair_2t<3>(b),
+                      xa.z, xa.w);
+            mma_16816(acc[2][nb], code_pair_2t<4>(a), code_pair_2t<4>(b), code_pair_2t<5>(a), code_pair_2t<5>(b),
+                      xb.x, xb.y);
+            mma_16816(acc[3][nb], code_pair_2t<6>(a), code_pair_2t<6>(b), code_pair_2t<7>(a), code_pair_2t<7>(b),
+                      xb.z, xb.w);
           }
         };
         if (nch == C::kChunks) {  // every stage but a row's last: no bounds tests

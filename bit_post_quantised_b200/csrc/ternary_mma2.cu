@@ -297,10 +297,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
           if (kc + sub < kc_total) {
             uint32_t t[32];
             const uint4 v = *reinterpret_cast<const uint4*>(cp + sub * C::kCSub);
-            decode_word(v.x, t + 0);
-            decode_word(v.y, t + 8);
-            decode_word(v.z, t + 16);
-            decode_word(v.w, t + 24);
+            decode_word_2t(v.x, t + 0);  // A holds 2t: the epilogue halves the scale
+            decode_word_2t(v.y, t + 8);
+            decode_word_2t(v.z, t + 16);
+            decode_word_2t(v.w, t + 24);
             tmem_st32(dst + sub * 32, t);
           }
         }
@@ -325,7 +325,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const Problem& P = *t.P;
       const int ab = lt % AB;
       const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
-      const float sc = P.scales[n];
+      const float sc = 0.5f * P.scales[n];  // A held 2t
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
       tc_fence_after();
