@@ -21,6 +21,11 @@ Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
 * ``pack_tiled / unpack_tiled`` -- the tile-interleaved device layout.
 * ``linear(x_bits, T, s, b_bits)`` -- ``y = s * (x @ T^T) + b`` in double
   (Section 4: activations are not quantised).
+* ``gelu_tanh(y, col0)``, ``linear_act(...)`` -- the tanh form of GELU on
+  output columns [col0, N), the activation a fused epilogue of the MLP's
+  first linear applies.  The pages quantise every linear of FLUX's blocks
+  (Section 3.1) but do not describe the operations between them; this is
+  FLUX.1's MLP activation, written from its definition.
 
 bf16 tensors are passed as their raw uint16 bit patterns.
 """
@@ -69,6 +74,7 @@ def _load():
         lib.oracle_unpack_tiled.argtypes = [_ptr, _i64, _i64, _ptr]
         lib.oracle_unpack_tiled.restype = ctypes.c_int
         lib.oracle_linear.argtypes = [_ptr, _i64, _i64, _ptr, _ptr, _ptr, _i64, _ptr]
+        lib.oracle_gelu_tanh.argtypes = [_ptr, _i64, _i64, _i64]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -185,3 +191,33 @@ def linear(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None) -> np.
     y = np.empty((M, N), np.float64)
     _load().oracle_linear(_p(x_bits), M, K, _p(T), _p(s), bp, N, _p(y))
     return y
+
+
+ACT_NONE = 0
+ACT_GELU_TANH = 1
+
+
+def gelu_tanh(y: np.ndarray, col0: int = 0) -> np.ndarray:
+    """The tanh form of GELU on columns [col0, N) of a float64 [M, N] array
+    (a new array; columns below col0 unchanged):
+    g(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))."""
+    y = np.array(y, dtype=np.float64, order="C", copy=True)
+    if y.ndim != 2:
+        raise ValueError("y must be [M, N]")
+    M, N = y.shape
+    if not 0 <= col0 <= N:
+        raise ValueError("col0 out of range")
+    _load().oracle_gelu_tanh(_p(y), M, N, col0)
+    return y
+
+
+def linear_act(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, act: int = ACT_NONE,
+               col0: int = 0) -> np.ndarray:
+    """``linear`` followed by the activation ``act`` on output columns
+    [col0, N): the layer with a fused epilogue, in float64."""
+    y = linear(x_bits, T, s, b_bits)
+    if act == ACT_NONE:
+        return y
+    if act == ACT_GELU_TANH:
+        return gelu_tanh(y, col0)
+    raise ValueError("unknown activation")

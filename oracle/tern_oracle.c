@@ -194,6 +194,21 @@ void oracle_linear(const uint16_t *x, int64_t M, int64_t K, const int8_t *T,
     }
 }
 
+/* The tanh form of GELU, applied in place to columns [col0, N) of y [M, N]:
+ *     g(v) = 0.5 * v * (1 + tanh(sqrt(2/pi) * (v + 0.044715 * v^3))).
+ * The pages quantise the linears of FLUX's transformer blocks (Section 3.1)
+ * but do not describe the operations around them; FLUX.1's MLP applies this
+ * activation to the output of its first linear, which is what a fused
+ * epilogue of that linear computes.  Written from the definition, in double. */
+void oracle_gelu_tanh(double *y, int64_t M, int64_t N, int64_t col0) {
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = col0; n < N; ++n) {
+            const double v = y[m * N + n];
+            y[m * N + n] = 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+        }
+}
+
 /* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -299,3 +299,56 @@ def test_storage_ratio_matches_pages():
     assert round(ratio, 1) == 7.7
     # without the per-channel scales and the 0.5% kept in 16 bit it would be 8x
     assert 16 / 2 == 8.0
+
+
+# ------------------------------------------------- fused GELU epilogue (tanh form)
+# Pins of oracle.gelu_tanh that do not retype its formula: an exact symmetry,
+# the Taylor coefficients at 0 (which fix sqrt(2/pi) and 0.044715), the
+# limits, and torch's own implementation of the same activation.
+
+def test_gelu_tanh_symmetry_and_limits():
+    rng = np.random.default_rng(7)
+    v = rng.normal(0.0, 3.0, size=(4, 257))
+    g, gm = oracle.gelu_tanh(v), oracle.gelu_tanh(-v)
+    # g(v) - g(-v) = v: 0.5 v (1 + t) + 0.5 v (1 - t) with t odd in v
+    assert np.allclose(g - gm, v, rtol=0, atol=1e-12)
+    big = np.array([[10.0, 20.0, 40.0]])
+    assert np.array_equal(oracle.gelu_tanh(big), big)
+    assert np.all(np.abs(oracle.gelu_tanh(-big)) < 1e-15)
+    assert oracle.gelu_tanh(np.zeros((1, 3))).tolist() == [[0.0, 0.0, 0.0]]
+
+
+def test_gelu_tanh_taylor_coefficients_at_zero():
+    # even part (g(h) + g(-h)) / 2 = (c/2) h^2 + (c a - c^3/3)/2 h^4 + O(h^6),
+    # c = sqrt(2/pi), a = 0.044715
+    c, a = np.sqrt(2.0 / np.pi), 0.044715
+    h1, h2 = 1e-2, 2e-2
+    e = lambda h: 0.5 * (oracle.gelu_tanh(np.array([[h]]))[0, 0] + oracle.gelu_tanh(np.array([[-h]]))[0, 0])
+    # eliminate the h^4 term from two step sizes: c2 = (16 e(h1) - e(h2)) / (12 h1^2)
+    c2 = (16 * e(h1) - e(h2)) / (12 * h1 * h1)
+    assert abs(c2 - c / 2) < 1e-9
+    # and the h^4 coefficient from the same two steps: e(h)/h^2 = c2 + c4 h^2 + O(h^4)
+    c4 = (e(h2) / h2 ** 2 - e(h1) / h1 ** 2) / (h2 ** 2 - h1 ** 2)
+    assert abs(c4 - 0.5 * (c * a - c ** 3 / 3)) < 1e-5
+
+
+def test_gelu_tanh_matches_torch():
+    v = torch.linspace(-12, 12, 4801, dtype=torch.float64).reshape(1, -1)
+    ref = torch.nn.functional.gelu(v, approximate="tanh").numpy()
+    assert np.allclose(oracle.gelu_tanh(v.numpy()), ref, rtol=1e-13, atol=1e-15)
+
+
+def test_linear_act_touches_only_columns_from_col0():
+    rng = np.random.default_rng(3)
+    M, K, N = 3, 64, 256
+    x = workloads.bf16_bits(torch.randn(M, K).to(torch.bfloat16))
+    T = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    s = rng.uniform(0.01, 0.03, size=N)
+    b = workloads.bf16_bits((torch.randn(N) * 0.01).to(torch.bfloat16))
+    y = oracle.linear(x, T, s, b)
+    ya = oracle.linear_act(x, T, s, b, oracle.ACT_GELU_TANH, 128)
+    assert np.array_equal(ya[:, :128], y[:, :128])
+    assert np.array_equal(ya[:, 128:], oracle.gelu_tanh(y[:, 128:]))
+    assert np.array_equal(oracle.linear_act(x, T, s, b, oracle.ACT_NONE, 0), y)
+    with pytest.raises(ValueError):
+        oracle.linear_act(x, T, s, b, 7, 0)
