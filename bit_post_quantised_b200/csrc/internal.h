@@ -21,6 +21,8 @@ struct alignas(64) Problem {
   int n_tiles, m_tiles, splits;
   int chunks_per_split;     // 64-wide k chunks per split
   int unit_begin;            // first work unit (CTA, or 2-SM tile) of this problem
+  int act;                   // epilogue activation (kActNone / kActGeluTanh)
+  int act_col0;              // first output column the activation applies to
 };
 
 constexpr int kMaxProblems = 15;  // keeps the kernel parameter block under 4 KiB

@@ -70,6 +70,27 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+// Epilogue activations (the values of tern_act in tern.h).
+constexpr int kActNone = 0;
+constexpr int kActGeluTanh = 1;
+
+// The tanh form of GELU, g(v) = 0.5 v (1 + tanh(u)), u = sqrt(2/pi) (v +
+// 0.044715 v^3), evaluated as v / (1 + e^(-2u)) (the same function, since
+// 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u))): no cancellation for large negative
+// v, where 1 + tanh(u) would lose its digits.  fp32, a few ulp.
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+  // e^(-2u) overflows to +inf for u < -44: the quotient is then 0 (as the
+  // true value, |g| < 1e-37, rounds to in bf16).
+  return __fdividef(v, 1.0f + __expf(-2.0f * u));
+}
+
+// y = v or act(v) for output channel n, given the problem's activation and
+// its first activated column.
+__device__ __forceinline__ float apply_act(float v, int act, int n, int act_col0) {
+  return (act == kActGeluTanh && n >= act_col0) ? gelu_tanh(v) : v;
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(uint32_t(b) << 16);
 }

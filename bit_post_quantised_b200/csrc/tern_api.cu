@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "kernel_common.cuh"
 #include "ptx.cuh"
 #include "tern.h"
 
@@ -219,6 +220,26 @@ tern_status check_linear(const tern_linear_args& a) {
   return TERN_OK;
 }
 
+static_assert(kActNone == TERN_ACT_NONE && kActGeluTanh == TERN_ACT_GELU_TANH, "kernel and ABI activation codes");
+
+// Epilogue activation of one problem (TERN_ACT_NONE for the plain layer).
+struct ActSpec {
+  int act = TERN_ACT_NONE;
+  int64_t col0 = 0;
+};
+
+tern_status check_act(int act, int64_t col0, int64_t N) {
+  if (act != TERN_ACT_NONE && act != TERN_ACT_GELU_TANH) return fail(TERN_ERR_INVALID_ARG, "unknown activation %d", act);
+  if (col0 < 0 || col0 > N)
+    return fail(TERN_ERR_INVALID_ARG, "act_col0=%lld outside [0, N=%lld]", (long long)col0, (long long)N);
+  return TERN_OK;
+}
+
+void set_act(Problem* p, const ActSpec* acts, int i) {
+  p->act = acts ? acts[i].act : TERN_ACT_NONE;
+  p->act_col0 = acts ? int(acts[i].col0) : 0;
+}
+
 // Up to 16 tokens run on the register-fed GEMV kernel, in n8 blocks.
 constexpr int64_t kGemvMaxM = 16;
 int gemv_nt(int64_t M) { return M <= 8 ? 1 : 2; }
@@ -292,8 +313,8 @@ tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int
 
 // Launches the problems `idx` of `args` (all with pair_tok == tok) on the
 // pair-tile kernel, up to kMaxProblems per launch.
-tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int>& idx, int tok, Batch& batch,
-                             const DeviceState* ds, cudaStream_t cs) {
+tern_status launch_2sm_group(const tern_linear_args* args, const ActSpec* acts, const std::vector<int>& idx, int tok,
+                             Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
     int64_t total = 0;
@@ -302,6 +323,7 @@ tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int
       int64_t tiles = 0;
       tern_status s = fill_problem_2sm(args[idx[g]], tok, &batch.p[n], &tiles);
       if (s != TERN_OK) return s;
+      set_act(&batch.p[n], acts, idx[g]);
       batch.p[n].unit_begin = int(total);
       total += tiles;
       if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
@@ -321,8 +343,8 @@ tern_status launch_2sm_group(const tern_linear_args* args, const std::vector<int
 // Launches the problems `idx` of `args` (all with M <= 8 nt) on the GEMV
 // kernel, up to kMaxProblems per launch.  K is split over a cluster of up to
 // eight CTAs when the launch has fewer 128-channel slabs than the GPU has SMs.
-tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<int>& idx, int nt, Batch& batch,
-                              const DeviceState* ds, cudaStream_t cs) {
+tern_status launch_gemv_group(const tern_linear_args* args, const ActSpec* acts, const std::vector<int>& idx, int nt,
+                              Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
     int64_t slabs = 0;
@@ -342,6 +364,7 @@ tern_status launch_gemv_group(const tern_linear_args* args, const std::vector<in
       p->K = int(a.K);
       p->n_tiles = int(a.N / 128);
       p->m_tiles = 1;
+      set_act(p, acts, idx[g]);
       p->unit_begin = int(slabs);
       slabs += a.N / 128;
       min_chunks = std::min<int64_t>(min_chunks, a.K / 64);
@@ -404,12 +427,16 @@ tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float e
   return TERN_OK;
 }
 
-tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
-                        const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
-                        tern_stream_t stream) {
-  const tern_linear_args a{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K};
+}  // extern "C"
+
+namespace tern {
+namespace {
+
+tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stream_t stream) {
+  const int64_t M = a.M, N = a.N, K = a.K;
   tern_status s = check_linear(a);
   if (s != TERN_OK) return s;
+  if ((s = check_act(act.act, act.col0, N)) != TERN_OK) return s;
   if (M == 0) return TERN_OK;
   int dev;
   DeviceState* ds;
@@ -420,13 +447,13 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
     static Batch batch_g;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch_g_mu;
     std::lock_guard<std::mutex> lock(batch_g_mu);
-    return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
+    return launch_gemv_group(&a, &act, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
   }
   if (const int ptok = pair_tok(a, ds)) {
     static Batch batch2;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch2_mu;
     std::lock_guard<std::mutex> lock(batch2_mu);
-    return launch_2sm_group(&a, std::vector<int>{0}, ptok, batch2, ds, cs);
+    return launch_2sm_group(&a, &act, std::vector<int>{0}, ptok, batch2, ds, cs);
   }
   const int tok = pick_tok(M);
   int splits = 1;
@@ -444,6 +471,7 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
   int64_t ctas = 0;
   if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;
   Problem& p = batch.p[0];
+  set_act(&p, &act, 0);
   if (p.splits > 1) {
     const size_t ws_bytes = size_t(p.splits) * size_t(tiles) * tok * 128 * sizeof(float);
     if ((s = get_workspace(dev, cs, ws_bytes, size_t(tiles), &p.ws, &p.counters)) != TERN_OK) return s;
@@ -458,10 +486,10 @@ tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* pa
   return TERN_OK;
 }
 
-tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream) {
-  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+tern_status batch_impl(const tern_linear_args* args, const ActSpec* acts, int count, tern_stream_t stream) {
   for (int i = 0; i < count; ++i) {
     tern_status s = check_linear(args[i]);
+    if (s == TERN_OK && acts) s = check_act(acts[i].act, acts[i].col0, args[i].N);
     if (s != TERN_OK) {
       t_last_error = "problem " + std::to_string(i) + ": " + t_last_error;
       return s;
@@ -481,13 +509,13 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
       if (args[i].M > 0 && args[i].M <= kGemvMaxM && gemv_nt(args[i].M) == nt) group.push_back(i);
-    if ((s = launch_gemv_group(args, group, nt, batch, ds, cs)) != TERN_OK) return s;
+    if ((s = launch_gemv_group(args, acts, group, nt, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int ptok : {64, 256}) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
       if (args[i].M > 0 && pair_tok(args[i], ds) == ptok) group.push_back(i);
-    if ((s = launch_2sm_group(args, group, ptok, batch, ds, cs)) != TERN_OK) return s;
+    if ((s = launch_2sm_group(args, acts, group, ptok, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int tok : kTokTiles) {
     std::vector<int> group;
@@ -500,6 +528,7 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
       for (size_t g = g0; g < group.size() && n < kMaxProblems; ++g, ++n) {
         int64_t ctas = 0;
         if ((s = fill_problem(args[group[g]], tok, 1, &batch.p[n], &ctas)) != TERN_OK) return s;
+        set_act(&batch.p[n], acts, group[g]);
         batch.p[n].unit_begin = int(total);
         total += ctas;
         if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
@@ -513,6 +542,43 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
     }
   }
   return TERN_OK;
+}
+
+}  // namespace
+}  // namespace tern
+
+extern "C" {
+
+tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                        const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                        tern_stream_t stream) {
+  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, ActSpec{}, stream);
+}
+
+tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                            const float* scales, const void* bias_bf16, int64_t N, int act, int64_t act_col0,
+                            void* y_bf16, tern_stream_t stream) {
+  ActSpec spec;
+  spec.act = act;
+  spec.col0 = act_col0;
+  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, spec, stream);
+}
+
+tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream) {
+  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+  return batch_impl(args, nullptr, count, stream);
+}
+
+tern_status tern_linear_batch_act(const tern_linear_act_args* args, int count, tern_stream_t stream) {
+  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+  std::vector<tern_linear_args> lin(size_t(std::max(count, 0)));
+  std::vector<ActSpec> acts(size_t(std::max(count, 0)));
+  for (int i = 0; i < count; ++i) {
+    lin[i] = args[i].linear;
+    acts[i].act = args[i].act;
+    acts[i].col0 = args[i].act_col0;
+  }
+  return batch_impl(lin.data(), acts.data(), count, stream);
 }
 
 tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,
@@ -650,8 +716,9 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
   // Neither the small-M GEMV nor the pair-tile kernel needs scratch.
-  if (M <= kGemvMaxM) return launch_gemv_group(&a, std::vector<int>{0}, gemv_nt(M), batch, ds, cs);
-  if (const int ptok = pair_tok(a, ds)) return launch_2sm_group(&a, std::vector<int>{0}, ptok, batch, ds, cs);
+  if (M <= kGemvMaxM) return launch_gemv_group(&a, nullptr, std::vector<int>{0}, gemv_nt(M), batch, ds, cs);
+  if (const int ptok = pair_tok(a, ds))
+    return launch_2sm_group(&a, nullptr, std::vector<int>{0}, ptok, batch, ds, cs);
 
   // Same tile and split choice as tern_linear, so the two give identical y.
   const int tok = pick_tok(M);

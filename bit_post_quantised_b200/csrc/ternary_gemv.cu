@@ -101,6 +101,7 @@ struct GemvProb {
   const uint16_t* bias;
   __nv_bfloat16* y;
   int unit_begin, M, N, K, chunks_per_split;
+  int act, act_col0;  // epilogue activation and its first column
 };
 
 __device__ __forceinline__ int unit_problem(const GemvProb* probs, int count, int u, int* slab) {
@@ -157,6 +158,8 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     g.N = q.N;
     g.K = q.K;
     g.chunks_per_split = q.chunks_per_split;
+    g.act = q.act;
+    g.act_col0 = q.act_col0;
   }
   const int nprob = batch.count;
   __syncthreads();
@@ -313,12 +316,16 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
         for (int nb = 0; nb < NT; ++nb) {
           const int t0 = 8 * nb + 2 * c;
           if (t0 < P.M) {
-            P.y[size_t(t0) * P.N + n_out] = __float2bfloat16_rn(fmaf(d[nb][0], s0, b0));
-            P.y[size_t(t0) * P.N + n_out + 8] = __float2bfloat16_rn(fmaf(d[nb][2], s1, b1));
+            P.y[size_t(t0) * P.N + n_out] =
+                __float2bfloat16_rn(apply_act(fmaf(d[nb][0], s0, b0), P.act, n_out, P.act_col0));
+            P.y[size_t(t0) * P.N + n_out + 8] =
+                __float2bfloat16_rn(apply_act(fmaf(d[nb][2], s1, b1), P.act, n_out + 8, P.act_col0));
           }
           if (t0 + 1 < P.M) {
-            P.y[size_t(t0 + 1) * P.N + n_out] = __float2bfloat16_rn(fmaf(d[nb][1], s0, b0));
-            P.y[size_t(t0 + 1) * P.N + n_out + 8] = __float2bfloat16_rn(fmaf(d[nb][3], s1, b1));
+            P.y[size_t(t0 + 1) * P.N + n_out] =
+                __float2bfloat16_rn(apply_act(fmaf(d[nb][1], s0, b0), P.act, n_out, P.act_col0));
+            P.y[size_t(t0 + 1) * P.N + n_out + 8] =
+                __float2bfloat16_rn(apply_act(fmaf(d[nb][3], s1, b1), P.act, n_out + 8, P.act_col0));
           }
         }
       }

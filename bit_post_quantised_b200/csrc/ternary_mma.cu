@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = row0 + c0 + j;
-          if (m < M) P.y[size_t(m) * N + n] = __float2bfloat16_rn(fmaf(__uint_as_float(v[j]), sc, bi));
+          if (m < M)
+            P.y[size_t(m) * N + n] =
+                __float2bfloat16_rn(apply_act(fmaf(__uint_as_float(v[j]), sc, bi), P.act, n, P.act_col0));
         }
       }
     } else {
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
           float acc = 0.f;
           for (int sp = 0; sp < P.splits; ++sp)
             acc += __ldcg(P.ws + ((size_t(sp) * tiles + tile) * TOK + c) * 128 + r);
-          P.y[size_t(m) * N + n] = __float2bfloat16_rn(fmaf(acc, sc, bi));
+          P.y[size_t(m) * N + n] = __float2bfloat16_rn(apply_act(fmaf(acc, sc, bi), P.act, n, P.act_col0));
         }
         if (dw == 0 && lane == 0) P.counters[tile] = 0;  // ready for the next launch
       }

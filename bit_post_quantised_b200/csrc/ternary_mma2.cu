@@ -326,23 +326,44 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const int ab = lt % AB;
       const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
       const float sc = 0.5f * P.scales[n];  // A held 2t
+      const bool gelu = P.act == kActGeluTanh && n >= P.act_col0;
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
       tc_fence_after();
       uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
+      if (__any_sync(0xffffffffu, gelu)) {
+        // The activation's transcendentals run after the accumulator is
+        // released, so they overlap the next tile's MMAs: keep y in fp32.
+        float f[kCols];
 #pragma unroll
-      for (int c0 = 0; c0 < kCols; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < kCols; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          out[c0 / 2 + j] = pack_bf16x2(fmaf(__uint_as_float(v[2 * j]), sc, bi),
-                                        fmaf(__uint_as_float(v[2 * j + 1]), sc, bi));
+          for (int j = 0; j < 32; ++j) f[c0 + j] = fmaf(__uint_as_float(v[j]), sc, bi);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+#pragma unroll
+        for (int j = 0; j < kCols / 2; ++j)
+          out[j] = gelu ? pack_bf16x2(gelu_tanh(f[2 * j]), gelu_tanh(f[2 * j + 1])) : pack_bf16x2(f[2 * j], f[2 * j + 1]);
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            out[c0 / 2 + j] = pack_bf16x2(fmaf(__uint_as_float(v[2 * j]), sc, bi),
+                                          fmaf(__uint_as_float(v[2 * j + 1]), sc, bi));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
       const int row0 = t.m_tile * C::kTokPair + half * kCols;
       const int rows = min(kCols, P.M - row0);
       uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;

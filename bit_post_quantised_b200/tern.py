@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
                 -6: "TERN_ERR_NO_DEVICE"}
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
-            "tern_linear_batch",
+            "tern_linear_act", "tern_linear_batch", "tern_linear_batch_act",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -39,6 +39,15 @@ class LinearArgs(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("y", ctypes.c_void_p),
                 ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+class LinearActArgs(ctypes.Structure):
+    """Mirror of tern_linear_act_args."""
+    _fields_ = [("linear", LinearArgs), ("act", ctypes.c_int), ("act_col0", ctypes.c_int64)]
+
+
+ACT_NONE = 0       # tern_act values
+ACT_GELU_TANH = 1
 
 
 def library_path() -> str:
@@ -63,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.tern_linear_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
         L.tern_linear_noalloc.restype = st
         L.tern_linear_batch.argtypes = [ctypes.POINTER(LinearArgs), ctypes.c_int, vp]
+        L.tern_linear_act.argtypes = [vp, i64, i64, vp, vp, vp, i64, ctypes.c_int, i64, vp, vp]
+        L.tern_linear_act.restype = st
+        L.tern_linear_batch_act.argtypes = [ctypes.POINTER(LinearActArgs), ctypes.c_int, vp]
+        L.tern_linear_batch_act.restype = st
         L.tern_linear_batch.restype = st
         L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
         L.tern_dequantize.restype = st
@@ -148,6 +161,34 @@ def linear_batch(problems: Sequence[dict], stream=None) -> None:
                             None if p.get("bias") is None else p["bias"].data_ptr(),
                             p["y"].data_ptr(), M, N, K)
     _check(lib().tern_linear_batch(arr, len(problems), _stream(stream)))
+
+
+def linear_act(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+               bias: Optional[torch.Tensor] = None, act: int = ACT_GELU_TANH, act_col0: int = 0,
+               out: Optional[torch.Tensor] = None, stream=None):
+    """tern_linear_act: the linear with `act` fused into its epilogue on
+    output columns [act_col0, N)."""
+    M, K = x.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().tern_linear_act(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, act, act_col0,
+                                 _ptr(out), _stream(stream)))
+    return out
+
+
+def linear_batch_act(problems: Sequence[dict], stream=None) -> None:
+    """tern_linear_batch_act over dicts as linear_batch's plus act (default
+    none) and act_col0 (default 0)."""
+    arr = (LinearActArgs * max(1, len(problems)))()
+    for i, p in enumerate(problems):
+        M, K = p["x"].shape
+        N = p["scales"].shape[0]
+        arr[i] = LinearActArgs(LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
+                                          None if p.get("bias") is None else p["bias"].data_ptr(),
+                                          p["y"].data_ptr(), M, N, K),
+                               p.get("act", ACT_NONE), p.get("act_col0", 0))
+    _check(lib().tern_linear_batch_act(arr, len(problems), _stream(stream)))
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional[torch.Tensor] = None,

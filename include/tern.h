@@ -135,6 +135,32 @@ TERN_API tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_t 
                                 const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
                                 tern_stream_t stream);
 
+/* Activations a fused epilogue applies (tern_linear_act, tern_linear_batch_act). */
+typedef enum {
+  TERN_ACT_NONE = 0,      /* the plain layer */
+  TERN_ACT_GELU_TANH = 1  /* g(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))) */
+} tern_act;
+
+/*
+ * tern_linear with an activation fused into the kernel's epilogue:
+ *     y[m,n] = act(s_n * sum_k x[m,k] * T[n,k] + b_n)   for n >= act_col0,
+ *     y[m,n] =     s_n * sum_k x[m,k] * T[n,k] + b_n    for n <  act_col0,
+ * with act applied to the fp32 value before its one rounding to bf16.
+ *   act       a tern_act value; TERN_ACT_NONE gives exactly tern_linear.
+ *   act_col0  first activated output column, 0 <= act_col0 <= N (FLUX's
+ *             single blocks compute q, k, v and the MLP's first projection in
+ *             one linear and activate only the MLP part).
+ * Other arguments, routing and errors as tern_linear; an unknown act or an
+ * act_col0 outside [0, N] returns TERN_ERR_INVALID_ARG.  The pages quantise
+ * every linear of FLUX's transformer blocks (Section 3.1) but do not describe
+ * the operations between them: fusing the activation of FLUX.1's MLP into its
+ * first linear is an interface choice of this library, saving one read and
+ * one write of that linear's output.
+ */
+TERN_API tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, const void* packed,
+                            const float* scales, const void* bias_bf16, int64_t N, int act,
+                            int64_t act_col0, void* y_bf16, tern_stream_t stream);
+
 /* One independent linear problem of a batch (same meaning as tern_linear). */
 typedef struct {
   const void* x;      /* [M, K] bf16 */
@@ -155,6 +181,16 @@ typedef struct {
  * workspace (only the single-call path for 16 < M <= 64 splits K into one).
  */
 TERN_API tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream);
+
+/* One problem of tern_linear_batch_act: a linear and its epilogue activation. */
+typedef struct {
+  tern_linear_args linear;
+  int act;          /* tern_act */
+  int64_t act_col0; /* first activated output column */
+} tern_linear_act_args;
+
+/* tern_linear_batch with a per-problem epilogue activation (as tern_linear_act). */
+TERN_API tern_status tern_linear_batch_act(const tern_linear_act_args* args, int count, tern_stream_t stream);
 
 /*
  * Expands packed codes to the dequantised bf16 weight W'[n,k] = T[n,k] * s_n

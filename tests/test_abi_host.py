@@ -135,3 +135,33 @@ def test_binding_fails_loudly_without_library(tmp_path):
 
 def test_linear_with_no_tokens_is_a_host_noop(L):
     assert call_linear(L, M=0, x=0, y=0) == OK
+
+
+def test_linear_act_rejects_on_host(L):
+    """Unknown activations and activated-column starts outside [0, N] are
+    refused before any device work; the other checks are tern_linear's."""
+    def call(act, col0, N=256, y=F + 0x300000):
+        return L.tern_linear_act(ctypes.c_void_p(F), 16, 256, ctypes.c_void_p(F + 0x100000),
+                                 ctypes.c_void_p(F + 0x200000), None, N, act, col0, ctypes.c_void_p(y), None)
+    assert call(7, 0) == INVALID
+    assert call(-1, 0) == INVALID
+    assert call(tern.ACT_GELU_TANH, -1) == INVALID
+    assert call(tern.ACT_GELU_TANH, 257) == INVALID
+    assert call(tern.ACT_GELU_TANH, 0, N=100) == SHAPE
+    assert call(tern.ACT_GELU_TANH, 0, y=F + 0x300004) == MISALIGNED
+    # M = 0 is a no-op that still validates the activation
+    assert L.tern_linear_act(None, 0, 256, ctypes.c_void_p(F), ctypes.c_void_p(F + 0x100000), None, 256,
+                             tern.ACT_GELU_TANH, 256, None, None) == 0
+    assert L.tern_linear_act(None, 0, 256, ctypes.c_void_p(F), ctypes.c_void_p(F + 0x100000), None, 256,
+                             5, 0, None, None) == INVALID
+
+
+def test_batch_act_rejects_on_host(L):
+    arr = (tern.LinearActArgs * 2)()
+    ok = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, 16, 256, 256)
+    arr[0] = tern.LinearActArgs(ok, tern.ACT_GELU_TANH, 128)
+    arr[1] = tern.LinearActArgs(ok, tern.ACT_GELU_TANH, 300)
+    assert L.tern_linear_batch_act(arr, 2, None) == INVALID
+    assert b"problem 1" in L.tern_last_error()
+    assert L.tern_linear_batch_act(arr, 0, None) == 0
+    assert L.tern_linear_batch_act(None, 1, None) == INVALID

@@ -312,3 +312,76 @@ def test_device_wait_timeout_is_reported_and_context_survives():
     assert tern.device_status() == -5
     assert tern.device_status() == 0  # cleared by the read
     run_linear_case(8, 128, 64, seed=5)  # the context is still usable
+
+
+# ------------------------------------------------ fused activation epilogue
+@pytest.mark.parametrize("M,N,K,col0", [
+    (1, 384, 256, 0),        # GEMV, 8-token blocks
+    (12, 256, 320, 128),     # GEMV, two 8-token blocks, activation on the upper half
+    (40, 512, 256, 0),       # 64-token tcgen05 tiles
+    (300, 512, 192, 256),    # CTA-pair tiles, activation on the second pair tile
+    (300, 512, 192, 100),    # CTA-pair tiles, activation from inside a warp's channels
+    (1024, 1024, 512, 0),    # several pair tiles per CTA pair
+    (70, 384, 128, 0),       # single-CTA fallback (N % 256 != 0)
+    (40, 384, 1024, 129),    # fallback with split K (partials summed by the last CTA)
+])
+def test_linear_act_gelu(M, N, K, col0):
+    W = rand_bf16((N, K), 0.02, M + N)
+    x = rand_bf16((M, K), 1.0, M + K)
+    b = rand_bf16((N,), 0.01, N + K)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear_act(x.cuda(), packed, scales, b.cuda(), tern.ACT_GELU_TANH, col0)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    y_ref = oracle.linear_act(bits(x), T, s, bits(b), oracle.ACT_GELU_TANH, col0)
+    check_y(y, y_ref)
+    # the columns below col0 are the plain layer, bit for bit
+    y_plain = tern.linear(x.cuda(), packed, scales, b.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(y[:, :col0], y_plain[:, :col0])
+
+
+def test_linear_act_none_is_linear():
+    W = rand_bf16((512, 256), 0.02, 5)
+    x = rand_bf16((300, 256), 1.0, 6).cuda()
+    packed, scales = quantize_on_gpu(W)
+    assert torch.equal(tern.linear_act(x, packed, scales, None, tern.ACT_NONE, 0),
+                       tern.linear(x, packed, scales, None))
+
+
+def test_linear_act_gelu_flux_mlp_up_sampled():
+    """The MLP up projection of the FLUX stack with its GELU fused, at full size
+    (4608 tokens), in the launch configuration of the layer; 32 sampled rows."""
+    L = workloads.CONFIGS["mlp_up"]
+    x, W, b = workloads.make_inputs(L)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear_act(x.cuda(), packed, scales, b.cuda(), tern.ACT_GELU_TANH, 0)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    rows = np.sort(np.random.default_rng(11).choice(L.M, 32, replace=False))
+    rows[-1] = L.M - 1
+    ref = oracle.linear_act(bits(x[rows]), T, s, bits(b), oracle.ACT_GELU_TANH, 0)
+    check_y(y[torch.from_numpy(rows).cuda()], ref)
+
+
+def test_linear_batch_act_mixed():
+    cases = [(1, 256, 192, tern.ACT_GELU_TANH, 0), (9, 384, 256, tern.ACT_NONE, 0),
+             (40, 512, 256, tern.ACT_GELU_TANH, 256), (300, 256, 320, tern.ACT_GELU_TANH, 0),
+             (70, 128, 128, tern.ACT_GELU_TANH, 64), (600, 512, 192, tern.ACT_NONE, 0)]
+    probs, refs = [], []
+    for i, (M, N, K, act, col0) in enumerate(cases):
+        W = rand_bf16((N, K), 0.02, 400 + i)
+        x = rand_bf16((M, K), 1.0, 500 + i)
+        b = rand_bf16((N,), 0.01, 600 + i)
+        packed, scales = quantize_on_gpu(W)
+        T, s = check_quantize(W, packed, scales, {})
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        probs.append(dict(x=x.cuda(), packed=packed, scales=scales, bias=b.cuda(), y=y, act=act, act_col0=col0))
+        refs.append(oracle.linear_act(bits(x), T, s, bits(b), act, col0))
+    tern.linear_batch_act(probs)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    for p, r in zip(probs, refs):
+        check_y(p["y"], r)
