@@ -417,6 +417,14 @@ def side_table(device, peaks, stream):
         entry = {"M": L.M, "N": L.N, "K": L.K, "us": t * 1e6, "tflops": L.flop / t / 1e12,
                  "packed_gbs": L.packed_bytes / t / 1e9, "roofline_frac": max(flop_t, byte_t) / t,
                  "bound": "tensor" if flop_t > byte_t else "hbm"}
+        if name == "mlp_up":
+            # FLUX's MLP activation fused into the epilogue, against the HBM
+            # time a separate bf16 GELU pass over y would need (read + write)
+            acts = [(lambda p=p, s=s: tern.linear_act(x, p, s, b, tern.ACT_GELU_TANH, 0, out=y))
+                    for p, s in packs]
+            ta = graph_time(acts * reps, 5, stream)
+            entry["gelu_fused_us"] = ta * 1e6
+            entry["gelu_separate_pass_us_at_hbm_peak"] = 2 * 2 * L.M * L.N / peaks["hbm_gbs"] / 1e9 * 1e6
         if name in ("mlp_up", "mlp_down", "mod6_m64"):
             Wd = tern.dequantize(packs[0][0], packs[0][1], L.K, stream=stream)
             torch.cuda.synchronize()
@@ -443,8 +451,10 @@ def stack_rows(device, peaks, stream):
     """The whole ternary linear stack of one FLUX.1-dev forward at 1024x1024
     (19 double + 38 single blocks; weights drawn on the device from N(0, 0.02)
     per layer seed and quantised, only the codes kept), run block by block
-    through tern_linear_batch with synthetic activations, and the 76 adaLN
-    modulation GEMVs of a forward alone: batched versus one call each."""
+    through tern_linear_batch_act with synthetic activations and the MLP's
+    GELU fused into its first linear (the MLP columns of a single block's
+    fused projection), and the 76 adaLN modulation GEMVs of a forward alone:
+    batched versus one call each."""
     import torch
 
     from bit_post_quantised_b200 import tern, workloads
@@ -474,17 +484,23 @@ def stack_rows(device, peaks, stream):
             L = layers[i]
             if L.N not in bias:
                 bias[L.N] = (torch.randn(L.N, device=device) * 0.01).to(torch.bfloat16)
+            act, col0 = tern.ACT_NONE, 0
+            if L.name.endswith(".mlp_up"):
+                act = tern.ACT_GELU_TANH
+            elif L.name.endswith(".qkv_mlp"):
+                act, col0 = tern.ACT_GELU_TANH, 3 * workloads.HIDDEN  # q, k, v, then the MLP part
             probs.append(dict(x=buf(xs, (L.M, L.K), (L.M, L.K)), packed=packs[i][0], scales=packs[i][1],
-                              bias=bias[L.N], y=buf(ys, (j, L.M, L.N), (L.M, L.N))))
+                              bias=bias[L.N], y=buf(ys, (j, L.M, L.N), (L.M, L.N)), act=act, act_col0=col0))
         problems.append(probs)
     flop = sum(L.flop for L in layers)
 
     def forward():
         for probs in problems:
-            tern.linear_batch(probs, stream=stream)
+            tern.linear_batch_act(probs, stream=stream)
 
     t = graph_time([forward], 3, stream)
-    out = {"flux_stack": {"layers": len(layers), "launch_groups": "one tern_linear_batch per block",
+    out = {"flux_stack": {"layers": len(layers), "launch_groups": "one tern_linear_batch_act per block",
+                          "epilogue": "GELU (tanh form) fused into every MLP up projection",
                           "ms_per_forward": t * 1e3, "tflops": flop / t / 1e12,
                           "tensor_roofline_ms": flop / (peaks["bf16_tflops"] * 1e12) * 1e3,
                           "packed_weight_gb": sum(L.packed_bytes for L in layers) / 1e9}}
