@@ -394,6 +394,18 @@ int ctas_per_sm(int tok) {
   return std::max(1, std::min(by_smem, by_tmem));
 }
 
+// K splits of the single-CTA fallback kernel for one problem: with few tokens
+// (tok <= 64), enough splits that every SM streams codes, at least 4 chunks
+// of 64 k per split, at most 16.
+int fallback_splits(int64_t M, int64_t N, int64_t K, int tok, const DeviceState* ds) {
+  if (tok > 64) return 1;
+  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
+  int splits = 1;
+  if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
+  return std::max(1, std::min(splits, 16));
+}
+
 }  // namespace
 }  // namespace tern
 
@@ -456,14 +468,8 @@ tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stre
     return launch_2sm_group(&a, &act, std::vector<int>{0}, ptok, batch2, ds, cs);
   }
   const int tok = pick_tok(M);
-  int splits = 1;
+  const int splits = fallback_splits(M, N, K, tok, ds);
   const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
-  if (tok <= 64) {
-    // Few tokens: split K so that every SM streams codes.
-    const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
-    if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
-    splits = std::max(1, std::min(splits, 16));
-  }
   static Batch batch;  // built under the lock below; ~4 KiB, copied into the launch
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
@@ -722,13 +728,8 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
 
   // Same tile and split choice as tern_linear, so the two give identical y.
   const int tok = pick_tok(M);
-  int splits = 1;
+  const int splits = fallback_splits(M, N, K, tok, ds);
   const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
-  if (tok <= 64) {
-    const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
-    if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
-    splits = std::max(1, std::min(splits, 16));
-  }
   std::memset(static_cast<void*>(&batch), 0, sizeof batch);
   int64_t ctas = 0;
   if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;
