@@ -23,7 +23,10 @@ struct alignas(64) Problem {
   int unit_begin;            // first work unit (CTA, or 2-SM tile) of this problem
   int act;                   // epilogue activation (kActNone / kActGeluTanh)
   int act_col0;              // first output column the activation applies to
+  const __nv_bfloat16* residual;  // [M, N] or null: y = residual + gate * act(v)
+  const __nv_bfloat16* gate;      // [N] or null (gate 1)
 };
+static_assert(sizeof(Problem) == 256, "Problem layout");
 
 constexpr int kMaxProblems = 15;  // keeps the kernel parameter block under 4 KiB
 
@@ -34,6 +37,7 @@ struct Batch {
   unsigned long long wait_limit_ns;
   unsigned int* status;     // per-device status word (bounded waits report here)
 };
+static_assert(sizeof(Batch) <= 4096, "kernel parameter block");
 
 // Token-tile sizes (UMMA N) with a compiled kernel.
 constexpr int kTokTiles[] = {32, 64, 128};

@@ -91,6 +91,15 @@ __device__ __forceinline__ float apply_act(float v, int act, int n, int act_col0
   return (act == kActGeluTanh && n >= act_col0) ? gelu_tanh(v) : v;
 }
 
+// The whole epilogue after v = acc * s + b, in fp32 (one rounding follows):
+// a = act(v) on the activated columns, then residual[m, n] + gate[n] * a
+// where a residual is given (gate 1 where none is).
+__device__ __forceinline__ float epilogue_value(float v, int act, int n, int act_col0, const uint16_t* residual,
+                                                size_t mn, float gate) {
+  const float a = apply_act(v, act, n, act_col0);
+  return residual ? fmaf(gate, a, __uint_as_float(uint32_t(residual[mn]) << 16)) : gate * a;
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(uint32_t(b) << 16);
 }

@@ -222,22 +222,30 @@ tern_status check_linear(const tern_linear_args& a) {
 
 static_assert(kActNone == TERN_ACT_NONE && kActGeluTanh == TERN_ACT_GELU_TANH, "kernel and ABI activation codes");
 
-// Epilogue activation of one problem (TERN_ACT_NONE for the plain layer).
-struct ActSpec {
-  int act = TERN_ACT_NONE;
-  int64_t col0 = 0;
-};
+// (The epilogue of one problem is a tern_epilogue; all zero is the plain layer.)
 
-tern_status check_act(int act, int64_t col0, int64_t N) {
-  if (act != TERN_ACT_NONE && act != TERN_ACT_GELU_TANH) return fail(TERN_ERR_INVALID_ARG, "unknown activation %d", act);
-  if (col0 < 0 || col0 > N)
-    return fail(TERN_ERR_INVALID_ARG, "act_col0=%lld outside [0, N=%lld]", (long long)col0, (long long)N);
+tern_status check_epilogue(const tern_epilogue& e, const tern_linear_args& a) {
+  if (e.act != TERN_ACT_NONE && e.act != TERN_ACT_GELU_TANH)
+    return fail(TERN_ERR_INVALID_ARG, "unknown activation %d", e.act);
+  if (e.act_col0 < 0 || e.act_col0 > a.N)
+    return fail(TERN_ERR_INVALID_ARG, "act_col0=%lld outside [0, N=%lld]", (long long)e.act_col0, (long long)a.N);
+  if (!aligned(e.residual, 2) || !aligned(e.gate, 2))
+    return fail(TERN_ERR_MISALIGNED, "residual and gate need 2-byte alignment");
+  const size_t ybytes = size_t(a.M) * size_t(a.N) * 2;
+  // The residual may be y itself (an in-place update: each element is read
+  // before the same thread writes it); any other overlap with y would race.
+  if (e.residual && e.residual != a.y && overlaps(e.residual, ybytes, a.y, ybytes))
+    return fail(TERN_ERR_INVALID_ARG, "residual overlaps y without being y");
+  if (overlaps(e.gate, e.gate ? size_t(a.N) * 2 : 0, a.y, ybytes)) return fail(TERN_ERR_INVALID_ARG, "gate overlaps y");
   return TERN_OK;
 }
 
-void set_act(Problem* p, const ActSpec* acts, int i) {
-  p->act = acts ? acts[i].act : TERN_ACT_NONE;
-  p->act_col0 = acts ? int(acts[i].col0) : 0;
+void set_epilogue(Problem* p, const tern_epilogue* epis, int i) {
+  if (!epis) return;  // the Problem was zeroed: plain layer
+  p->act = epis[i].act;
+  p->act_col0 = int(epis[i].act_col0);
+  p->residual = static_cast<const __nv_bfloat16*>(epis[i].residual);
+  p->gate = static_cast<const __nv_bfloat16*>(epis[i].gate);
 }
 
 // Up to 16 tokens run on the register-fed GEMV kernel, in n8 blocks.
@@ -313,7 +321,7 @@ tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int
 
 // Launches the problems `idx` of `args` (all with pair_tok == tok) on the
 // pair-tile kernel, up to kMaxProblems per launch.
-tern_status launch_2sm_group(const tern_linear_args* args, const ActSpec* acts, const std::vector<int>& idx, int tok,
+tern_status launch_2sm_group(const tern_linear_args* args, const tern_epilogue* epis, const std::vector<int>& idx, int tok,
                              Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
@@ -323,7 +331,7 @@ tern_status launch_2sm_group(const tern_linear_args* args, const ActSpec* acts, 
       int64_t tiles = 0;
       tern_status s = fill_problem_2sm(args[idx[g]], tok, &batch.p[n], &tiles);
       if (s != TERN_OK) return s;
-      set_act(&batch.p[n], acts, idx[g]);
+      set_epilogue(&batch.p[n], epis, idx[g]);
       batch.p[n].unit_begin = int(total);
       total += tiles;
       if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
@@ -343,7 +351,7 @@ tern_status launch_2sm_group(const tern_linear_args* args, const ActSpec* acts, 
 // Launches the problems `idx` of `args` (all with M <= 8 nt) on the GEMV
 // kernel, up to kMaxProblems per launch.  K is split over a cluster of up to
 // eight CTAs when the launch has fewer 128-channel slabs than the GPU has SMs.
-tern_status launch_gemv_group(const tern_linear_args* args, const ActSpec* acts, const std::vector<int>& idx, int nt,
+tern_status launch_gemv_group(const tern_linear_args* args, const tern_epilogue* epis, const std::vector<int>& idx, int nt,
                               Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
@@ -364,7 +372,7 @@ tern_status launch_gemv_group(const tern_linear_args* args, const ActSpec* acts,
       p->K = int(a.K);
       p->n_tiles = int(a.N / 128);
       p->m_tiles = 1;
-      set_act(p, acts, idx[g]);
+      set_epilogue(p, epis, idx[g]);
       p->unit_begin = int(slabs);
       slabs += a.N / 128;
       min_chunks = std::min<int64_t>(min_chunks, a.K / 64);
@@ -444,11 +452,11 @@ tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float e
 namespace tern {
 namespace {
 
-tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stream_t stream) {
+tern_status linear_impl(const tern_linear_args& a, const tern_epilogue& epi, tern_stream_t stream) {
   const int64_t M = a.M, N = a.N, K = a.K;
   tern_status s = check_linear(a);
   if (s != TERN_OK) return s;
-  if ((s = check_act(act.act, act.col0, N)) != TERN_OK) return s;
+  if ((s = check_epilogue(epi, a)) != TERN_OK) return s;
   if (M == 0) return TERN_OK;
   int dev;
   DeviceState* ds;
@@ -459,13 +467,13 @@ tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stre
     static Batch batch_g;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch_g_mu;
     std::lock_guard<std::mutex> lock(batch_g_mu);
-    return launch_gemv_group(&a, &act, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
+    return launch_gemv_group(&a, &epi, std::vector<int>{0}, gemv_nt(M), batch_g, ds, cs);
   }
   if (const int ptok = pair_tok(a, ds)) {
     static Batch batch2;  // built under the lock below; ~4 KiB, copied into the launch
     static std::mutex batch2_mu;
     std::lock_guard<std::mutex> lock(batch2_mu);
-    return launch_2sm_group(&a, &act, std::vector<int>{0}, ptok, batch2, ds, cs);
+    return launch_2sm_group(&a, &epi, std::vector<int>{0}, ptok, batch2, ds, cs);
   }
   const int tok = pick_tok(M);
   const int splits = fallback_splits(M, N, K, tok, ds);
@@ -477,7 +485,7 @@ tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stre
   int64_t ctas = 0;
   if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;
   Problem& p = batch.p[0];
-  set_act(&p, &act, 0);
+  set_epilogue(&p, &epi, 0);
   if (p.splits > 1) {
     const size_t ws_bytes = size_t(p.splits) * size_t(tiles) * tok * 128 * sizeof(float);
     if ((s = get_workspace(dev, cs, ws_bytes, size_t(tiles), &p.ws, &p.counters)) != TERN_OK) return s;
@@ -492,10 +500,10 @@ tern_status linear_impl(const tern_linear_args& a, const ActSpec& act, tern_stre
   return TERN_OK;
 }
 
-tern_status batch_impl(const tern_linear_args* args, const ActSpec* acts, int count, tern_stream_t stream) {
+tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, int count, tern_stream_t stream) {
   for (int i = 0; i < count; ++i) {
     tern_status s = check_linear(args[i]);
-    if (s == TERN_OK && acts) s = check_act(acts[i].act, acts[i].col0, args[i].N);
+    if (s == TERN_OK && epis) s = check_epilogue(epis[i], args[i]);
     if (s != TERN_OK) {
       t_last_error = "problem " + std::to_string(i) + ": " + t_last_error;
       return s;
@@ -515,13 +523,13 @@ tern_status batch_impl(const tern_linear_args* args, const ActSpec* acts, int co
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
       if (args[i].M > 0 && args[i].M <= kGemvMaxM && gemv_nt(args[i].M) == nt) group.push_back(i);
-    if ((s = launch_gemv_group(args, acts, group, nt, batch, ds, cs)) != TERN_OK) return s;
+    if ((s = launch_gemv_group(args, epis, group, nt, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int ptok : {64, 256}) {
     std::vector<int> group;
     for (int i = 0; i < count; ++i)
       if (args[i].M > 0 && pair_tok(args[i], ds) == ptok) group.push_back(i);
-    if ((s = launch_2sm_group(args, acts, group, ptok, batch, ds, cs)) != TERN_OK) return s;
+    if ((s = launch_2sm_group(args, epis, group, ptok, batch, ds, cs)) != TERN_OK) return s;
   }
   for (int tok : kTokTiles) {
     std::vector<int> group;
@@ -534,7 +542,7 @@ tern_status batch_impl(const tern_linear_args* args, const ActSpec* acts, int co
       for (size_t g = g0; g < group.size() && n < kMaxProblems; ++g, ++n) {
         int64_t ctas = 0;
         if ((s = fill_problem(args[group[g]], tok, 1, &batch.p[n], &ctas)) != TERN_OK) return s;
-        set_act(&batch.p[n], acts, group[g]);
+        set_epilogue(&batch.p[n], epis, group[g]);
         batch.p[n].unit_begin = int(total);
         total += ctas;
         if (total > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "batch too large");
@@ -558,15 +566,15 @@ extern "C" {
 tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
                         const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
                         tern_stream_t stream) {
-  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, ActSpec{}, stream);
+  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, tern_epilogue{}, stream);
 }
 
 tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, const void* packed,
                             const float* scales, const void* bias_bf16, int64_t N, int act, int64_t act_col0,
                             void* y_bf16, tern_stream_t stream) {
-  ActSpec spec;
+  tern_epilogue spec{};
   spec.act = act;
-  spec.col0 = act_col0;
+  spec.act_col0 = act_col0;
   return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, spec, stream);
 }
 
@@ -578,13 +586,25 @@ tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stre
 tern_status tern_linear_batch_act(const tern_linear_act_args* args, int count, tern_stream_t stream) {
   if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
   std::vector<tern_linear_args> lin(size_t(std::max(count, 0)));
-  std::vector<ActSpec> acts(size_t(std::max(count, 0)));
+  std::vector<tern_epilogue> epis(size_t(std::max(count, 0)));
   for (int i = 0; i < count; ++i) {
     lin[i] = args[i].linear;
-    acts[i].act = args[i].act;
-    acts[i].col0 = args[i].act_col0;
+    epis[i] = tern_epilogue{};
+    epis[i].act = args[i].act;
+    epis[i].act_col0 = args[i].act_col0;
   }
-  return batch_impl(lin.data(), acts.data(), count, stream);
+  return batch_impl(lin.data(), epis.data(), count, stream);
+}
+
+tern_status tern_linear_epilogue(const tern_linear_args* args, const tern_epilogue* epilogue, tern_stream_t stream) {
+  if (!args) return fail(TERN_ERR_INVALID_ARG, "null args");
+  return linear_impl(*args, epilogue ? *epilogue : tern_epilogue{}, stream);
+}
+
+tern_status tern_linear_batch_epilogue(const tern_linear_args* args, const tern_epilogue* epilogues, int count,
+                                       tern_stream_t stream) {
+  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+  return batch_impl(args, epilogues, count, stream);
 }
 
 tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,

@@ -102,6 +102,8 @@ struct GemvProb {
   __nv_bfloat16* y;
   int unit_begin, M, N, K, chunks_per_split;
   int act, act_col0;  // epilogue activation and its first column
+  const uint16_t* residual;  // [M, N] or null
+  const uint16_t* gate;      // [N] or null
 };
 
 __device__ __forceinline__ int unit_problem(const GemvProb* probs, int count, int u, int* slab) {
@@ -160,6 +162,8 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     g.chunks_per_split = q.chunks_per_split;
     g.act = q.act;
     g.act_col0 = q.act_col0;
+    g.residual = reinterpret_cast<const uint16_t*>(q.residual);
+    g.gate = reinterpret_cast<const uint16_t*>(q.gate);
   }
   const int nprob = batch.count;
   __syncthreads();
@@ -223,7 +227,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     if (warp < C::kWarps) {
       // Scale and bias of this lane's two output channels, loaded now and used
       // after the stream (only rank 0 stores).
-      float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
+      float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f, g0 = 1.f, g1 = 1.f;
       if (rank == 0) {
         s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
         s1 = 0.5f * P.scales[n_out + 8];
@@ -231,6 +235,10 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
         if (bias) {
           b0 = bf16_bits_to_float(bias[n_out]);
           b1 = bf16_bits_to_float(bias[n_out + 8]);
+        }
+        if (P.gate) {
+          g0 = bf16_bits_to_float(P.gate[n_out]);
+          g1 = bf16_bits_to_float(P.gate[n_out + 8]);
         }
       }
       const int kc_total = P.K >> 6;
@@ -315,17 +323,18 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
 #pragma unroll
         for (int nb = 0; nb < NT; ++nb) {
           const int t0 = 8 * nb + 2 * c;
+          const size_t m0 = size_t(t0) * P.N, m1 = m0 + P.N;
           if (t0 < P.M) {
-            P.y[size_t(t0) * P.N + n_out] =
-                __float2bfloat16_rn(apply_act(fmaf(d[nb][0], s0, b0), P.act, n_out, P.act_col0));
-            P.y[size_t(t0) * P.N + n_out + 8] =
-                __float2bfloat16_rn(apply_act(fmaf(d[nb][2], s1, b1), P.act, n_out + 8, P.act_col0));
+            P.y[m0 + n_out] = __float2bfloat16_rn(
+                epilogue_value(fmaf(d[nb][0], s0, b0), P.act, n_out, P.act_col0, P.residual, m0 + n_out, g0));
+            P.y[m0 + n_out + 8] = __float2bfloat16_rn(
+                epilogue_value(fmaf(d[nb][2], s1, b1), P.act, n_out + 8, P.act_col0, P.residual, m0 + n_out + 8, g1));
           }
           if (t0 + 1 < P.M) {
-            P.y[size_t(t0 + 1) * P.N + n_out] =
-                __float2bfloat16_rn(apply_act(fmaf(d[nb][1], s0, b0), P.act, n_out, P.act_col0));
-            P.y[size_t(t0 + 1) * P.N + n_out + 8] =
-                __float2bfloat16_rn(apply_act(fmaf(d[nb][3], s1, b1), P.act, n_out + 8, P.act_col0));
+            P.y[m1 + n_out] = __float2bfloat16_rn(
+                epilogue_value(fmaf(d[nb][1], s0, b0), P.act, n_out, P.act_col0, P.residual, m1 + n_out, g0));
+            P.y[m1 + n_out + 8] = __float2bfloat16_rn(
+                epilogue_value(fmaf(d[nb][3], s1, b1), P.act, n_out + 8, P.act_col0, P.residual, m1 + n_out + 8, g1));
           }
         }
       }

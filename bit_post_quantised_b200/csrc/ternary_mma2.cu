@@ -326,14 +326,19 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const int ab = lt % AB;
       const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
       const float sc = 0.5f * P.scales[n];  // A held 2t
-      const bool gelu = P.act == kActGeluTanh && n >= P.act_col0;
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
+      const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
+      const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
+      const bool plain = P.act == kActNone && !res && !P.gate;  // the same for the whole problem
+      const int row0 = t.m_tile * C::kTokPair + half * kCols;
+      const int rows = min(kCols, P.M - row0);
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
       tc_fence_after();
-      uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
-      if (__any_sync(0xffffffffu, gelu)) {
-        // The activation's transcendentals run after the accumulator is
-        // released, so they overlap the next tile's MMAs: keep y in fp32.
+      uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+      if (!plain) {
+        // The epilogue's activation and residual reads run after the
+        // accumulator is released, so they overlap the next tile's MMAs:
+        // keep y in fp32 until its store.
         float f[kCols];
 #pragma unroll
         for (int c0 = 0; c0 < kCols; c0 += 32) {
@@ -346,10 +351,17 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
 #pragma unroll
-        for (int j = 0; j < kCols / 2; ++j)
-          out[j] = gelu ? pack_bf16x2(gelu_tanh(f[2 * j]), gelu_tanh(f[2 * j + 1])) : pack_bf16x2(f[2 * j], f[2 * j + 1]);
+        for (int c = 0; c < kCols; ++c)
+          if (c < rows) {
+            const float a = apply_act(f[c], act, n, act_col0);
+            const float y = rp ? fmaf(gt, a, bf16_bits_to_float(rp[c * ld])) : gt * a;
+            yp[c * ld] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+          }
       } else {
+        uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
 #pragma unroll
         for (int c0 = 0; c0 < kCols; c0 += 32) {
           uint32_t v[32];
@@ -363,13 +375,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
-      }
-      const int row0 = t.m_tile * C::kTokPair + half * kCols;
-      const int rows = min(kCols, P.M - row0);
-      uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
 #pragma unroll
-      for (int c = 0; c < kCols; ++c)
-        if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+        for (int c = 0; c < kCols; ++c)
+          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+      }
     }
   }
 

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
                 -6: "TERN_ERR_NO_DEVICE"}
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
-            "tern_linear_act", "tern_linear_batch", "tern_linear_batch_act",
+            "tern_linear_act", "tern_linear_epilogue", "tern_linear_batch", "tern_linear_batch_act",
+            "tern_linear_batch_epilogue",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -44,6 +45,12 @@ class LinearArgs(ctypes.Structure):
 class LinearActArgs(ctypes.Structure):
     """Mirror of tern_linear_act_args."""
     _fields_ = [("linear", LinearArgs), ("act", ctypes.c_int), ("act_col0", ctypes.c_int64)]
+
+
+class Epilogue(ctypes.Structure):
+    """Mirror of tern_epilogue."""
+    _fields_ = [("act", ctypes.c_int), ("act_col0", ctypes.c_int64), ("residual", ctypes.c_void_p),
+                ("gate", ctypes.c_void_p)]
 
 
 ACT_NONE = 0       # tern_act values
@@ -76,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.tern_linear_act.restype = st
         L.tern_linear_batch_act.argtypes = [ctypes.POINTER(LinearActArgs), ctypes.c_int, vp]
         L.tern_linear_batch_act.restype = st
+        L.tern_linear_epilogue.argtypes = [ctypes.POINTER(LinearArgs), ctypes.POINTER(Epilogue), vp]
+        L.tern_linear_epilogue.restype = st
+        L.tern_linear_batch_epilogue.argtypes = [ctypes.POINTER(LinearArgs), ctypes.POINTER(Epilogue), ctypes.c_int,
+                                                 vp]
+        L.tern_linear_batch_epilogue.restype = st
         L.tern_linear_batch.restype = st
         L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
         L.tern_dequantize.restype = st
@@ -189,6 +201,44 @@ def linear_batch_act(problems: Sequence[dict], stream=None) -> None:
                                           p["y"].data_ptr(), M, N, K),
                                p.get("act", ACT_NONE), p.get("act_col0", 0))
     _check(lib().tern_linear_batch_act(arr, len(problems), _stream(stream)))
+
+
+def _linear_args(p: dict) -> LinearArgs:
+    M, K = p["x"].shape
+    N = p["scales"].shape[0]
+    return LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
+                      None if p.get("bias") is None else p["bias"].data_ptr(), p["y"].data_ptr(), M, N, K)
+
+
+def _epilogue(p: dict) -> Epilogue:
+    return Epilogue(p.get("act", ACT_NONE), p.get("act_col0", 0), _ptr(p.get("residual")), _ptr(p.get("gate")))
+
+
+def linear_epilogue(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                    bias: Optional[torch.Tensor] = None, act: int = ACT_NONE, act_col0: int = 0,
+                    residual: Optional[torch.Tensor] = None, gate: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, stream=None):
+    """tern_linear_epilogue: y = residual + gate * act(x . T^T * s + b) (see
+    tern_epilogue); `out` may be `residual` itself for an in-place update."""
+    M, K = x.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    a = _linear_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
+    e = _epilogue(dict(act=act, act_col0=act_col0, residual=residual, gate=gate))
+    _check(lib().tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
+    return out
+
+
+def linear_batch_epilogue(problems: Sequence[dict], stream=None) -> None:
+    """tern_linear_batch_epilogue over dicts as linear_batch's plus the
+    optional keys act, act_col0, residual and gate."""
+    n = max(1, len(problems))
+    args, epis = (LinearArgs * n)(), (Epilogue * n)()
+    for i, p in enumerate(problems):
+        args[i] = _linear_args(p)
+        epis[i] = _epilogue(p)
+    _check(lib().tern_linear_batch_epilogue(args, epis, len(problems), _stream(stream)))
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional[torch.Tensor] = None,

@@ -172,6 +172,38 @@ typedef struct {
 } tern_linear_args;
 
 /*
+ * A fused epilogue.  With v = s_n * sum_k x[m,k] * T[n,k] + b_n in fp32:
+ *     a = act(v) for n >= act_col0, else v;
+ *     y[m,n] = residual[m,n] + gate[n] * a     (residual NULL: 0; gate NULL: 1),
+ * in fp32, then one rounding to bf16.  All zero is the plain layer.
+ *   act, act_col0  as tern_linear_act.
+ *   residual       [M, N] bf16, row-major, or NULL.  It may be y itself (an
+ *                  in-place update of a residual stream); any other overlap
+ *                  with y is TERN_ERR_INVALID_ARG.  2-byte aligned.
+ *   gate           [N] bf16 or NULL, 2-byte aligned, not overlapping y.
+ * FLUX.1's blocks add their attention output projection and their MLP's
+ * second linear to the residual stream scaled by an adaLN-Zero gate taken
+ * from the modulation GEMV's output; with residual = y = the stream and gate
+ * = that slice, the update happens inside the linear's epilogue.  The pages
+ * describe no operation between the quantised linears (Section 3.1): this is
+ * an interface choice of this library.
+ */
+typedef struct {
+  int act;              /* tern_act */
+  int64_t act_col0;     /* first activated output column */
+  const void* residual; /* [M, N] bf16 or NULL */
+  const void* gate;     /* [N] bf16 or NULL */
+} tern_epilogue;
+
+/* tern_linear of *args with the fused epilogue *epilogue (NULL: none). */
+TERN_API tern_status tern_linear_epilogue(const tern_linear_args* args, const tern_epilogue* epilogue,
+                                 tern_stream_t stream);
+
+/* tern_linear_batch with epilogues[i] for problem i (epilogues NULL: none). */
+TERN_API tern_status tern_linear_batch_epilogue(const tern_linear_args* args, const tern_epilogue* epilogues,
+                                       int count, tern_stream_t stream);
+
+/*
  * Several independent ternary linears (for instance the per-stream adaLN
  * modulation GEMVs and projections of one FLUX block) with as few launches as
  * possible: problems with similar M share one grouped launch (M <= 8, M <= 16,

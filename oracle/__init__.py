@@ -221,3 +221,25 @@ def linear_act(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, ac
     if act == ACT_GELU_TANH:
         return gelu_tanh(y, col0)
     raise ValueError("unknown activation")
+
+
+def linear_epilogue(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, act: int = ACT_NONE,
+                    col0: int = 0, residual_bits=None, gate_bits=None) -> np.ndarray:
+    """The layer with a fused epilogue, in float64: a = act(v) on columns
+    [col0, N) of v = linear(...), then residual + gate * a (residual [M, N]
+    and gate [N] are bf16 bit patterns; absent residual = 0, absent gate = 1).
+    FLUX.1 adds its attention and MLP outputs to the residual stream scaled by
+    an adaLN-Zero gate; the pages describe no operation between the quantised
+    linears, so this follows that model's definition."""
+    a = linear_act(x_bits, T, s, b_bits, act, col0)
+    if gate_bits is not None:
+        g = bf16_bits_to_f64(_c(gate_bits, np.uint16))
+        if g.shape != (a.shape[1],):
+            raise ValueError("gate shape mismatch")
+        a = a * g[None, :]
+    if residual_bits is not None:
+        r = bf16_bits_to_f64(_c(residual_bits, np.uint16))
+        if r.shape != a.shape:
+            raise ValueError("residual shape mismatch")
+        a = r + a
+    return a

@@ -165,3 +165,22 @@ def test_batch_act_rejects_on_host(L):
     assert b"problem 1" in L.tern_last_error()
     assert L.tern_linear_batch_act(arr, 0, None) == 0
     assert L.tern_linear_batch_act(None, 1, None) == INVALID
+
+
+def test_epilogue_rejects_on_host(L):
+    """Residual and gate checks of tern_linear_epilogue, before any device work."""
+    a = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, 16, 256, 256)
+    y_bytes = 16 * 256 * 2
+
+    def call(**kw):
+        e = tern.Epilogue(kw.get("act", 0), kw.get("col0", 0), kw.get("residual"), kw.get("gate"))
+        return L.tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), None)
+    assert call(residual=F + 0x300000 + 2) == INVALID        # partial overlap with y
+    assert call(residual=F + 0x300000 - y_bytes + 2) == INVALID
+    assert call(residual=F + 0x500001) == MISALIGNED
+    assert call(gate=F + 0x500001) == MISALIGNED
+    assert call(gate=F + 0x300000 + 64) == INVALID           # gate inside y
+    assert call(act=3) == INVALID
+    assert L.tern_linear_epilogue(None, None, None) == INVALID
+    assert L.tern_linear_batch_epilogue(None, None, 2, None) == INVALID
+    assert L.tern_linear_batch_epilogue(None, None, 0, None) == 0

@@ -385,3 +385,59 @@ def test_linear_batch_act_mixed():
     assert tern.device_status() == 0
     for p, r in zip(probs, refs):
         check_y(p["y"], r)
+
+
+# --------------------------------------- fused gated residual (adaLN-Zero) epilogue
+@pytest.mark.parametrize("M,N,K,act,col0,inplace", [
+    (1, 384, 256, 0, 0, True),        # GEMV, in-place residual stream update
+    (12, 256, 320, 1, 128, False),    # GEMV, GELU on half the channels + residual
+    (40, 512, 256, 0, 0, True),       # 64-token tiles
+    (300, 512, 192, 0, 0, True),      # CTA-pair tiles, in place
+    (300, 512, 192, 1, 100, False),   # CTA-pair tiles, GELU + residual + gate
+    (70, 384, 128, 0, 0, True),       # fallback
+    (40, 384, 1024, 1, 0, False),     # fallback with split K
+])
+def test_linear_epilogue_gated_residual(M, N, K, act, col0, inplace):
+    W = rand_bf16((N, K), 0.02, M + 3 * N)
+    x = rand_bf16((M, K), 1.0, M + 5 * K)
+    b = rand_bf16((N,), 0.01, N + 7)
+    r = rand_bf16((M, N), 1.0, M * N + 1)
+    g = rand_bf16((N,), 0.5, N + 11)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    rd = r.cuda()
+    out = rd if inplace else torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    y = tern.linear_epilogue(x.cuda(), packed, scales, b.cuda(), act, col0, residual=rd, gate=g.cuda(), out=out)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    if inplace:
+        assert y.data_ptr() == rd.data_ptr()
+    y_ref = oracle.linear_epilogue(bits(x), T, s, bits(b), act, col0, bits(r), bits(g))
+    check_y(y, y_ref)
+
+
+def test_linear_batch_epilogue_mixed():
+    """A batch holding every kernel class with different epilogues, some in place."""
+    cases = [(1, 256, 192, dict(act=1)), (9, 384, 256, dict(res=True, gate=True, inplace=True)),
+             (40, 512, 256, dict(res=True)), (300, 256, 320, dict(gate=True)),
+             (70, 128, 128, dict(act=1, act_col0=64, res=True, gate=True)), (600, 512, 192, dict())]
+    probs, refs = [], []
+    for i, (M, N, K, e) in enumerate(cases):
+        W = rand_bf16((N, K), 0.02, 700 + i)
+        x = rand_bf16((M, K), 1.0, 800 + i)
+        b = rand_bf16((N,), 0.01, 900 + i)
+        r = rand_bf16((M, N), 1.0, 1000 + i) if e.get("res") else None
+        g = rand_bf16((N,), 0.5, 1100 + i) if e.get("gate") else None
+        packed, scales = quantize_on_gpu(W)
+        T, s = check_quantize(W, packed, scales, {})
+        rd = None if r is None else r.cuda()
+        y = rd if e.get("inplace") else torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        probs.append(dict(x=x.cuda(), packed=packed, scales=scales, bias=b.cuda(), y=y, act=e.get("act", 0),
+                          act_col0=e.get("act_col0", 0), residual=rd, gate=None if g is None else g.cuda()))
+        refs.append(oracle.linear_epilogue(bits(x), T, s, bits(b), e.get("act", 0), e.get("act_col0", 0),
+                                           None if r is None else bits(r), None if g is None else bits(g)))
+    tern.linear_batch_epilogue(probs)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    for p, ref in zip(probs, refs):
+        check_y(p["y"], ref)

@@ -352,3 +352,29 @@ def test_linear_act_touches_only_columns_from_col0():
     assert np.array_equal(oracle.linear_act(x, T, s, b, oracle.ACT_NONE, 0), y)
     with pytest.raises(ValueError):
         oracle.linear_act(x, T, s, b, 7, 0)
+
+
+def test_linear_epilogue_gate_and_residual_algebra():
+    """residual + gate * a: gate 0 gives the residual exactly, no residual and
+    no gate give linear_act, and the gated part scales linearly with gate."""
+    rng = np.random.default_rng(4)
+    M, K, N = 5, 128, 256
+    x = workloads.bf16_bits(torch.randn(M, K).to(torch.bfloat16))
+    T = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    s = rng.uniform(0.01, 0.03, size=N)
+    b = workloads.bf16_bits((torch.randn(N) * 0.01).to(torch.bfloat16))
+    r = workloads.bf16_bits(torch.randn(M, N).to(torch.bfloat16))
+    g = workloads.bf16_bits((torch.rand(N) * 2 - 0.5).to(torch.bfloat16))
+    zero = workloads.bf16_bits(torch.zeros(N, dtype=torch.bfloat16))
+    two = workloads.bf16_bits(torch.full((N,), 2.0, dtype=torch.bfloat16))
+    one = workloads.bf16_bits(torch.ones(N, dtype=torch.bfloat16))
+    r64 = oracle.bf16_bits_to_f64(r)
+    for act, col0 in ((oracle.ACT_NONE, 0), (oracle.ACT_GELU_TANH, 96)):
+        a = oracle.linear_act(x, T, s, b, act, col0)
+        assert np.array_equal(oracle.linear_epilogue(x, T, s, b, act, col0), a)
+        assert np.array_equal(oracle.linear_epilogue(x, T, s, b, act, col0, r, zero), r64)
+        y1 = oracle.linear_epilogue(x, T, s, b, act, col0, r, one)
+        y2 = oracle.linear_epilogue(x, T, s, b, act, col0, r, two)
+        assert np.allclose(y2 - r64, 2 * (y1 - r64), rtol=1e-14, atol=1e-14)
+        yg = oracle.linear_epilogue(x, T, s, b, act, col0, None, g)
+        assert np.allclose(yg, a * oracle.bf16_bits_to_f64(g)[None, :], rtol=1e-15, atol=0)
