@@ -100,6 +100,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// Asks for the 128-byte line holding `p` to be brought into L2 (no register
+// result, no ordering).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------------- TMA copies
 // Untiled bulk copy global -> shared, completing bytes on an mbarrier.
 // Both addresses 16-byte aligned, size a multiple of 16.

@@ -320,23 +320,30 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
               for (int e = 0; e < 4; ++e)
                 d[nb][e] += ld_shared_cluster_f32(mapa_shared(mine + uint32_t(nb * 4 + e) * 4, uint32_t(r)));
         }
+        // This lane's outputs: tokens t0 = 8 nb + 2c (+1), channels n_out
+        // (+8).  The residual may be y itself, so every residual value is
+        // read before the first store.
+        float rv[NT][4];
 #pragma unroll
-        for (int nb = 0; nb < NT; ++nb) {
-          const int t0 = 8 * nb + 2 * c;
-          const size_t m0 = size_t(t0) * P.N, m1 = m0 + P.N;
-          if (t0 < P.M) {
-            P.y[m0 + n_out] = __float2bfloat16_rn(
-                epilogue_value(fmaf(d[nb][0], s0, b0), P.act, n_out, P.act_col0, P.residual, m0 + n_out, g0));
-            P.y[m0 + n_out + 8] = __float2bfloat16_rn(
-                epilogue_value(fmaf(d[nb][2], s1, b1), P.act, n_out + 8, P.act_col0, P.residual, m0 + n_out + 8, g1));
+        for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 8 * nb + 2 * c + (e & 1);
+            const int nn = n_out + (e >> 1) * 8;
+            rv[nb][e] = (P.residual && t < P.M) ? bf16_bits_to_float(P.residual[size_t(t) * P.N + nn]) : 0.f;
           }
-          if (t0 + 1 < P.M) {
-            P.y[m1 + n_out] = __float2bfloat16_rn(
-                epilogue_value(fmaf(d[nb][1], s0, b0), P.act, n_out, P.act_col0, P.residual, m1 + n_out, g0));
-            P.y[m1 + n_out + 8] = __float2bfloat16_rn(
-                epilogue_value(fmaf(d[nb][3], s1, b1), P.act, n_out + 8, P.act_col0, P.residual, m1 + n_out + 8, g1));
+#pragma unroll
+        for (int nb = 0; nb < NT; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 8 * nb + 2 * c + (e & 1);
+            const int nn = n_out + (e >> 1) * 8;
+            if (t < P.M) {
+              const float v = fmaf(d[nb][e], e >> 1 ? s1 : s0, e >> 1 ? b1 : b0);
+              const float a = apply_act(v, P.act, nn, P.act_col0);
+              P.y[size_t(t) * P.N + nn] = __float2bfloat16_rn(fmaf(e >> 1 ? g1 : g0, a, rv[nb][e]));
+            }
           }
-        }
       }
       if (splits > 1) cluster_sync_relaxed();  // rank 0 has read every partial before they change
     } else if (splits > 1) {

@@ -188,12 +188,16 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
         uint32_t v[16];
         tmem_ld16(tmem + lane_off + c0, v);
         tmem_wait_ld();
+        float rv[16];  // residual loads of the group first (it may be y itself)
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          rv[j] = (res && row0 + c0 + j < M) ? bf16_bits_to_float(res[size_t(row0 + c0 + j) * N + n]) : 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = row0 + c0 + j;
           if (m < M)
-            P.y[size_t(m) * N + n] = __float2bfloat16_rn(epilogue_value(
-                fmaf(__uint_as_float(v[j]), sc, bi), P.act, n, P.act_col0, res, size_t(m) * N + n, gt));
+            P.y[size_t(m) * N + n] = __float2bfloat16_rn(
+                fmaf(gt, apply_act(fmaf(__uint_as_float(v[j]), sc, bi), P.act, n, P.act_col0), rv[j]));
         }
       }
     } else {

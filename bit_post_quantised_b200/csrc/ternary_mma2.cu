@@ -147,7 +147,10 @@ struct Tc<false> {
   static __device__ __forceinline__ void sync_all() { __syncthreads(); }
 };
 
-template <int TOK, bool PAIR>
+// EPI: the fused epilogues a launch needs -- 0 none, 1 activations only, 2
+// residual or gate as well.  Each level is its own instantiation, so a richer
+// epilogue cannot cost a plainer launch registers.
+template <int TOK, bool PAIR, int EPI>
 __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   using C = Cfg2<TOK, PAIR>;
   using T = Tc<PAIR>;
@@ -327,18 +330,64 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
       const float sc = 0.5f * P.scales[n];  // A held 2t
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
-      const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
-      const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
-      const bool plain = P.act == kActNone && !res && !P.gate;  // the same for the whole problem
-      const int row0 = t.m_tile * C::kTokPair + half * kCols;
-      const int rows = min(kCols, P.M - row0);
+      bool plain = true;  // the same for the whole problem
+      if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate;
+      if constexpr (EPI == 2) {
+        // Bring this tile's residual rows into L2 while its MMAs run, so the
+        // loads after the release do not wait for HBM.
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
+        if (res)
+          for (int c = 0; c < min(kCols, P.M - row0); ++c) prefetch_l2(res + size_t(row0 + c) * P.N + n);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
       tc_fence_after();
-      uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
-      if (!plain) {
-        // The epilogue's activation and residual reads run after the
-        // accumulator is released, so they overlap the next tile's MMAs:
-        // keep y in fp32 until its store.
+      if (plain || EPI == 1) {
+        uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
+        if (plain) {
+#pragma unroll
+          for (int c0 = 0; c0 < kCols; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              out[c0 / 2 + j] = pack_bf16x2(fmaf(__uint_as_float(v[2 * j]), sc, bi),
+                                            fmaf(__uint_as_float(v[2 * j + 1]), sc, bi));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        } else {
+          // Activation only: its transcendentals run after the accumulator
+          // is released, overlapping the next tile's MMAs; y stays fp32 until
+          // then.
+          float f[kCols];
+#pragma unroll
+          for (int c0 = 0; c0 < kCols; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[c0 + j] = fmaf(__uint_as_float(v[j]), sc, bi);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+#pragma unroll
+          for (int j = 0; j < kCols / 2; ++j)
+            out[j] = pack_bf16x2(apply_act(f[2 * j], P.act, n, P.act_col0),
+                                 apply_act(f[2 * j + 1], P.act, n, P.act_col0));
+        }
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+#pragma unroll
+        for (int c = 0; c < kCols; ++c)
+          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+      } else {
+        // Residual and gate (with or without the activation): fp32 until the
+        // store, everything after the release.
         float f[kCols];
 #pragma unroll
         for (int c0 = 0; c0 < kCols; c0 += 32) {
@@ -351,33 +400,27 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
-        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
         const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+        const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
+        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
 #pragma unroll
-        for (int c = 0; c < kCols; ++c)
-          if (c < rows) {
-            const float a = apply_act(f[c], act, n, act_col0);
-            const float y = rp ? fmaf(gt, a, bf16_bits_to_float(rp[c * ld])) : gt * a;
-            yp[c * ld] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-          }
-      } else {
-        uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
+        for (int c = 0; c < kCols; ++c) f[c] = apply_act(f[c], act, n, act_col0);
 #pragma unroll
-        for (int c0 = 0; c0 < kCols; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < kCols; c0 += 8) {
+          // The residual may be y itself: a group's loads all go out before
+          // its stores (an element's load precedes its own store; the others
+          // are different addresses), so they are not serialised one by one.
+          float rv[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            out[c0 / 2 + j] = pack_bf16x2(fmaf(__uint_as_float(v[2 * j]), sc, bi),
-                                          fmaf(__uint_as_float(v[2 * j + 1]), sc, bi));
+          for (int j = 0; j < 8; ++j) rv[j] = (rp && c0 + j < rows) ? bf16_bits_to_float(rp[(c0 + j) * ld]) : 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c0 + j < rows) yp[(c0 + j) * ld] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gt, f[c0 + j], rv[j])));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
-#pragma unroll
-        for (int c = 0; c < kCols; ++c)
-          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
       }
     }
   }
@@ -393,23 +436,23 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
 }
 
 // Pair tiles run as clusters of two CTAs; single-CTA tiles without clusters.
-template <int TOK>
+template <int TOK, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<TOK, true>::kThreads, 1)
     ternary_pair_kernel(const __grid_constant__ Batch batch) {
-  tile_kernel_body<TOK, true>(batch);
+  tile_kernel_body<TOK, true, EPI>(batch);
 }
-template <int TOK>
+template <int TOK, int EPI>
 __global__ void __launch_bounds__(Cfg2<TOK, false>::kThreads, 1)
     ternary_tile_kernel(const __grid_constant__ Batch batch) {
-  tile_kernel_body<TOK, false>(batch);
+  tile_kernel_body<TOK, false, EPI>(batch);
 }
-template <int TOK, bool PAIR>
+template <int TOK, bool PAIR, int EPI>
 constexpr auto tile_kernel() {
-  if constexpr (PAIR) return ternary_pair_kernel<TOK>;
-  else return ternary_tile_kernel<TOK>;
+  if constexpr (PAIR) return ternary_pair_kernel<TOK, EPI>;
+  else return ternary_tile_kernel<TOK, EPI>;
 }
 
-template <int TOK, bool PAIR>
+template <int TOK, bool PAIR, int EPI>
 static cudaError_t configure_tile() {
   static unsigned long long configured = 0;  // one bit per device ordinal
   int dev = 0;
@@ -417,7 +460,7 @@ static cudaError_t configure_tile() {
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
   if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & (1ull << dev))) {
-    e = cudaFuncSetAttribute(tile_kernel<TOK, PAIR>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tile_kernel<TOK, PAIR, EPI>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg2<TOK, PAIR>::kSmemBytes);
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
@@ -426,29 +469,45 @@ static cudaError_t configure_tile() {
 }
 
 // `ctas_or_pairs` CTAs (one-CTA tiles) or clusters of two (pair tiles).
-template <int TOK, bool PAIR>
+template <int TOK, bool PAIR, int EPI>
 static cudaError_t launch_tile(const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
   using C = Cfg2<TOK, PAIR>;
-  cudaError_t e = configure_tile<TOK, PAIR>();
+  cudaError_t e = configure_tile<TOK, PAIR, EPI>();
   if (e != cudaSuccess) return e;
-  tile_kernel<TOK, PAIR>()<<<C::kCtas * ctas_or_pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
+  tile_kernel<TOK, PAIR, EPI>()<<<C::kCtas * ctas_or_pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
-  if (pair && tok == 256) return launch_tile<256, true>(batch, ctas_or_pairs, stream);
-  if (!pair && tok == 64) return launch_tile<64, false>(batch, ctas_or_pairs, stream);
+  int epi = 0;
+  for (int i = 0; i < batch.count; ++i) {
+    if (batch.p[i].residual || batch.p[i].gate) epi = 2;
+    else if (batch.p[i].act != kActNone) epi = std::max(epi, 1);
+  }
+  if (pair && tok == 256) {
+    if (epi == 2) return launch_tile<256, true, 2>(batch, ctas_or_pairs, stream);
+    if (epi == 1) return launch_tile<256, true, 1>(batch, ctas_or_pairs, stream);
+    return launch_tile<256, true, 0>(batch, ctas_or_pairs, stream);
+  }
+  if (!pair && tok == 64) {
+    if (epi == 2) return launch_tile<64, false, 2>(batch, ctas_or_pairs, stream);
+    if (epi == 1) return launch_tile<64, false, 1>(batch, ctas_or_pairs, stream);
+    return launch_tile<64, false, 0>(batch, ctas_or_pairs, stream);
+  }
   return cudaErrorInvalidValue;
 }
 
 int max_active_clusters_2sm() {
-  if (configure_tile<256, true>() != cudaSuccess || configure_tile<64, false>() != cudaSuccess) return 0;
+  if (configure_tile<256, true, 0>() != cudaSuccess || configure_tile<256, true, 1>() != cudaSuccess ||
+      configure_tile<256, true, 2>() != cudaSuccess || configure_tile<64, false, 0>() != cudaSuccess ||
+      configure_tile<64, false, 1>() != cudaSuccess || configure_tile<64, false, 2>() != cudaSuccess)
+    return 0;
   int n = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 148);
   cfg.blockDim = dim3(Cfg2<256, true>::kThreads);
   cfg.dynamicSmemBytes = Cfg2<256, true>::kSmemBytes;
-  if (cudaOccupancyMaxActiveClusters(&n, ternary_pair_kernel<256>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&n, ternary_pair_kernel<256, 0>, &cfg) != cudaSuccess) return 0;
   return n;
 }
 
