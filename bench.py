@@ -451,9 +451,10 @@ def stack_rows(device, peaks, stream):
     """The whole ternary linear stack of one FLUX.1-dev forward at 1024x1024
     (19 double + 38 single blocks; weights drawn on the device from N(0, 0.02)
     per layer seed and quantised, only the codes kept), run block by block
-    through tern_linear_batch_act with synthetic activations and the MLP's
+    through tern_linear_batch_epilogue with synthetic activations, the MLP's
     GELU fused into its first linear (the MLP columns of a single block's
-    fused projection), and the 76 adaLN modulation GEMVs of a forward alone:
+    fused projection) and the gated residual update fused into the output
+    projections, and the 76 adaLN modulation GEMVs of a forward alone:
     batched versus one call each."""
     import torch
 
@@ -484,23 +485,30 @@ def stack_rows(device, peaks, stream):
             L = layers[i]
             if L.N not in bias:
                 bias[L.N] = (torch.randn(L.N, device=device) * 0.01).to(torch.bfloat16)
-            act, col0 = tern.ACT_NONE, 0
+            p = dict(x=buf(xs, (L.M, L.K), (L.M, L.K)), packed=packs[i][0], scales=packs[i][1], bias=bias[L.N],
+                     y=buf(ys, (j, L.M, L.N), (L.M, L.N)))
             if L.name.endswith(".mlp_up"):
-                act = tern.ACT_GELU_TANH
+                p["act"] = tern.ACT_GELU_TANH
             elif L.name.endswith(".qkv_mlp"):
-                act, col0 = tern.ACT_GELU_TANH, 3 * workloads.HIDDEN  # q, k, v, then the MLP part
-            probs.append(dict(x=buf(xs, (L.M, L.K), (L.M, L.K)), packed=packs[i][0], scales=packs[i][1],
-                              bias=bias[L.N], y=buf(ys, (j, L.M, L.N), (L.M, L.N)), act=act, act_col0=col0))
+                p["act"], p["act_col0"] = tern.ACT_GELU_TANH, 3 * workloads.HIDDEN  # q, k, v, then the MLP
+            elif L.name.endswith((".proj", ".mlp_down", ".proj_out")):
+                # gated update of a residual stream, in place (adaLN-Zero); one
+                # buffer per problem, as the problems of a batch run concurrently
+                stream_buf = buf(ys, ("stream", j, L.M, L.N), (L.M, L.N))
+                p["y"], p["residual"] = stream_buf, stream_buf
+                p["gate"] = buf(xs, ("gate", L.N), (L.N,))
+            probs.append(p)
         problems.append(probs)
     flop = sum(L.flop for L in layers)
 
     def forward():
         for probs in problems:
-            tern.linear_batch_act(probs, stream=stream)
+            tern.linear_batch_epilogue(probs, stream=stream)
 
     t = graph_time([forward], 3, stream)
-    out = {"flux_stack": {"layers": len(layers), "launch_groups": "one tern_linear_batch_act per block",
-                          "epilogue": "GELU (tanh form) fused into every MLP up projection",
+    out = {"flux_stack": {"layers": len(layers), "launch_groups": "one tern_linear_batch_epilogue per block",
+                          "epilogue": ("GELU (tanh form) fused into every MLP up projection; gated in-place "
+                                       "residual update fused into every attention/MLP output projection"),
                           "ms_per_forward": t * 1e3, "tflops": flop / t / 1e12,
                           "tensor_roofline_ms": flop / (peaks["bf16_tflops"] * 1e12) * 1e3,
                           "packed_weight_gb": sum(L.packed_bytes for L in layers) / 1e9}}
