@@ -25,6 +25,9 @@ struct alignas(64) Problem {
   int act_col0;              // first output column the activation applies to
   const __nv_bfloat16* residual;  // [M, N] or null: y = residual + gate * act(v)
   const __nv_bfloat16* gate;      // [N] or null (gate 1)
+  int norm_col0, norm_col1;       // RMS-normalised columns (128-column groups), empty if equal
+  float norm_eps;
+  const __nv_bfloat16* norm_weight;  // [N] or null (weight 1)
 };
 static_assert(sizeof(Problem) == 256, "Problem layout");
 

@@ -237,6 +237,28 @@ tern_status check_epilogue(const tern_epilogue& e, const tern_linear_args& a) {
   if (e.residual && e.residual != a.y && overlaps(e.residual, ybytes, a.y, ybytes))
     return fail(TERN_ERR_INVALID_ARG, "residual overlaps y without being y");
   if (overlaps(e.gate, e.gate ? size_t(a.N) * 2 : 0, a.y, ybytes)) return fail(TERN_ERR_INVALID_ARG, "gate overlaps y");
+  if (e.norm_col0 < 0 || e.norm_col1 < e.norm_col0 || e.norm_col1 > a.N || e.norm_col0 % 128 || e.norm_col1 % 128)
+    return fail(TERN_ERR_INVALID_ARG, "norm columns [%lld, %lld) must be 128-aligned within [0, N=%lld]",
+                (long long)e.norm_col0, (long long)e.norm_col1, (long long)a.N);
+  if (e.norm_col0 != e.norm_col1) {
+    if (!(e.norm_eps > 0.f) || !std::isfinite(e.norm_eps))
+      return fail(TERN_ERR_INVALID_ARG, "norm_eps must be finite and > 0");
+    if (!aligned(e.norm_weight, 2)) return fail(TERN_ERR_MISALIGNED, "norm_weight needs 2-byte alignment");
+    if (overlaps(e.norm_weight, e.norm_weight ? size_t(a.N) * 2 : 0, a.y, ybytes))
+      return fail(TERN_ERR_INVALID_ARG, "norm_weight overlaps y");
+  }
+  return TERN_OK;
+}
+
+// The RMS normalisation exists only in the tcgen05 tile kernels: N % 256 ==
+// 0 and M > 16 (checked without a device), and the device able to run the
+// CTA-pair kernel for M > 64 (ptok from pair_tok; checked once it is known).
+tern_status check_norm_route(const tern_epilogue& e, const tern_linear_args& a, int ptok = -1) {
+  if (e.norm_col0 == e.norm_col1 || a.M == 0) return TERN_OK;
+  if (a.N % 256 != 0 || a.M <= 16 || ptok == 0)
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE,
+                "the RMS-normalising epilogue needs N %% 256 == 0 and M > 16 (M=%lld N=%lld)", (long long)a.M,
+                (long long)a.N);
   return TERN_OK;
 }
 
@@ -246,6 +268,10 @@ void set_epilogue(Problem* p, const tern_epilogue* epis, int i) {
   p->act_col0 = int(epis[i].act_col0);
   p->residual = static_cast<const __nv_bfloat16*>(epis[i].residual);
   p->gate = static_cast<const __nv_bfloat16*>(epis[i].gate);
+  p->norm_col0 = int(epis[i].norm_col0);
+  p->norm_col1 = int(epis[i].norm_col1);
+  p->norm_eps = epis[i].norm_eps;
+  p->norm_weight = static_cast<const __nv_bfloat16*>(epis[i].norm_weight);
 }
 
 // Up to 16 tokens run on the register-fed GEMV kernel, in n8 blocks.
@@ -457,10 +483,12 @@ tern_status linear_impl(const tern_linear_args& a, const tern_epilogue& epi, ter
   tern_status s = check_linear(a);
   if (s != TERN_OK) return s;
   if ((s = check_epilogue(epi, a)) != TERN_OK) return s;
+  if ((s = check_norm_route(epi, a)) != TERN_OK) return s;
   if (M == 0) return TERN_OK;
   int dev;
   DeviceState* ds;
   if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  if ((s = check_norm_route(epi, a, pair_tok(a, ds))) != TERN_OK) return s;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   if (M <= kGemvMaxM) {
@@ -504,6 +532,7 @@ tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, 
   for (int i = 0; i < count; ++i) {
     tern_status s = check_linear(args[i]);
     if (s == TERN_OK && epis) s = check_epilogue(epis[i], args[i]);
+    if (s == TERN_OK && epis) s = check_norm_route(epis[i], args[i]);
     if (s != TERN_OK) {
       t_last_error = "problem " + std::to_string(i) + ": " + t_last_error;
       return s;
@@ -514,6 +543,11 @@ tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, 
   DeviceState* ds;
   tern_status s = current_device(&dev, &ds);
   if (s != TERN_OK) return s;
+  for (int i = 0; epis && i < count; ++i)
+    if ((s = check_norm_route(epis[i], args[i], pair_tok(args[i], ds))) != TERN_OK) {
+      t_last_error = "problem " + std::to_string(i) + ": " + t_last_error;
+      return s;
+    }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   static Batch batch;

@@ -147,9 +147,30 @@ struct Tc<false> {
   static __device__ __forceinline__ void sync_all() { __syncthreads(); }
 };
 
+// Sums a[i] over the 32 lanes of the warp for every i and leaves the sum for
+// i = lane * (N / 32) + j in a[j], j < N / 32 (the other entries are dead).
+// Five butterfly steps, each halving the entries a lane keeps: N - N/32
+// shuffles in all.
+template <int N>
+__device__ __forceinline__ void warp_reduce_scatter(float (&a)[N], int lane) {
+  static_assert(N >= 32 && (N & (N - 1)) == 0, "N");
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int o = 16 >> step, half = (N >> step) / 2;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < half; ++j) {
+      const float send = up ? a[j] : a[j + half];
+      const float keep = up ? a[j + half] : a[j];
+      a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
 // EPI: the fused epilogues a launch needs -- 0 none, 1 activations only, 2
-// residual or gate as well.  Each level is its own instantiation, so a richer
-// epilogue cannot cost a plainer launch registers.
+// residual or gate as well, 3 RMS normalisation of 128-channel groups as
+// well.  Each level is its own instantiation, so a richer epilogue cannot
+// cost a plainer launch registers.
 template <int TOK, bool PAIR, int EPI>
 __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   using C = Cfg2<TOK, PAIR>;
@@ -166,6 +187,13 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   __shared__ __align__(8) uint64_t accempty_bar[AB]; // leader: both epilogues drained TMEM
   __shared__ __align__(8) uint64_t drain_bar;        // leader: every MMA issued is done
   __shared__ uint32_t tmem_base_sh;
+  // RMS normalisation (EPI == 3): per 64-token column group ("half") of the
+  // epilogue, each lane quarter's partial sums of squares, the inverse RMS per
+  // token, and two barriers (partials written, inverses written).
+  constexpr int kHalves = C::kEpiWarps / 4;
+  __shared__ float norm_part[EPI == 3 ? kHalves * 4 * C::kEpiCols : 1];
+  __shared__ float norm_inv[EPI == 3 ? kHalves * C::kEpiCols : 1];
+  __shared__ __align__(8) uint64_t norm_bar[EPI == 3 ? 2 * kHalves : 1];
   extern __shared__ uint8_t dyn_smem[];
 
   const uint64_t lim = batch.wait_limit_ns;
@@ -193,6 +221,8 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       mbar_init(smem_u32(&accempty_bar[b]), C::kCtas * C::kEpiWarps);
     }
     mbar_init(smem_u32(&drain_bar), 1);
+    if constexpr (EPI == 3)
+      for (int h = 0; h < 2 * kHalves; ++h) mbar_init(smem_u32(&norm_bar[h]), 4);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -323,6 +353,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t accempty_leader0 = T::leader_addr(smem_u32(&accempty_bar[0]));
     int lt = 0;
+    int norm_it = 0;  // normalised tiles so far (the phase of norm_bar)
     for (int u = u0; u < units; u += ustep, ++lt) {
       const Tile2 t = tile_of(batch, u);
       const Problem& P = *t.P;
@@ -331,8 +362,8 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const float sc = 0.5f * P.scales[n];  // A held 2t
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       bool plain = true;  // the same for the whole problem
-      if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate;
-      if constexpr (EPI == 2) {
+      if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate && P.norm_col0 == P.norm_col1;
+      if constexpr (EPI >= 2) {
         // Bring this tile's residual rows into L2 while its MMAs run, so the
         // loads after the release do not wait for HBM.
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
@@ -385,6 +416,77 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
           if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+      } else if (EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1) {
+        // RMS normalisation: the CTA's 128 channels are one group (n - r and
+        // the bounds are multiples of 128), so every warp of the CTA takes
+        // this branch for the tile.  The per-token sums of squares need all
+        // four lane quarters, so the accumulator is held (read twice from
+        // TMEM) until the normalised, activated and combined values are
+        // stored; registers hold 32 columns at a time.
+        constexpr int kChunk = 32;
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
+        bool ok_n = true;
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += kChunk) {
+          uint32_t v[kChunk];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
+          float sq[kChunk];
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) {
+            const float y = fmaf(__uint_as_float(v[j]), sc, bi);
+            sq[j] = y * y;
+          }
+          warp_reduce_scatter<kChunk>(sq, lane);  // token c0 + lane, this warp's 32 channels
+          norm_part[(half * 4 + quarter) * kCols + c0 + lane] = sq[0];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&norm_bar[2 * half]));
+        ok_n = mbar_wait(smem_u32(&norm_bar[2 * half]), norm_it & 1, lim, st);
+        if (quarter == 0 && ok_n)
+          for (int c = lane; c < kCols; c += 32) {
+            const float tot = (norm_part[(half * 4 + 0) * kCols + c] + norm_part[(half * 4 + 1) * kCols + c]) +
+                              (norm_part[(half * 4 + 2) * kCols + c] + norm_part[(half * 4 + 3) * kCols + c]);
+            norm_inv[half * kCols + c] = rsqrtf(tot * (1.0f / 128.0f) + P.norm_eps);
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&norm_bar[2 * half + 1]));
+        ok_n = mbar_wait(smem_u32(&norm_bar[2 * half + 1]), norm_it & 1, lim, st) && ok_n;
+        ++norm_it;
+        if (!__all_sync(0xffffffffu, ok_n)) break;
+        const float w = P.norm_weight ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.norm_weight)[n]) : 1.f;
+        const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+        const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
+        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += kChunk) {
+          uint32_t v[kChunk];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int g0 = 0; g0 < kChunk; g0 += 8) {
+            float rv[8];  // residual loads of the group go out before its stores
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = c0 + g0 + j;
+              rv[j] = (rp && c < rows) ? bf16_bits_to_float(rp[c * ld]) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = c0 + g0 + j;
+              if (c < rows) {
+                const float y = fmaf(__uint_as_float(v[g0 + j]), sc, bi) * (norm_inv[half * kCols + c] * w);
+                yp[c * ld] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gt, apply_act(y, act, n, act_col0), rv[j])));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
       } else {
         // Residual and gate (with or without the activation): fp32 until the
         // store, everything after the release.
@@ -481,15 +583,18 @@ static cudaError_t launch_tile(const Batch& batch, int ctas_or_pairs, cudaStream
 cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
   int epi = 0;
   for (int i = 0; i < batch.count; ++i) {
-    if (batch.p[i].residual || batch.p[i].gate) epi = 2;
+    if (batch.p[i].norm_col0 != batch.p[i].norm_col1) epi = 3;
+    else if (batch.p[i].residual || batch.p[i].gate) epi = std::max(epi, 2);
     else if (batch.p[i].act != kActNone) epi = std::max(epi, 1);
   }
   if (pair && tok == 256) {
+    if (epi == 3) return launch_tile<256, true, 3>(batch, ctas_or_pairs, stream);
     if (epi == 2) return launch_tile<256, true, 2>(batch, ctas_or_pairs, stream);
     if (epi == 1) return launch_tile<256, true, 1>(batch, ctas_or_pairs, stream);
     return launch_tile<256, true, 0>(batch, ctas_or_pairs, stream);
   }
   if (!pair && tok == 64) {
+    if (epi == 3) return launch_tile<64, false, 3>(batch, ctas_or_pairs, stream);
     if (epi == 2) return launch_tile<64, false, 2>(batch, ctas_or_pairs, stream);
     if (epi == 1) return launch_tile<64, false, 1>(batch, ctas_or_pairs, stream);
     return launch_tile<64, false, 0>(batch, ctas_or_pairs, stream);
@@ -499,8 +604,9 @@ cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas
 
 int max_active_clusters_2sm() {
   if (configure_tile<256, true, 0>() != cudaSuccess || configure_tile<256, true, 1>() != cudaSuccess ||
-      configure_tile<256, true, 2>() != cudaSuccess || configure_tile<64, false, 0>() != cudaSuccess ||
-      configure_tile<64, false, 1>() != cudaSuccess || configure_tile<64, false, 2>() != cudaSuccess)
+      configure_tile<256, true, 2>() != cudaSuccess || configure_tile<256, true, 3>() != cudaSuccess ||
+      configure_tile<64, false, 0>() != cudaSuccess || configure_tile<64, false, 1>() != cudaSuccess ||
+      configure_tile<64, false, 2>() != cudaSuccess || configure_tile<64, false, 3>() != cudaSuccess)
     return 0;
   int n = 0;
   cudaLaunchConfig_t cfg = {};

@@ -50,7 +50,8 @@ class LinearActArgs(ctypes.Structure):
 class Epilogue(ctypes.Structure):
     """Mirror of tern_epilogue."""
     _fields_ = [("act", ctypes.c_int), ("act_col0", ctypes.c_int64), ("residual", ctypes.c_void_p),
-                ("gate", ctypes.c_void_p)]
+                ("gate", ctypes.c_void_p), ("norm_col0", ctypes.c_int64), ("norm_col1", ctypes.c_int64),
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
 
 
 ACT_NONE = 0       # tern_act values
@@ -211,21 +212,26 @@ def _linear_args(p: dict) -> LinearArgs:
 
 
 def _epilogue(p: dict) -> Epilogue:
-    return Epilogue(p.get("act", ACT_NONE), p.get("act_col0", 0), _ptr(p.get("residual")), _ptr(p.get("gate")))
+    return Epilogue(p.get("act", ACT_NONE), p.get("act_col0", 0), _ptr(p.get("residual")), _ptr(p.get("gate")),
+                    p.get("norm_col0", 0), p.get("norm_col1", 0), _ptr(p.get("norm_weight")),
+                    p.get("norm_eps", 0.0))
 
 
 def linear_epilogue(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
                     bias: Optional[torch.Tensor] = None, act: int = ACT_NONE, act_col0: int = 0,
                     residual: Optional[torch.Tensor] = None, gate: Optional[torch.Tensor] = None,
+                    norm_cols=(0, 0), norm_weight: Optional[torch.Tensor] = None, norm_eps: float = 0.0,
                     out: Optional[torch.Tensor] = None, stream=None):
-    """tern_linear_epilogue: y = residual + gate * act(x . T^T * s + b) (see
-    tern_epilogue); `out` may be `residual` itself for an in-place update."""
+    """tern_linear_epilogue: y = residual + gate * act(norm(x . T^T * s + b))
+    (see tern_epilogue); `out` may be `residual` itself for an in-place
+    update; norm_cols = (first, end) of the RMS-normalised columns."""
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     a = _linear_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
-    e = _epilogue(dict(act=act, act_col0=act_col0, residual=residual, gate=gate))
+    e = _epilogue(dict(act=act, act_col0=act_col0, residual=residual, gate=gate, norm_col0=norm_cols[0],
+                       norm_col1=norm_cols[1], norm_weight=norm_weight, norm_eps=norm_eps))
     _check(lib().tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
     return out
 

@@ -172,7 +172,8 @@ typedef struct {
 } tern_linear_args;
 
 /*
- * A fused epilogue.  With v = s_n * sum_k x[m,k] * T[n,k] + b_n in fp32:
+ * A fused epilogue.  With v = s_n * sum_k x[m,k] * T[n,k] + b_n in fp32
+ * (RMS-normalised first on the normalised columns, see norm_col0 below):
  *     a = act(v) for n >= act_col0, else v;
  *     y[m,n] = residual[m,n] + gate[n] * a     (residual NULL: 0; gate NULL: 1),
  * in fp32, then one rounding to bf16.  All zero is the plain layer.
@@ -193,6 +194,15 @@ typedef struct {
   int64_t act_col0;     /* first activated output column */
   const void* residual; /* [M, N] bf16 or NULL */
   const void* gate;     /* [N] bf16 or NULL */
+  /* RMS normalisation over groups of 128 consecutive output columns (one
+   * attention head of FLUX.1's q or k) on columns [norm_col0, norm_col1),
+   * both multiples of 128 (equal: none), applied first, to v itself:
+   *     v <- v / sqrt(mean over the token's group of v^2 + norm_eps) * norm_weight[n].
+   * Only where the layer runs on the tcgen05 tile kernels (N % 256 == 0 and
+   * M > 16); elsewhere a requested normalisation is TERN_ERR_UNSUPPORTED_SHAPE. */
+  int64_t norm_col0, norm_col1;
+  const void* norm_weight; /* [N] bf16 or NULL (weight 1) */
+  float norm_eps;          /* > 0 and finite when a normalisation is requested */
 } tern_epilogue;
 
 /* tern_linear of *args with the fused epilogue *epilogue (NULL: none). */

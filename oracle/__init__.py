@@ -223,15 +223,42 @@ def linear_act(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, ac
     raise ValueError("unknown activation")
 
 
+def rms_norm_groups(y: np.ndarray, col0: int, col1: int, eps: float, w_bits=None, group: int = 128) -> np.ndarray:
+    """RMS normalisation of every token row over each group of `group`
+    consecutive columns in [col0, col1): v / sqrt(mean(v^2) + eps) * w[n]
+    (w bf16 bit patterns [N], absent = 1); other columns unchanged.  FLUX.1
+    normalises q and k per attention head (128 channels) this way."""
+    y = np.array(y, dtype=np.float64, order="C", copy=True)
+    M, N = y.shape
+    if not (0 <= col0 <= col1 <= N and col0 % group == 0 and col1 % group == 0):
+        raise ValueError("norm columns must be group-aligned within [0, N]")
+    w = np.ones(N) if w_bits is None else bf16_bits_to_f64(_c(w_bits, np.uint16))
+    for g0 in range(col0, col1, group):
+        blk = y[:, g0:g0 + group]
+        inv = 1.0 / np.sqrt(np.mean(blk * blk, axis=1, keepdims=True) + eps)
+        y[:, g0:g0 + group] = blk * inv * w[None, g0:g0 + group]
+    return y
+
+
 def linear_epilogue(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, act: int = ACT_NONE,
-                    col0: int = 0, residual_bits=None, gate_bits=None) -> np.ndarray:
-    """The layer with a fused epilogue, in float64: a = act(v) on columns
-    [col0, N) of v = linear(...), then residual + gate * a (residual [M, N]
-    and gate [N] are bf16 bit patterns; absent residual = 0, absent gate = 1).
-    FLUX.1 adds its attention and MLP outputs to the residual stream scaled by
-    an adaLN-Zero gate; the pages describe no operation between the quantised
-    linears, so this follows that model's definition."""
-    a = linear_act(x_bits, T, s, b_bits, act, col0)
+                    col0: int = 0, residual_bits=None, gate_bits=None, norm_cols=(0, 0), norm_w_bits=None,
+                    norm_eps: float = 0.0) -> np.ndarray:
+    """The layer with a fused epilogue, in float64: v = linear(...),
+    RMS-normalised per 128-column group on norm_cols, a = act(v) on columns
+    [col0, N), then residual + gate * a (residual [M, N] and gate [N] are bf16
+    bit patterns; absent residual = 0, absent gate = 1).  FLUX.1 normalises
+    q and k per head and adds its attention and MLP outputs to the residual
+    stream scaled by an adaLN-Zero gate; the pages describe no operation
+    between the quantised linears, so this follows that model's definition."""
+    v = linear(x_bits, T, s, b_bits)
+    if norm_cols[1] > norm_cols[0]:
+        v = rms_norm_groups(v, norm_cols[0], norm_cols[1], norm_eps, norm_w_bits)
+    if act == ACT_GELU_TANH:
+        a = gelu_tanh(v, col0)
+    elif act == ACT_NONE:
+        a = v
+    else:
+        raise ValueError("unknown activation")
     if gate_bits is not None:
         g = bf16_bits_to_f64(_c(gate_bits, np.uint16))
         if g.shape != (a.shape[1],):

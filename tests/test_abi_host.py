@@ -184,3 +184,20 @@ def test_epilogue_rejects_on_host(L):
     assert L.tern_linear_epilogue(None, None, None) == INVALID
     assert L.tern_linear_batch_epilogue(None, None, 2, None) == INVALID
     assert L.tern_linear_batch_epilogue(None, None, 0, None) == 0
+
+
+def test_norm_epilogue_rejects_on_host(L):
+    """The RMS-normalising epilogue: 128-aligned column bounds within [0, N],
+    eps > 0, and only shapes that run on the tcgen05 tile kernels."""
+    def call(M=40, N=256, c0=0, c1=128, eps=1e-6, w=None):
+        a = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, M, N, 256)
+        e = tern.Epilogue(0, 0, None, None, c0, c1, w, eps)
+        return L.tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), None)
+    assert call(c0=64) == INVALID
+    assert call(c1=384) == INVALID
+    assert call(c0=128, c1=0) == INVALID
+    assert call(eps=0.0) == INVALID
+    assert call(eps=float("nan")) == INVALID
+    assert call(w=F + 0x500001) == MISALIGNED
+    assert call(M=16) == SHAPE            # would run on the GEMV
+    assert call(N=384, c1=128) == SHAPE   # would run on the fallback kernel

@@ -441,3 +441,71 @@ def test_linear_batch_epilogue_mixed():
     assert tern.device_status() == 0
     for p, ref in zip(probs, refs):
         check_y(p["y"], ref)
+
+
+# ------------------------------------------------ RMS normalisation of 128-channel groups
+@pytest.mark.parametrize("M,N,K,cols,act,res", [
+    (300, 512, 192, (0, 256), 0, False),      # CTA-pair tiles: the first pair tile normalised
+    (300, 512, 192, (128, 384), 1, True),     # one CTA of each pair tile, with GELU and residual
+    (1024, 1024, 512, (0, 768), 0, False),    # several tiles per CTA pair (barrier phases)
+    (40, 512, 256, (128, 384), 0, False),     # 64-token tiles
+    (64, 768, 320, (0, 768), 0, True),        # 64-token tiles, all normalised, residual in place
+])
+def test_linear_epilogue_rms_norm(M, N, K, cols, act, res):
+    W = rand_bf16((N, K), 0.02, M + 13 * N)
+    x = rand_bf16((M, K), 1.0, M + 17 * K)
+    b = rand_bf16((N,), 0.01, N + 19)
+    w = (torch.rand(N, generator=torch.Generator().manual_seed(N)) + 0.5).to(torch.bfloat16)
+    r = rand_bf16((M, N), 1.0, M * N + 3) if res else None
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    rd = None if r is None else r.cuda()
+    out = rd if res else torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    y = tern.linear_epilogue(x.cuda(), packed, scales, b.cuda(), act, 0, residual=rd, norm_cols=cols,
+                             norm_weight=w.cuda(), norm_eps=1e-6, out=out)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    y_ref = oracle.linear_epilogue(bits(x), T, s, bits(b), act, 0, None if r is None else bits(r), None, cols,
+                                   bits(w), 1e-6)
+    check_y(y, y_ref)
+
+
+def test_linear_epilogue_rms_norm_flux_qkv_sampled():
+    """The FLUX QKV projection with q and k normalised per 128-channel head
+    (columns [0, 6144)), full size, sampled rows."""
+    L = workloads.CONFIGS["qkv"]
+    x, W, b = workloads.make_inputs(L)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    w = (torch.rand(L.N, generator=torch.Generator().manual_seed(2)) + 0.5).to(torch.bfloat16)
+    y = tern.linear_epilogue(x.cuda(), packed, scales, b.cuda(), norm_cols=(0, 2 * workloads.HIDDEN),
+                             norm_weight=w.cuda(), norm_eps=1e-6)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    rows = np.sort(np.random.default_rng(21).choice(L.M, 24, replace=False))
+    rows[-1] = L.M - 1
+    ref = oracle.linear_epilogue(bits(x[rows]), T, s, bits(b), 0, 0, None, None, (0, 2 * workloads.HIDDEN),
+                                 bits(w), 1e-6)
+    check_y(y[torch.from_numpy(rows).cuda()], ref)
+
+
+def test_linear_batch_epilogue_with_norm():
+    """A batch where one pair-tile problem normalises and the others do not:
+    the whole launch runs the normalising kernel."""
+    cases = [(300, 512, 192, (0, 256)), (600, 256, 320, (0, 0)), (40, 256, 256, (0, 256))]
+    probs, refs = [], []
+    for i, (M, N, K, cols) in enumerate(cases):
+        W = rand_bf16((N, K), 0.02, 1200 + i)
+        x = rand_bf16((M, K), 1.0, 1300 + i)
+        b = rand_bf16((N,), 0.01, 1400 + i)
+        packed, scales = quantize_on_gpu(W)
+        T, s = check_quantize(W, packed, scales, {})
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        probs.append(dict(x=x.cuda(), packed=packed, scales=scales, bias=b.cuda(), y=y, norm_col0=cols[0],
+                          norm_col1=cols[1], norm_eps=1e-6))
+        refs.append(oracle.linear_epilogue(bits(x), T, s, bits(b), 0, 0, None, None, cols, None, 1e-6))
+    tern.linear_batch_epilogue(probs)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    for p, ref in zip(probs, refs):
+        check_y(p["y"], ref)

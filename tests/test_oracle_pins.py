@@ -378,3 +378,28 @@ def test_linear_epilogue_gate_and_residual_algebra():
         assert np.allclose(y2 - r64, 2 * (y1 - r64), rtol=1e-14, atol=1e-14)
         yg = oracle.linear_epilogue(x, T, s, b, act, col0, None, g)
         assert np.allclose(yg, a * oracle.bf16_bits_to_f64(g)[None, :], rtol=1e-15, atol=0)
+
+
+def test_rms_norm_groups_properties_and_torch():
+    """Per-128-column RMS normalisation: unit mean square per group (eps 0),
+    scale invariance, groups independent, columns outside untouched, and
+    torch's rms_norm on each group."""
+    rng = np.random.default_rng(9)
+    y = rng.normal(0.0, 2.0, size=(6, 512))
+    n = oracle.rms_norm_groups(y, 128, 384, 0.0)
+    assert np.array_equal(n[:, :128], y[:, :128]) and np.array_equal(n[:, 384:], y[:, 384:])
+    for g0 in (128, 256):
+        assert np.allclose(np.mean(n[:, g0:g0 + 128] ** 2, axis=1), 1.0, rtol=1e-13)
+    assert np.allclose(oracle.rms_norm_groups(3.5 * y, 128, 384, 0.0)[:, 128:384], n[:, 128:384], rtol=1e-13,
+                       atol=1e-15)
+    y2 = y.copy()
+    y2[:, 128:256] *= 7.0
+    assert np.array_equal(oracle.rms_norm_groups(y2, 128, 384, 0.0)[:, 256:384], n[:, 256:384])
+    w = workloads.bf16_bits((torch.rand(512) + 0.5).to(torch.bfloat16))
+    got = oracle.rms_norm_groups(y, 0, 512, 1e-6, w)
+    wt = torch.from_numpy(oracle.bf16_bits_to_f64(w))
+    for g0 in range(0, 512, 128):
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(y[:, g0:g0 + 128]), (128,), wt[g0:g0 + 128], 1e-6)
+        assert np.allclose(got[:, g0:g0 + 128], ref.numpy(), rtol=1e-12, atol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.rms_norm_groups(y, 64, 256, 1e-6)
