@@ -457,36 +457,40 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         if (!__all_sync(0xffffffffu, ok_n)) break;
         const float w = P.norm_weight ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.norm_weight)[n]) : 1.f;
         const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
-        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
         const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
         const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
         const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
+        uint32_t out[kCols / 2];  // the finished values, bf16x2; stored after the release
 #pragma unroll
-        for (int c0 = 0; c0 < kCols; c0 += kChunk) {
-          uint32_t v[kChunk];
-          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+        for (int c0 = 0; c0 < kCols; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int g0 = 0; g0 < kChunk; g0 += 8) {
-            float rv[8];  // residual loads of the group go out before its stores
+          for (int g0 = 0; g0 < 16; g0 += 8) {
+            float rv[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const int c = c0 + g0 + j;
               rv[j] = (rp && c < rows) ? bf16_bits_to_float(rp[c * ld]) : 0.f;
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 8; j += 2) {
               const int c = c0 + g0 + j;
-              if (c < rows) {
-                const float y = fmaf(__uint_as_float(v[g0 + j]), sc, bi) * (norm_inv[half * kCols + c] * w);
-                yp[c * ld] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(gt, apply_act(y, act, n, act_col0), rv[j])));
-              }
+              const float y0 = fmaf(__uint_as_float(v[g0 + j]), sc, bi) * (norm_inv[half * kCols + c] * w);
+              const float y1 = fmaf(__uint_as_float(v[g0 + j + 1]), sc, bi) * (norm_inv[half * kCols + c + 1] * w);
+              out[c / 2] = pack_bf16x2(fmaf(gt, apply_act(y0, act, n, act_col0), rv[j]),
+                                       fmaf(gt, apply_act(y1, act, n, act_col0), rv[j + 1]));
             }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+#pragma unroll
+        for (int c = 0; c < kCols; ++c)
+          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
       } else {
         // Residual and gate (with or without the activation): fp32 until the
         // store, everything after the release.
