@@ -12,8 +12,8 @@
 // rows of the fp32 accumulator.  One instruction is 128 tensor cycles per
 // SM, and every x byte brought from L2 feeds 256 channels.
 //
-// Per CTA, per 128-wide k stage (36 KiB of shared memory, 6 stages; the last
-// stage of a row holds 64 k when K % 128 == 64):
+// Per CTA, per 128-wide k stage (36 KiB of shared memory, 6 stages, 4 with a
+// residual epilogue; the last stage of a row holds 64 k when K % 128 == 64):
 //   * warp 0 (producer): one 3-D TMA copy of its 128 x-rows x 128 k (two
 //     64-k chunks, 128-byte swizzle) and one bulk copy of its codes (128
 //     channels x 128 k, contiguous in the tile-interleaved layout), both
@@ -27,12 +27,16 @@
 //     from each CTA), issues the eight MMAs of the stage and commits, with
 //     one arrival in both CTAs, to empty[s] (shared-memory stage free) and
 //     aempty[a] (TMEM slot free).  The whole warp computes the operands and
-//     lane 0 issues the stage as one block, so the operands stay uniform.  Eight MMAs (1024 tensor cycles) between
-//     two waits of the issuing thread keep the tensor pipe fed; a wait every
-//     four MMAs measurably starves it.
-//   * warps 6-13 (epilogue): after the tile's last MMA, tcgen05.ld of the
-//     accumulator into registers, release to the leader at once (so the next
-//     tile's MMAs start), then y = acc * s + b rounded to bf16 and stored.
+//     its elected lane issues the stage as one block, so the operands stay
+//     uniform.  Eight MMAs (1024 tensor cycles) between two waits of the
+//     issuing thread keep the tensor pipe fed; a wait every four MMAs
+//     measurably starves it.
+//   * warps 6-21 (epilogue, 64 tokens each): after the tile's last MMA,
+//     tcgen05.ld of the accumulator into registers, release to the leader at
+//     once (the single accumulator holds up the next tile's MMAs until
+//     then), then y = acc * s + b rounded to bf16 and stored.  A residual
+//     epilogue copies each warp's residual slice into shared memory while
+//     the tile's MMAs run, so after the release it reads shared memory only.
 // Work is persistent: cluster c takes tiles c, c + #clusters, ...  No TMA
 // multicast is used: every copy reads this GPU's global memory into the
 // issuing CTA's own shared memory.
@@ -52,7 +56,10 @@ namespace {
 // !PAIR: one CTA per tile (cta_group::1, M = 128 channels, all TOK x rows),
 // used for TOK = 64, where a pair instruction would take as long as at
 // N = 256 but do a quarter of the work.
-template <int TOK, bool PAIR>
+// EPI >= 2 (residual or gate epilogues) trades two x stages for a shared
+// memory slice per epilogue warp where each tile's residual lands while its
+// MMAs run (4 stages keep the tensor pipe as busy as 6 on the plain layer).
+template <int TOK, bool PAIR, int EPI = 0>
 struct Cfg2 {
   static constexpr int kTokPair = TOK;
   static constexpr int kTokCta = PAIR ? TOK / 2 : TOK;  // x rows each CTA loads
@@ -64,7 +71,8 @@ struct Cfg2 {
   static constexpr int kCSub = 128 * 16;          // codes of 128 channels x 64 k
   static constexpr int kCBytes = 2 * kCSub;
   static constexpr int kStageBytes = kXBytes + kCBytes;
-  static constexpr int kStages = kStageBytes > 24 * 1024 ? 6 : 8;
+  static constexpr bool kResStaged = EPI >= 2;
+  static constexpr int kStages = kStageBytes > 24 * 1024 ? (kResStaged ? 4 : 6) : 8;
   static constexpr int kASlots = 4;               // decoded-weight slots in TMEM
   static constexpr int kACols = kBK / 2;          // 32-bit TMEM columns per slot (bf16x2)
   static constexpr int kDCols = TOK;              // one accumulator
@@ -82,7 +90,10 @@ struct Cfg2 {
   static constexpr int kEpiCols = TOK / (kEpiWarps / 4);
   static constexpr int kEpiWarp0 = 2 + kDecWarps;
   static constexpr int kThreads = (2 + kDecWarps + kEpiWarps) * 32;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // Residual slice of one epilogue warp: its kEpiCols tokens x 32 channels, bf16.
+  static constexpr int kResWarpBytes = kEpiCols * 64;
+  static constexpr int kResBytes = kResStaged ? kEpiWarps * kResWarpBytes : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kResBytes + 1024;
   static constexpr int kCtas = PAIR ? 2 : 1;      // CTAs sharing one MMA
   // kind::f16, D fp32, A/B bf16 K-major, N = TOK, M = 128 per CTA of the MMA.
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -90,7 +101,7 @@ struct Cfg2 {
   static_assert(TOK % 64 == 0 && TOK >= 64 && TOK <= 256, "UMMA N; 32-column epilogue loads per half");
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
   static_assert(kACol0 + kASlots * kACols <= kTmemCols, "TMEM columns");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kSmemBytes + 6 * 1024 <= 227 * 1024, "shared memory, with the static barriers and norm sums");
 };
 
 struct Tile2 {
@@ -173,7 +184,7 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&a)[N], int lane) {
 // cost a plainer launch registers.
 template <int TOK, bool PAIR, int EPI>
 __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
-  using C = Cfg2<TOK, PAIR>;
+  using C = Cfg2<TOK, PAIR, EPI>;
   using T = Tc<PAIR>;
   constexpr int S = C::kStages;
   constexpr int A = C::kASlots;
@@ -194,6 +205,8 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   __shared__ float norm_part[EPI == 3 ? kHalves * 4 * C::kEpiCols : 1];
   __shared__ float norm_inv[EPI == 3 ? kHalves * C::kEpiCols : 1];
   __shared__ __align__(8) uint64_t norm_bar[EPI == 3 ? 2 * kHalves : 1];
+  // EPI >= 2: per epilogue warp, its residual slice of the tile has landed.
+  __shared__ __align__(8) uint64_t res_bar[C::kResStaged ? C::kEpiWarps : 1];
   extern __shared__ uint8_t dyn_smem[];
 
   const uint64_t lim = batch.wait_limit_ns;
@@ -223,6 +236,8 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     mbar_init(smem_u32(&drain_bar), 1);
     if constexpr (EPI == 3)
       for (int h = 0; h < 2 * kHalves; ++h) mbar_init(smem_u32(&norm_bar[h]), 4);
+    if constexpr (C::kResStaged)
+      for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(smem_u32(&res_bar[w]), 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -354,6 +369,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     const uint32_t accempty_leader0 = T::leader_addr(smem_u32(&accempty_bar[0]));
     int lt = 0;
     int norm_it = 0;  // normalised tiles so far (the phase of norm_bar)
+    int res_it = 0;   // residual slices staged so far (the phase of res_bar[ew])
     for (int u = u0; u < units; u += ustep, ++lt) {
       const Tile2 t = tile_of(batch, u);
       const Problem& P = *t.P;
@@ -363,17 +379,92 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       bool plain = true;  // the same for the whole problem
       if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate && P.norm_col0 == P.norm_col1;
+      // Residual and gate without an activation ("early"): this warp's
+      // slice of the tile's residual (its 32 channels of kCols tokens, 64
+      // bytes per token) is copied into shared memory while the tile's MMAs
+      // run, and combined before the accumulator is released; after the
+      // release only the stores remain.  (Read from global memory after the
+      // release, the residual's round trips would hold up the next tile.)
+      bool early = false, staged = false;
+      float gt = 1.f;
       if constexpr (EPI >= 2) {
-        // Bring this tile's residual rows into L2 while its MMAs run, so the
-        // loads after the release do not wait for HBM.
-        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const bool normed = EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1;
         const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
-        if (res)
-          for (int c = 0; c < min(kCols, P.M - row0); ++c) prefetch_l2(res + size_t(row0 + c) * P.N + n);
+        early = !plain && !normed && P.act == kActNone && (reinterpret_cast<uintptr_t>(res) & 15) == 0;
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = max(0, min(kCols, P.M - row0));
+        if (early) {
+          if (P.gate) gt = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]);
+          if (res) {
+            // The warp read its previous slice before its last release.
+            fence_proxy_async_smem();
+            const uint32_t bar = smem_u32(&res_bar[ew]);
+            const uint32_t dst = smem_base + C::kStages * C::kStageBytes + ew * C::kResWarpBytes;
+            // 16-byte aligned: res is, N is a multiple of 128 and n - lane of 32
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(res + size_t(row0) * P.N + (n - lane));
+            if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(rows) * 64u);
+            __syncwarp();
+            for (int c = lane; c < rows; c += 32) tma_load_bulk(dst + c * 64, src + size_t(c) * P.N * 2, 64, bar);
+            staged = true;
+          }
+        } else if (res) {
+          // Otherwise bring the residual rows into L2, so the loads after the
+          // release do not wait for HBM.
+          for (int c = 0; c < rows; ++c) prefetch_l2(res + size_t(row0 + c) * P.N + n);
+        }
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) {
+        if (staged) mbar_wait(smem_u32(&res_bar[ew]), res_it & 1, lim, st);  // no copy may land after exit
+        break;
+      }
       tc_fence_after();
-      if (plain || EPI == 1) {
+      if (EPI >= 2 && early) {
+        // y = residual + gate * (acc * s + b), one rounding.  The accumulator
+        // is released as soon as acc * s + b is in registers; the residual
+        // slice is read from shared memory after that.
+        float f[kCols];
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[c0 + j] = fmaf(__uint_as_float(v[j]), sc, bi);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        uint32_t out[kCols / 2];  // bf16x2: tokens (2i, 2i + 1) of this lane's channel
+        if (staged) {
+          const bool ok_r = mbar_wait(smem_u32(&res_bar[ew]), res_it & 1, lim, st);
+          ++res_it;
+          if (!__all_sync(0xffffffffu, ok_r)) break;
+          // Tokens past M read stale shared memory; they are not stored.
+          const uint16_t* sres =
+              reinterpret_cast<const uint16_t*>(smem_gen + C::kStages * C::kStageBytes + ew * C::kResWarpBytes) + lane;
+#pragma unroll
+          for (int i = 0; i < kCols / 2; ++i)
+            out[i] = pack_bf16x2(fmaf(gt, f[2 * i], bf16_bits_to_float(sres[2 * i * 32])),
+                                 fmaf(gt, f[2 * i + 1], bf16_bits_to_float(sres[(2 * i + 1) * 32])));
+        } else {
+#pragma unroll
+          for (int i = 0; i < kCols / 2; ++i) out[i] = pack_bf16x2(fmaf(gt, f[2 * i], 0.f), fmaf(gt, f[2 * i + 1], 0.f));
+        }
+        // Two channels of one token per word (lane l: channels 2(l % 16) and
+        // 2(l % 16) + 1 of token 2i + l / 16) for 4-byte stores.
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
+        const int ld = P.N;
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + (n - lane) + 2 * (lane & 15);
+        const uint32_t sel = (lane >> 4) ? 0x7632u : 0x5410u;
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const uint32_t a = __shfl_sync(0xffffffffu, out[i], 2 * (lane & 15));
+          const uint32_t b = __shfl_sync(0xffffffffu, out[i], 2 * (lane & 15) + 1);
+          const int c = 2 * i + (lane >> 4);
+          if (c < rows) *reinterpret_cast<uint32_t*>(yp + c * ld) = __byte_perm(a, b, sel);
+        }
+      } else if (plain || EPI == 1) {
         uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
         if (plain) {
 #pragma unroll
@@ -567,7 +658,7 @@ static cudaError_t configure_tile() {
   if (dev >= 64) return cudaErrorInvalidDevice;
   if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & (1ull << dev))) {
     e = cudaFuncSetAttribute(tile_kernel<TOK, PAIR, EPI>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg2<TOK, PAIR>::kSmemBytes);
+                             Cfg2<TOK, PAIR, EPI>::kSmemBytes);
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
@@ -577,7 +668,7 @@ static cudaError_t configure_tile() {
 // `ctas_or_pairs` CTAs (one-CTA tiles) or clusters of two (pair tiles).
 template <int TOK, bool PAIR, int EPI>
 static cudaError_t launch_tile(const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
-  using C = Cfg2<TOK, PAIR>;
+  using C = Cfg2<TOK, PAIR, EPI>;
   cudaError_t e = configure_tile<TOK, PAIR, EPI>();
   if (e != cudaSuccess) return e;
   tile_kernel<TOK, PAIR, EPI>()<<<C::kCtas * ctas_or_pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
