@@ -56,9 +56,11 @@ namespace {
 // !PAIR: one CTA per tile (cta_group::1, M = 128 channels, all TOK x rows),
 // used for TOK = 64, where a pair instruction would take as long as at
 // N = 256 but do a quarter of the work.
-// EPI >= 2 (residual or gate epilogues) trades two x stages for a shared
+// EPI == 2 (residual or gate epilogues) trades two x stages for a shared
 // memory slice per epilogue warp where each tile's residual lands while its
 // MMAs run (4 stages keep the tensor pipe as busy as 6 on the plain layer).
+// EPI == 3 keeps 6: its normalising epilogue holds the accumulator long
+// enough that the deeper pipeline pays (4 stages: +18 us on QKV).
 template <int TOK, bool PAIR, int EPI = 0>
 struct Cfg2 {
   static constexpr int kTokPair = TOK;
@@ -71,7 +73,7 @@ struct Cfg2 {
   static constexpr int kCSub = 128 * 16;          // codes of 128 channels x 64 k
   static constexpr int kCBytes = 2 * kCSub;
   static constexpr int kStageBytes = kXBytes + kCBytes;
-  static constexpr bool kResStaged = EPI >= 2;
+  static constexpr bool kResStaged = EPI == 2;
   static constexpr int kStages = kStageBytes > 24 * 1024 ? (kResStaged ? 4 : 6) : 8;
   static constexpr int kASlots = 4;               // decoded-weight slots in TMEM
   static constexpr int kACols = kBK / 2;          // 32-bit TMEM columns per slot (bf16x2)
@@ -205,7 +207,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   __shared__ float norm_part[EPI == 3 ? kHalves * 4 * C::kEpiCols : 1];
   __shared__ float norm_inv[EPI == 3 ? kHalves * C::kEpiCols : 1];
   __shared__ __align__(8) uint64_t norm_bar[EPI == 3 ? 2 * kHalves : 1];
-  // EPI >= 2: per epilogue warp, its residual slice of the tile has landed.
+  // EPI == 2: per epilogue warp, its residual slice of the tile has landed.
   __shared__ __align__(8) uint64_t res_bar[C::kResStaged ? C::kEpiWarps : 1];
   extern __shared__ uint8_t dyn_smem[];
 
@@ -379,18 +381,19 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       bool plain = true;  // the same for the whole problem
       if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate && P.norm_col0 == P.norm_col1;
-      // Residual and gate without an activation ("early"): this warp's
-      // slice of the tile's residual (its 32 channels of kCols tokens, 64
-      // bytes per token) is copied into shared memory while the tile's MMAs
-      // run, and combined before the accumulator is released; after the
-      // release only the stores remain.  (Read from global memory after the
-      // release, the residual's round trips would hold up the next tile.)
+      // Residual, gate and activation ("early", EPI == 2): this warp's slice
+      // of the tile's residual (its 32 channels of kCols tokens, 64 bytes per
+      // token) is copied into shared memory while the tile's MMAs run; after
+      // the release the epilogue reads shared memory only.  (Read from global
+      // memory after the release, the residual's round trips and the
+      // registers they need made the epilogue longer than the next tile's
+      // MMAs.)
       bool early = false, staged = false;
       float gt = 1.f;
       if constexpr (EPI >= 2) {
         const bool normed = EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1;
         const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
-        early = !plain && !normed && P.act == kActNone && (reinterpret_cast<uintptr_t>(res) & 15) == 0;
+        early = C::kResStaged && !plain && !normed && (reinterpret_cast<uintptr_t>(res) & 15) == 0;
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = max(0, min(kCols, P.M - row0));
         if (early) {
@@ -418,10 +421,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         break;
       }
       tc_fence_after();
-      if (EPI >= 2 && early) {
-        // y = residual + gate * (acc * s + b), one rounding.  The accumulator
-        // is released as soon as acc * s + b is in registers; the residual
-        // slice is read from shared memory after that.
+      if (C::kResStaged && early) {
+        // y = residual + gate * act(acc * s + b), one rounding.  The
+        // accumulator is released as soon as acc * s + b is in registers; the
+        // activation and the residual slice (from shared memory) come after.
         float f[kCols];
 #pragma unroll
         for (int c0 = 0; c0 < kCols; c0 += 32) {
@@ -434,6 +437,11 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        if (P.act != kActNone) {
+          const int act = P.act, act_col0 = P.act_col0;
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) f[c] = apply_act(f[c], act, n, act_col0);
+        }
         uint32_t out[kCols / 2];  // bf16x2: tokens (2i, 2i + 1) of this lane's channel
         if (staged) {
           const bool ok_r = mbar_wait(smem_u32(&res_bar[ew]), res_it & 1, lim, st);
