@@ -26,6 +26,15 @@ Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
   first linear applies.  The pages quantise every linear of FLUX's blocks
   (Section 3.1) but do not describe the operations between them; this is
   FLUX.1's MLP activation, written from its definition.
+* ``rms_norm_groups``, ``linear_epilogue(...)`` -- the fused epilogues of
+  FLUX.1's blocks: q/k RMS normalisation per head, the activation, and the
+  gated residual update.
+* ``adaln_modulate(x_bits, scale_bits, shift_bits, eps, tokens_per_row)`` --
+  layer normalisation of each token row (no affine) modulated by a row of
+  the adaLN modulation output: ``(x - mean) / sqrt(var + eps) * (1 + scale)
+  + shift``, what FLUX.1's blocks feed to their first linears.  Like the
+  epilogues, an operation between the quantised linears that the pages do
+  not describe (Section 3.1), written from that model's definition.
 
 bf16 tensors are passed as their raw uint16 bit patterns.
 """
@@ -270,3 +279,30 @@ def linear_epilogue(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=Non
             raise ValueError("residual shape mismatch")
         a = r + a
     return a
+
+
+def adaln_modulate(x_bits: np.ndarray, scale_bits: np.ndarray, shift_bits: np.ndarray, eps: float,
+                   tokens_per_row=None) -> np.ndarray:
+    """Layer normalisation of every token row of x [M, K] (mean and biased
+    variance over K, no affine), then the adaLN modulation with row g =
+    m // tokens_per_row of scale and shift [G, K]:
+        out[m, k] = (x[m, k] - mean_m) / sqrt(var_m + eps) * (1 + scale[g, k]) + shift[g, k],
+    in float64 over the exact bf16 inputs.  tokens_per_row None: every row
+    uses scale[0] and shift[0]."""
+    x = bf16_bits_to_f64(_c(x_bits, np.uint16))
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = x.shape
+    T = M if tokens_per_row is None else int(tokens_per_row)
+    if T < 1:
+        raise ValueError("tokens_per_row must be >= 1")
+    G = max(1, -(-M // T))
+    sc = bf16_bits_to_f64(_c(scale_bits, np.uint16)).reshape(-1, K)
+    sh = bf16_bits_to_f64(_c(shift_bits, np.uint16)).reshape(-1, K)
+    if sc.shape[0] < G or sh.shape[0] < G:
+        raise ValueError("scale and shift need one row per group of tokens_per_row tokens")
+    mean = x.mean(axis=1, keepdims=True)
+    var = ((x - mean) ** 2).mean(axis=1, keepdims=True)
+    v = (x - mean) / np.sqrt(var + eps)
+    g = np.arange(M) // T
+    return v * (1.0 + sc[g]) + sh[g]

@@ -403,3 +403,54 @@ def test_rms_norm_groups_properties_and_torch():
         assert np.allclose(got[:, g0:g0 + 128], ref.numpy(), rtol=1e-12, atol=1e-14)
     with pytest.raises(ValueError):
         oracle.rms_norm_groups(y, 64, 256, 1e-6)
+
+
+def test_adaln_modulate_closed_form_and_torch():
+    """adaLN modulation: a row of alternating +-a has mean 0 and variance a^2,
+    so its normalised values are +-a / sqrt(a^2 + eps) exactly; with scale
+    and shift the closed form (1 + scale) * that + shift (a sign slip, a
+    dropped 1 + or a shift applied before the scale fails it).  With scale =
+    shift = 0 it is torch's layer_norm without affine, in float64."""
+    K = 16
+    a, eps = 0.75, 1e-6
+    row = np.array([a if k % 2 == 0 else -a for k in range(K)])
+    sc = (np.arange(K) - 8) / 16.0  # bf16-exact
+    sh = (3 * np.arange(K) - 20) / 32.0
+    x_bits, sc_bits, sh_bits = to_bf16_bits(row[None, :]), to_bf16_bits(sc), to_bf16_bits(sh)
+    got = oracle.adaln_modulate(x_bits, sc_bits, sh_bits, eps)
+    sc64 = oracle.bf16_bits_to_f64(sc_bits)
+    sh64 = oracle.bf16_bits_to_f64(sh_bits)
+    n = np.where(np.arange(K) % 2 == 0, 1.0, -1.0) * a / np.sqrt(a * a + eps)
+    assert np.allclose(got[0], n * (1.0 + sc64) + sh64, rtol=1e-14, atol=1e-15)
+
+    rng = np.random.default_rng(11)
+    x = torch.from_numpy(rng.normal(0.3, 2.0, size=(5, 384))).to(torch.bfloat16)
+    xb = workloads.bf16_bits(x)
+    zeros = np.zeros(384, np.uint16)
+    got = oracle.adaln_modulate(xb, zeros, zeros, 1e-6)
+    ref = torch.nn.functional.layer_norm(x.double(), (384,), eps=1e-6).numpy()
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_adaln_modulate_invariants_and_row_groups():
+    """With eps = 0 the normalisation ignores a positive scale and an offset
+    of the row; each token row takes modulation row m // tokens_per_row."""
+    rng = np.random.default_rng(12)
+    M, K, T = 6, 256, 4
+    xv = rng.integers(-32, 33, size=(M, K)) / 8.0  # on a grid where 2x + 1 stays exact in bf16
+    x_bits = to_bf16_bits(xv)
+    sc_bits = workloads.bf16_bits((torch.rand(2, K) - 0.5).to(torch.bfloat16))
+    sh_bits = workloads.bf16_bits((torch.rand(2, K) - 0.5).to(torch.bfloat16))
+    base = oracle.adaln_modulate(x_bits, sc_bits, sh_bits, 0.0, T)
+    moved_bits = to_bf16_bits(xv * 2.0 + 1.0)
+    assert np.allclose(oracle.adaln_modulate(moved_bits, sc_bits, sh_bits, 0.0, T), base, rtol=1e-12, atol=1e-12)
+    # rows 0..3 use modulation row 0, rows 4..5 row 1
+    top = oracle.adaln_modulate(x_bits[:T], sc_bits[0], sh_bits[0], 0.0)
+    bot = oracle.adaln_modulate(x_bits[T:], sc_bits[1], sh_bits[1], 0.0)
+    assert np.array_equal(base[:T], top) and np.array_equal(base[T:], bot)
+    # unit variance and zero mean of the normalised rows (scale = shift = 0)
+    zeros = np.zeros(K, np.uint16)
+    v = oracle.adaln_modulate(x_bits, zeros, zeros, 0.0)
+    assert np.allclose(v.mean(axis=1), 0.0, atol=1e-13) and np.allclose(v.var(axis=1), 1.0, rtol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.adaln_modulate(x_bits, sc_bits[:1], sh_bits[:1], 0.0, T)
