@@ -390,8 +390,9 @@ def graph_time(calls, replays, stream):
 
 def side_table(device, peaks, stream):
     """Per-kernel figures for the other rows of the path (not the headline):
-    the adaLN modulation GEMV sweep, the MLP layers, quantise/pack, and bf16
-    cuBLAS on the dequantised weight as context.  Weights rotate over enough
+    the adaLN modulation GEMV sweep, the MLP layers, quantise/pack, the adaLN
+    modulation of normalised activations, and bf16 cuBLAS on the dequantised
+    weight (torch's unfused normalisation for the latter) as context.  Weights rotate over enough
     copies that they do not stay in L2 between launches."""
     import torch
     import torch.nn.functional as F
@@ -443,6 +444,23 @@ def side_table(device, peaks, stream):
     rows["quantize_pack_21504x3072"] = {"us": t * 1e6, "gbs": nbytes / t / 1e9,
                                         "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
     del W, p, s
+    # adaLN modulation of a single block's 4608 token rows (one image), four
+    # x/out pairs rotating (226 MB > L2); torch's unfused layer_norm, multiply
+    # and add as context
+    M, K = 4608, 3072
+    mod = (torch.randn(1, 6 * K, device=device) * 0.1).to(torch.bfloat16)
+    xs_ = [(torch.randn(M, K, device=device)).to(torch.bfloat16) for _ in range(4)]
+    outs_ = [torch.empty_like(xs_[0]) for _ in range(4)]
+    calls = [(lambda x=x, o=o: tern.adaln_modulate(x, mod[:, K:2 * K], mod[:, :K], 1e-6, out=o))
+             for x, o in zip(xs_, outs_)]
+    t = graph_time(calls * 3, 5, stream)
+    nbytes = 2 * 2 * M * K + 2 * 2 * K
+    sc_, sh_ = mod[0, K:2 * K], mod[0, :K]
+    tu = graph_time([(lambda x=x: F.layer_norm(x, (K,), eps=1e-6) * (1 + sc_) + sh_) for x in xs_] * 3, 5, stream)
+    rows["adaln_modulate_4608x3072"] = {"us": t * 1e6, "gbs": nbytes / t / 1e9,
+                                        "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"],
+                                        "torch_unfused_us": tu * 1e6}
+    del xs_, outs_, mod
     rows.update(stack_rows(device, peaks, stream))
     return rows
 

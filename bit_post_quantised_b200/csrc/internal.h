@@ -79,6 +79,13 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N,
                               __nv_bfloat16* out, cudaStream_t stream);
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, unsigned int* status,
                                  cudaStream_t stream);
+// adaLN modulation of layer-normalised token rows (one warp per row, the row
+// in registers): K % 8 == 0, K <= kAdaMaxK, 16-byte aligned rows, scale and
+// shift rows mod_ld elements apart.
+constexpr int kAdaMaxK = 4096;
+cudaError_t launch_adaln_modulate(const __nv_bfloat16* x, int M, int K, const __nv_bfloat16* scale,
+                                  const __nv_bfloat16* shift, int mod_ld, int tokens_per_row, float eps,
+                                  __nv_bfloat16* out, cudaStream_t stream);
 int smem_bytes_for_tok(int tok);
 // Persistent tcgen05 tile kernel: tok-token tiles of 256 channels on CTA pairs
 // (pair, cta_group::2; tok 256 for M > 64) or of 128 channels on single CTAs

@@ -473,6 +473,37 @@ tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float e
   return TERN_OK;
 }
 
+tern_status tern_adaln_modulate(const void* x, int64_t M, int64_t K, const void* scale, const void* shift,
+                                int64_t mod_ld, int64_t tokens_per_row, float eps, void* out,
+                                tern_stream_t stream) {
+  if (M < 0 || K < 0 || mod_ld < 0) return fail(TERN_ERR_INVALID_ARG, "negative size");
+  if (K < 8 || K % 8 != 0 || K > kAdaMaxK || M > int64_t(INT32_MAX) || tokens_per_row < 1 ||
+      tokens_per_row > int64_t(INT32_MAX) || mod_ld < K || mod_ld % 8 != 0 || mod_ld > int64_t(INT32_MAX))
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "adaln_modulate: M=%lld K=%lld mod_ld=%lld tokens_per_row=%lld",
+                (long long)M, (long long)K, (long long)mod_ld, (long long)tokens_per_row);
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(TERN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (M == 0) return TERN_OK;  // no row: the pointers are not used
+  if (!x || !scale || !shift || !out) return fail(TERN_ERR_INVALID_ARG, "null x, scale, shift or out");
+  if (!aligned(x, 16) || !aligned(scale, 16) || !aligned(shift, 16) || !aligned(out, 16))
+    return fail(TERN_ERR_MISALIGNED, "x, scale, shift and out need 16-byte alignment");
+  const size_t xb = size_t(M) * size_t(K) * 2;
+  const int64_t G = (M + tokens_per_row - 1) / tokens_per_row;
+  const size_t mb = (size_t(G - 1) * size_t(mod_ld) + size_t(K)) * 2;
+  if (out != x && overlaps(out, xb, x, xb)) return fail(TERN_ERR_INVALID_ARG, "out overlaps x without being x");
+  if (overlaps(out, xb, scale, mb) || overlaps(out, xb, shift, mb))
+    return fail(TERN_ERR_INVALID_ARG, "out overlaps scale or shift");
+  int dev;
+  DeviceState* ds;
+  tern_status s;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  cudaError_t e = launch_adaln_modulate(static_cast<const __nv_bfloat16*>(x), int(M), int(K),
+                                        static_cast<const __nv_bfloat16*>(scale),
+                                        static_cast<const __nv_bfloat16*>(shift), int(mod_ld), int(tokens_per_row),
+                                        eps, static_cast<__nv_bfloat16*>(out), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "adaln_modulate launch");
+  return TERN_OK;
+}
+
 }  // extern "C"
 
 namespace tern {

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
             "tern_linear_act", "tern_linear_epilogue", "tern_linear_batch", "tern_linear_batch_act",
-            "tern_linear_batch_epilogue",
+            "tern_linear_batch_epilogue", "tern_adaln_modulate",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
                                                  vp]
         L.tern_linear_batch_epilogue.restype = st
         L.tern_linear_batch.restype = st
+        L.tern_adaln_modulate.argtypes = [vp, i64, i64, vp, vp, i64, i64, ctypes.c_float, vp, vp]
+        L.tern_adaln_modulate.restype = st
         L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
         L.tern_dequantize.restype = st
         L.tern_get_device_status.argtypes = [vp]
@@ -135,6 +137,24 @@ def quantize_pack(W: torch.Tensor, eps: float = 1e-5, packed: Optional[torch.Ten
     _check(lib().tern_quantize_pack(_ptr(W), N, K, float(eps), _ptr(packed), _ptr(scales),
                                     _stream(stream)))
     return packed, scales
+
+
+def adaln_modulate(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, eps: float = 1e-6,
+                   tokens_per_row: Optional[int] = None, mod_ld: Optional[int] = None,
+                   out: Optional[torch.Tensor] = None, stream=None):
+    """tern_adaln_modulate: out = LayerNorm(x) * (1 + scale[g]) + shift[g] per
+    token row, g = row // tokens_per_row (default: every row uses row 0).
+    scale and shift are bf16 with rows mod_ld elements apart (default: their
+    own row stride), e.g. slices of the modulation output; out may be x."""
+    M, K = x.shape
+    T = M if tokens_per_row is None else int(tokens_per_row)
+    if mod_ld is None:
+        mod_ld = scale.stride(0) if scale.dim() == 2 else K
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().tern_adaln_modulate(_ptr(x), M, K, _ptr(scale), _ptr(shift), int(mod_ld), max(T, 1), float(eps),
+                                     _ptr(out), _stream(stream)))
+    return out
 
 
 def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,

@@ -242,6 +242,32 @@ TERN_API tern_status tern_linear_batch_act(const tern_linear_act_args* args, int
 TERN_API tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,
                             void* W_bf16_out, tern_stream_t stream);
 
+/*
+ * adaLN modulation of layer-normalised activations, one pass.  FLUX.1's
+ * blocks feed their first linears (QKV, MLP up; the fused projection of a
+ * single block) with their token rows layer-normalised without affine and
+ * modulated by a shift and a scale row of the block's adaLN modulation
+ * output.  The pages quantise those linears (page "1.58-bit FLUX", Section
+ * 3.1) and keep activations in 16 bits (Section 4) but do not describe this
+ * step; it is an interface choice of this library.  Per token row m, with
+ * g = m / tokens_per_row:
+ *     out[m,k] = (x[m,k] - mean_m) / sqrt(var_m + eps) * (1 + scale[g,k]) + shift[g,k],
+ * mean_m and the biased variance var_m over k in fp32, then one rounding to bf16.
+ *   x, out          [M, K] bf16, row-major, 16-byte aligned.  out may be x
+ *                   itself (in place); any other overlap is TERN_ERR_INVALID_ARG.
+ *   scale, shift    ceil(M / tokens_per_row) rows of K bf16, row g at
+ *                   scale + g * mod_ld (mod_ld >= K elements; e.g. slices of
+ *                   the [B, 6 * hidden] modulation output with mod_ld =
+ *                   6 * hidden), 16-byte aligned, mod_ld % 8 == 0, not
+ *                   overlapping out.
+ *   eps             >= 0 and finite (FLUX.1: 1e-6).
+ *   M >= 0 (0: nothing launched, no pointer used), tokens_per_row >= 1, K % 8 == 0 and
+ *   8 <= K <= 4096, else TERN_ERR_UNSUPPORTED_SHAPE.
+ */
+TERN_API tern_status tern_adaln_modulate(const void* x, int64_t M, int64_t K, const void* scale, const void* shift,
+                                int64_t mod_ld, int64_t tokens_per_row, float eps, void* out,
+                                tern_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: TERN_ERR_TIMEOUT if any kernel's bounded wait ran out since
  * the last call, TERN_OK otherwise (TERN_ERR_CUDA if the sync itself failed). */

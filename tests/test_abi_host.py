@@ -201,3 +201,24 @@ def test_norm_epilogue_rejects_on_host(L):
     assert call(w=F + 0x500001) == MISALIGNED
     assert call(M=16) == SHAPE            # would run on the GEMV
     assert call(N=384, c1=128) == SHAPE   # would run on the fallback kernel
+
+
+def test_adaln_rejects_on_host(L):
+    """tern_adaln_modulate's shape, alignment and overlap checks, before any
+    device work; M = 0 is a successful no-op."""
+    x, sc, sh, out = F, F + 0x100000, F + 0x200000, F + 0x300000
+
+    def call(M=16, K=256, scale=sc, shift=sh, ld=256, T=16, eps=1e-6, o=out, xx=x):
+        return L.tern_adaln_modulate(xx, M, K, scale, shift, ld, T, eps, o, None)
+    assert call(K=100) == SHAPE            # K % 8
+    assert call(K=8192, ld=8192) == SHAPE  # longer than a row in registers
+    assert call(ld=200) == SHAPE           # mod_ld < K
+    assert call(ld=260) == SHAPE           # mod_ld % 8
+    assert call(T=0) == SHAPE
+    assert call(M=-1) == INVALID
+    assert call(eps=-1.0) == INVALID and call(eps=float("inf")) == INVALID
+    assert call(xx=None) == INVALID and call(scale=None) == INVALID
+    assert call(xx=x + 8) == MISALIGNED and call(shift=sh + 2) == MISALIGNED and call(o=out + 4) == MISALIGNED
+    assert call(o=x + 16) == INVALID       # partial overlap with x
+    assert call(o=sc - 16 * 256 * 2 + 16) == INVALID  # out runs into scale
+    assert call(M=0) == 0
