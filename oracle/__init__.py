@@ -163,22 +163,31 @@ def unpack_canonical(P: np.ndarray, N: int, K: int):
     return T, int(bad)
 
 
+def tiled_bytes(N: int, K: int) -> int:
+    """Size of the tiled layout: N rounded up to whole 128-channel slabs."""
+    return -(-N // 128) * 128 * K // 4
+
+
 def pack_tiled(T: np.ndarray) -> np.ndarray:
+    """Tiled device layout of T [N, K] (N % 16 == 0, K % 64 == 0); channels
+    past N up to the next multiple of 128 hold zero codes."""
     T = _c(T, np.int8)
     N, K = T.shape
-    P = np.empty(N * K // 4, np.uint8)
+    P = np.empty(tiled_bytes(N, K), np.uint8)
     if _load().oracle_pack_tiled(_p(T), N, K, _p(P)) != 0:
-        raise ValueError("tiled layout needs N % 128 == 0 and K % 64 == 0")
+        raise ValueError("tiled layout needs N % 16 == 0 and K % 64 == 0")
     return P
 
 
 def unpack_tiled(P: np.ndarray, N: int, K: int):
     """Returns (T, number of invalid codes)."""
     P = _c(P, np.uint8)
+    if P.size < tiled_bytes(N, K):
+        raise ValueError("packed buffer smaller than the tiled layout")
     T = np.empty((N, K), np.int8)
     bad = _load().oracle_unpack_tiled(_p(P), N, K, _p(T))
     if bad < 0:
-        raise ValueError("tiled layout needs N % 128 == 0 and K % 64 == 0")
+        raise ValueError("tiled layout needs N % 16 == 0 and K % 64 == 0")
     return T, int(bad)
 
 

@@ -146,10 +146,17 @@ static void tiled_position(int64_t n, int64_t k, int64_t K, int64_t *byte, int *
     *shift = bit % 8;
 }
 
-/* Returns -1 if the shape does not tile (N%128 or K%64 nonzero), else 0. */
+/* Bytes of the tiled layout: whole slabs of 128 channels, so N rounds up to
+ * a multiple of 128 and the rows past N hold zero codes. */
+int64_t oracle_tiled_bytes(int64_t N, int64_t K) {
+    return ((N + 127) / 128) * 128 * K / 4;
+}
+
+/* Returns -1 if the shape does not tile (N%16 or K%64 nonzero), else 0.  P
+ * holds oracle_tiled_bytes(N, K) bytes; the padding rows are written as 0. */
 int oracle_pack_tiled(const int8_t *T, int64_t N, int64_t K, uint8_t *P) {
-    if (N % 128 != 0 || K % 64 != 0) return -1;
-    memset(P, 0, (size_t)(N * K / 4));
+    if (N <= 0 || N % 16 != 0 || K % 64 != 0) return -1;
+    memset(P, 0, (size_t)oracle_tiled_bytes(N, K));
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {
             int64_t byte;
@@ -162,7 +169,7 @@ int oracle_pack_tiled(const int8_t *T, int64_t N, int64_t K, uint8_t *P) {
 
 /* Returns -1 for a shape that does not tile, else the number of invalid codes. */
 int oracle_unpack_tiled(const uint8_t *P, int64_t N, int64_t K, int8_t *T) {
-    if (N % 128 != 0 || K % 64 != 0) return -1;
+    if (N <= 0 || N % 16 != 0 || K % 64 != 0) return -1;
     int bad = 0;
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) {

@@ -210,6 +210,37 @@ def test_tiled_layout_hand_positions(pos):
     np.testing.assert_array_equal(U, T)
 
 
+def test_tiled_layout_ragged_n_pads_whole_slabs():
+    """N % 128 != 0 (N % 16 == 0): the layout keeps whole 128-channel slabs;
+    an element of the first slab keeps its hand-computed position (which
+    does not depend on N), the channels past N are zero bytes, and unpack
+    inverts pack."""
+    used = 0
+    for N0, K, n, k, value, byte, shift in read_positions():
+        if n >= 48:
+            continue
+        T = np.zeros((48, K), np.int8)
+        T[n, k] = value
+        P = oracle.pack_tiled(T)
+        assert P.size == 128 * K // 4
+        assert list(np.nonzero(P)[0]) == [byte] and P[byte] == ((value & 3) << shift)
+        used += 1
+    assert used >= 2
+    rng = np.random.default_rng(4)
+    N, K = 208, 128  # two slabs, the second 80 channels deep
+    T = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    P = oracle.pack_tiled(T)
+    assert P.size == 256 * K // 4
+    for kc in range(K // 64):  # slab 1, chunk kc: rows 80..127 are padding
+        g0 = (1 * (K // 64) + kc) * 2048
+        assert not P[g0 + 80 * 16:g0 + 128 * 16].any()
+    U, bad = oracle.unpack_tiled(P, N, K)
+    assert bad == 0
+    np.testing.assert_array_equal(U, T)
+    with pytest.raises(ValueError):
+        oracle.pack_tiled(np.zeros((40, 64), np.int8))
+
+
 def test_tiled_is_a_permutation_of_canonical():
     rng = np.random.default_rng(1)
     N, K = 256, 192
