@@ -16,7 +16,9 @@
 // k = 8L..8L+7 builds half of the 32-bit word for 16 consecutive k, its
 // neighbour lane the other half.  Rows of up to 4096 values stay in
 // registers between the two steps; longer rows are read twice (the second
-// time from L2).
+// time from L2).  When N is not a multiple of 128 a second small kernel
+// completes the last slab with zero-code rows (no scale), which the linear
+// kernels never store.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -49,6 +51,19 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w, uint32_t thr_pair) {
   const uint32_t nz = (~((thr_pair | 0x80008000u) - mag) >> 15) & 0x00010001u;
   const uint32_t neg = (w >> 15) & 0x00010001u;
   return nz | ((nz & neg) << 1);
+}
+
+// The padding rows n = N .. Np - 1 of the last 128-channel slab (N % 128
+// != 0): their code words are zero and they have no scale.  One thread per
+// 32-bit word (word w of a row holds k = 16w .. 16w + 15).
+__global__ void zero_pad_rows_kernel(uint8_t* __restrict__ packed, int N, int K) {
+  const int words = K >> 4;
+  const int pad_rows = ((N + 127) & ~127) - N;
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)pad_rows * words) return;
+  const int n = N + int(i / words), w = int(i % words);
+  uint8_t* slab = packed + size_t(n >> 7) * size_t(K >> 6) * 2048 + size_t(n & 127) * 16;
+  *reinterpret_cast<uint32_t*>(slab + size_t(w >> 2) * 2048 + (w & 3) * 4) = 0u;
 }
 
 // Same computation with the row held in registers, so W is read from HBM
@@ -212,6 +227,10 @@ cudaError_t launch_quantize_pack(const __nv_bfloat16* W, int N, int K, float eps
     quantize_pack_regs_kernel<16><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
   else
     quantize_pack_long_kernel<<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+  if (N % 128 != 0) {
+    const long long n_words = (long long)(((N + 127) & ~127) - N) * (K >> 4);
+    zero_pad_rows_kernel<<<unsigned((n_words + 255) / 256), 256, 0, stream>>>(packed, N, K);
+  }
   return cudaGetLastError();
 }
 

@@ -191,10 +191,15 @@ constexpr int64_t kMaxN = int64_t(1) << 20;
 constexpr int64_t kMaxK = int64_t(1) << 20;
 constexpr int64_t kMaxM = int64_t(1) << 26;
 
+// 128-channel slabs of the tiled layout: N rounds up, the padding channels
+// hold zero codes and are never stored.
+int64_t n_slabs(int64_t N) { return (N + 127) / 128; }
+size_t packed_size(int64_t N, int64_t K) { return size_t(n_slabs(N)) * 128 * size_t(K) / 4; }
+
 tern_status check_nk(int64_t N, int64_t K) {
   if (N < 0 || K < 0) return fail(TERN_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
-  if (N == 0 || K == 0 || N % 128 != 0 || K % 64 != 0)
-    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "need N %% 128 == 0 and K %% 64 == 0, got N=%lld K=%lld",
+  if (N == 0 || K == 0 || N % 16 != 0 || K % 64 != 0)
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "need N %% 16 == 0 and K %% 64 == 0, got N=%lld K=%lld",
                 (long long)N, (long long)K);
   if (N > kMaxN || K > kMaxK)
     return fail(TERN_ERR_UNSUPPORTED_SHAPE, "N or K above 2^20 (N=%lld K=%lld)", (long long)N, (long long)K);
@@ -213,7 +218,7 @@ tern_status check_linear(const tern_linear_args& a) {
     return fail(TERN_ERR_MISALIGNED, "x, packed and y need 16-byte, scales 4-byte, bias 2-byte alignment");
   const size_t ybytes = size_t(a.M) * size_t(a.N) * 2;
   if (overlaps(a.y, ybytes, a.x, size_t(a.M) * size_t(a.K) * 2) ||
-      overlaps(a.y, ybytes, a.packed, size_t(a.N) * size_t(a.K) / 4) ||
+      overlaps(a.y, ybytes, a.packed, packed_size(a.N, a.K)) ||
       overlaps(a.y, ybytes, a.scales, size_t(a.N) * 4) ||
       overlaps(a.y, ybytes, a.bias, a.bias ? size_t(a.N) * 2 : 0))
     return fail(TERN_ERR_INVALID_ARG, "y overlaps an input");
@@ -298,7 +303,7 @@ tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, 
   p->M = int(a.M);
   p->N = int(a.N);
   p->K = int(a.K);
-  p->n_tiles = int(a.N / 128);
+  p->n_tiles = int(n_slabs(a.N));
   p->m_tiles = int((a.M + tok - 1) / tok);
   const int kc_total = int(a.K / 64);
   int splits = std::max(1, std::min(splits_wanted, kc_total));
@@ -396,11 +401,11 @@ tern_status launch_gemv_group(const tern_linear_args* args, const tern_epilogue*
       p->M = int(a.M);
       p->N = int(a.N);
       p->K = int(a.K);
-      p->n_tiles = int(a.N / 128);
+      p->n_tiles = int(n_slabs(a.N));
       p->m_tiles = 1;
       set_epilogue(p, epis, idx[g]);
       p->unit_begin = int(slabs);
-      slabs += a.N / 128;
+      slabs += n_slabs(a.N);
       min_chunks = std::min<int64_t>(min_chunks, a.K / 64);
     }
     if (slabs > 65535) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "more than 65535 slabs of 128 channels in one launch");
@@ -433,7 +438,7 @@ int ctas_per_sm(int tok) {
 // of 64 k per split, at most 16.
 int fallback_splits(int64_t M, int64_t N, int64_t K, int tok, const DeviceState* ds) {
   if (tok > 64) return 1;
-  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  const int64_t tiles = n_slabs(N) * ((M + tok - 1) / tok);
   const int64_t target = int64_t(ds->sms) * ctas_per_sm(tok);
   int splits = 1;
   if (tiles < target) splits = int(std::min<int64_t>(target / tiles, std::max<int64_t>(1, K / 64 / 4)));
@@ -448,8 +453,8 @@ using namespace tern;
 extern "C" {
 
 size_t tern_packed_bytes(int64_t N, int64_t K) {
-  if (N <= 0 || K <= 0 || N % 128 != 0 || K % 64 != 0 || N > kMaxN || K > kMaxK) return 0;
-  return size_t(N) * size_t(K) / 4;
+  if (N <= 0 || K <= 0 || N % 16 != 0 || K % 64 != 0 || N > kMaxN || K > kMaxK) return 0;
+  return packed_size(N, K);
 }
 
 tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float eps, void* packed,
@@ -460,7 +465,7 @@ tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K, float e
   if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(TERN_ERR_INVALID_ARG, "eps must be finite and >= 0");
   if (!aligned(W_bf16, 16) || !aligned(packed, 16) || !aligned(scales, 4))
     return fail(TERN_ERR_MISALIGNED, "W and packed need 16-byte, scales 4-byte alignment");
-  const size_t wb = size_t(N) * size_t(K) * 2, pb = size_t(N) * size_t(K) / 4, sb = size_t(N) * 4;
+  const size_t wb = size_t(N) * size_t(K) * 2, pb = packed_size(N, K), sb = size_t(N) * 4;
   if (overlaps(packed, pb, W_bf16, wb) || overlaps(scales, sb, W_bf16, wb) || overlaps(packed, pb, scales, sb))
     return fail(TERN_ERR_INVALID_ARG, "outputs overlap each other or W");
   int dev;
@@ -536,7 +541,7 @@ tern_status linear_impl(const tern_linear_args& a, const tern_epilogue& epi, ter
   }
   const int tok = pick_tok(M);
   const int splits = fallback_splits(M, N, K, tok, ds);
-  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  const int64_t tiles = n_slabs(N) * ((M + tok - 1) / tok);
   static Batch batch;  // built under the lock below; ~4 KiB, copied into the launch
   static std::mutex batch_mu;
   std::lock_guard<std::mutex> lock(batch_mu);
@@ -679,7 +684,7 @@ tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, 
   if (!packed || !scales || !W_bf16_out) return fail(TERN_ERR_INVALID_ARG, "null pointer");
   if (!aligned(packed, 16) || !aligned(W_bf16_out, 16) || !aligned(scales, 4))
     return fail(TERN_ERR_MISALIGNED, "packed and output need 16-byte, scales 4-byte alignment");
-  if (overlaps(W_bf16_out, size_t(N) * size_t(K) * 2, packed, size_t(N) * size_t(K) / 4) ||
+  if (overlaps(W_bf16_out, size_t(N) * size_t(K) * 2, packed, packed_size(N, K)) ||
       overlaps(W_bf16_out, size_t(N) * size_t(K) * 2, scales, size_t(N) * 4))
     return fail(TERN_ERR_INVALID_ARG, "output overlaps an input");
   int dev;
@@ -814,7 +819,7 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
   // Same tile and split choice as tern_linear, so the two give identical y.
   const int tok = pick_tok(M);
   const int splits = fallback_splits(M, N, K, tok, ds);
-  const int64_t tiles = (N / 128) * ((M + tok - 1) / tok);
+  const int64_t tiles = n_slabs(N) * ((M + tok - 1) / tok);
   std::memset(static_cast<void*>(&batch), 0, sizeof batch);
   int64_t ctas = 0;
   if ((s = fill_problem(a, tok, splits, &batch.p[0], &ctas)) != TERN_OK) return s;

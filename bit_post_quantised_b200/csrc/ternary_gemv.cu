@@ -224,11 +224,14 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) d[nb][e] = 0.f;
     const int n_out = slab * 128 + grp * 16 + g;
+    // N % 16 == 0: a 16-channel group is wholly inside N or wholly padding
+    // (zero codes; its sums are computed like the others and not stored).
+    const bool live = slab * 128 + grp * 16 < P.N;
     if (warp < C::kWarps) {
       // Scale and bias of this lane's two output channels, loaded now and used
       // after the stream (only rank 0 stores).
       float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f, g0 = 1.f, g1 = 1.f;
-      if (rank == 0) {
+      if (rank == 0 && live) {
         s0 = 0.5f * P.scales[n_out];  // codes expand to 2t
         s1 = 0.5f * P.scales[n_out + 8];
         const uint16_t* bias = P.bias;
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int t = 8 * nb + 2 * c + (e & 1);
             const int nn = n_out + (e >> 1) * 8;
-            rv[nb][e] = (P.residual && t < P.M) ? bf16_bits_to_float(P.residual[size_t(t) * P.N + nn]) : 0.f;
+            rv[nb][e] = (P.residual && live && t < P.M) ? bf16_bits_to_float(P.residual[size_t(t) * P.N + nn]) : 0.f;
           }
 #pragma unroll
         for (int nb = 0; nb < NT; ++nb)
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int t = 8 * nb + 2 * c + (e & 1);
             const int nn = n_out + (e >> 1) * 8;
-            if (t < P.M) {
+            if (live && t < P.M) {
               const float v = fmaf(d[nb][e], e >> 1 ? s1 : s0, e >> 1 ? b1 : b0);
               const float a = apply_act(v, P.act, nn, P.act_col0);
               P.y[size_t(t) * P.N + nn] = __float2bfloat16_rn(fmaf(e >> 1 ? g1 : g0, a, rv[nb][e]));

@@ -179,11 +179,12 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
     const int col_end = min(TOK, col_begin + kColsPerHalf);
     const int n = n_tile * 128 + r;
     const int M = P.M, N = P.N;
+    const bool live = n < N;  // channels past N (the last slab's zero-code rows) are not stored
     const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
     if (P.splits == 1) {
-      const float sc = P.scales[n];
-      const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
-      const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
+      const float sc = live ? P.scales[n] : 0.f;
+      const float gt = P.gate && live ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
+      const float bi = P.bias && live ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
       for (int c0 = col_begin; c0 < col_end; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem + lane_off + c0, v);
@@ -191,11 +192,11 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
         float rv[16];  // residual loads of the group first (it may be y itself)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          rv[j] = (res && row0 + c0 + j < M) ? bf16_bits_to_float(res[size_t(row0 + c0 + j) * N + n]) : 0.f;
+          rv[j] = (res && live && row0 + c0 + j < M) ? bf16_bits_to_float(res[size_t(row0 + c0 + j) * N + n]) : 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = row0 + c0 + j;
-          if (m < M)
+          if (live && m < M)
             P.y[size_t(m) * N + n] = __float2bfloat16_rn(
                 fmaf(gt, apply_act(fmaf(__uint_as_float(v[j]), sc, bi), P.act, n, P.act_col0), rv[j]));
         }
@@ -218,18 +219,20 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
       named_barrier_sync(1, kDecThreads);
       if (last_sh) {
         __threadfence();
-        const float sc = P.scales[n];
-        const float bi =
-            P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
-        const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
-        for (int c = col_begin; c < col_end; ++c) {
-          const int m = row0 + c;
-          if (m >= M) break;
-          float acc = 0.f;
-          for (int sp = 0; sp < P.splits; ++sp)
-            acc += __ldcg(P.ws + ((size_t(sp) * tiles + tile) * TOK + c) * 128 + r);
-          P.y[size_t(m) * N + n] = __float2bfloat16_rn(
-              epilogue_value(fmaf(acc, sc, bi), P.act, n, P.act_col0, res, size_t(m) * N + n, gt));
+        if (live) {
+          const float sc = P.scales[n];
+          const float bi =
+              P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
+          const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
+          for (int c = col_begin; c < col_end; ++c) {
+            const int m = row0 + c;
+            if (m >= M) break;
+            float acc = 0.f;
+            for (int sp = 0; sp < P.splits; ++sp)
+              acc += __ldcg(P.ws + ((size_t(sp) * tiles + tile) * TOK + c) * 128 + r);
+            P.y[size_t(m) * N + n] = __float2bfloat16_rn(
+                epilogue_value(fmaf(acc, sc, bi), P.act, n, P.act_col0, res, size_t(m) * N + n, gt));
+          }
         }
         if (dw == 0 && lane == 0) P.counters[tile] = 0;  // ready for the next launch
       }

@@ -22,12 +22,14 @@
  *     default stream).  A host-detectable error returns at once with nothing
  *     launched.  Errors found on the device (a bounded wait that ran out) are
  *     reported later by tern_get_device_status().
- *   - Shapes: N % 128 == 0, K % 64 == 0, N, K >= 1; M >= 0 (M == 0 is a
+ *   - Shapes: N % 16 == 0, K % 64 == 0, N, K >= 1; M >= 0 (M == 0 is a
  *     no-op, and x and y may then be NULL).  Pointers to bf16/packed data must
  *     be 16-byte aligned, `scales` 4-byte aligned.  Outputs must not overlap
  *     inputs.
  *
- * Packed weight layout ("tile-interleaved", N*K/4 bytes, four codes per byte):
+ * Packed weight layout ("tile-interleaved", Np*K/4 bytes with Np = N rounded
+ * up to a multiple of 128, four codes per byte; the Np - N padding channels
+ * hold zero codes and are never stored):
  *   a code is the 2-bit two's complement integer (+1 -> 01, 0 -> 00,
  *   -1 -> 11; 10 never occurs).  Codes are grouped in 16-byte groups, one per
  *   (row n, 64-wide chunk c = k/64), the group at byte offset
@@ -61,15 +63,16 @@ typedef struct CUstream_st* tern_stream_t;
 typedef enum {
   TERN_OK = 0,
   TERN_ERR_INVALID_ARG = -1,      /* null pointer, negative size, overlap, bad eps */
-  TERN_ERR_UNSUPPORTED_SHAPE = -2, /* N % 128, K % 64, or a size beyond the limits */
+  TERN_ERR_UNSUPPORTED_SHAPE = -2, /* N % 16, K % 64, or a size beyond the limits */
   TERN_ERR_MISALIGNED = -3,       /* a pointer breaks the alignment rule above */
   TERN_ERR_CUDA = -4,             /* a CUDA runtime call or launch failed */
   TERN_ERR_TIMEOUT = -5,          /* a bounded device wait ran out (device status) */
   TERN_ERR_NO_DEVICE = -6         /* the current device is not an sm_100 GPU */
 } tern_status;
 
-/* Bytes of the packed codes of an N x K ternary matrix: N*K/4.  Returns 0 for
- * a shape the layout does not support (N % 128, K % 64, or non-positive). */
+/* Bytes of the packed codes of an N x K ternary matrix: Np*K/4, Np = N rounded
+ * up to a multiple of 128 (N*K/4 when N % 128 == 0).  Returns 0 for a shape
+ * the layout does not support (N % 16, K % 64, or non-positive). */
 TERN_API size_t tern_packed_bytes(int64_t N, int64_t K);
 
 /*
@@ -77,7 +80,7 @@ TERN_API size_t tern_packed_bytes(int64_t N, int64_t K);
  * BitNet b1.58 absmean rule it points to).
  *   W_bf16  [N, K] bf16, read only.
  *   eps     >= 0 and finite, added to the mean magnitude: s_n = mean|W_n| + eps.
- *   packed  [N*K/4] bytes, written in the tile-interleaved layout above.
+ *   packed  [tern_packed_bytes(N, K)] bytes, written in the tile-interleaved layout above.
  *   scales  [N] fp32, written: s_n (the dequantised weight is T[n,k] * s_n).
  * The mean is accumulated at better than fp32 precision and rounded once to
  * fp32; a code is +-1 exactly when |W[n,k]| > s_n / 2 (fp32 s_n), else 0,
@@ -91,7 +94,7 @@ TERN_API tern_status tern_quantize_pack(const void* W_bf16, int64_t N, int64_t K
  * Ternary linear layer y = (x . T^T) * s + b (page "1.58-bit FLUX",
  * Sections 1 and 4).
  *   x_bf16  [M, K] bf16 activations.
- *   packed  [N*K/4] codes from tern_quantize_pack (tile-interleaved layout).
+ *   packed  [tern_packed_bytes(N, K)] codes from tern_quantize_pack (tile-interleaved layout).
  *   scales  [N] fp32 per-output-channel scales.
  *   bias    [N] bf16, or NULL for no bias.
  *   y_bf16  [M, N] bf16 output, overwritten (round to nearest even).
@@ -164,7 +167,7 @@ TERN_API tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, c
 /* One independent linear problem of a batch (same meaning as tern_linear). */
 typedef struct {
   const void* x;      /* [M, K] bf16 */
-  const void* packed; /* [N*K/4] codes */
+  const void* packed; /* [tern_packed_bytes(N, K)] codes */
   const float* scales; /* [N] fp32 */
   const void* bias;   /* [N] bf16 or NULL */
   void* y;            /* [M, N] bf16 */

@@ -51,7 +51,10 @@ def test_library_exports_every_declared_symbol(L):
 def test_packed_bytes(L):
     assert tern.packed_bytes(9216, 3072) == 9216 * 3072 // 4
     assert tern.packed_bytes(128, 64) == 2048
-    for N, K in [(0, 64), (128, 0), (100, 64), (128, 48), (-128, 64), (1 << 21, 64)]:
+    # N % 16 == 0 but not % 128: whole 128-channel slabs (FLUX.1's 64-channel final projection)
+    assert tern.packed_bytes(64, 3072) == 128 * 3072 // 4
+    assert tern.packed_bytes(208, 128) == 256 * 128 // 4
+    for N, K in [(0, 64), (128, 0), (100, 64), (8, 64), (128, 48), (-128, 64), (1 << 21, 64)]:
         assert tern.packed_bytes(N, K) == 0
 
 
