@@ -575,6 +575,26 @@ tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, 
     }
   }
   if (count == 0) return TERN_OK;
+  // Problems of one launch run concurrently: no problem's y may overlap any
+  // buffer of another problem (its inputs, its residual or its y).
+  for (int i = 0; i < count; ++i) {
+    const tern_linear_args& a = args[i];
+    if (a.M == 0) continue;
+    const size_t ya = size_t(a.M) * size_t(a.N) * 2;
+    for (int j = 0; j < count; ++j) {
+      const tern_linear_args& b = args[j];
+      if (j == i || b.M == 0) continue;
+      const size_t yb = size_t(b.M) * size_t(b.N) * 2;
+      const void* res = epis ? epis[j].residual : nullptr;
+      const void* gate = epis ? epis[j].gate : nullptr;
+      const void* nw = epis ? epis[j].norm_weight : nullptr;
+      if (overlaps(a.y, ya, b.y, yb) || overlaps(a.y, ya, b.x, size_t(b.M) * size_t(b.K) * 2) ||
+          overlaps(a.y, ya, b.packed, packed_size(b.N, b.K)) || overlaps(a.y, ya, b.scales, size_t(b.N) * 4) ||
+          overlaps(a.y, ya, b.bias, b.bias ? size_t(b.N) * 2 : 0) || overlaps(a.y, ya, res, res ? yb : 0) ||
+          overlaps(a.y, ya, gate, gate ? size_t(b.N) * 2 : 0) || overlaps(a.y, ya, nw, nw ? size_t(b.N) * 2 : 0))
+        return fail(TERN_ERR_INVALID_ARG, "problem %d's y overlaps a buffer of problem %d", i, j);
+    }
+  }
   int dev;
   DeviceState* ds;
   tern_status s = current_device(&dev, &ds);

@@ -222,7 +222,9 @@ TERN_API tern_status tern_linear_batch_epilogue(const tern_linear_args* args, co
  * possible: problems with similar M share one grouped launch (M <= 8, M <= 16,
  * then the tcgen05 kernels).  `args` is host memory, read before the call
  * returns.  Every problem is validated before anything is launched; on an
- * error nothing runs.  count == 0 is a no-op.  Batched problems need no
+ * error nothing runs.  count == 0 is a no-op.  Problems may share inputs
+ * (x, codes, scales, bias, gate), but no problem's y may overlap any buffer
+ * of another problem (TERN_ERR_INVALID_ARG): they run concurrently.  Batched problems need no
  * workspace (only the single-call path for 16 < M <= 64 splits K into one).
  */
 TERN_API tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream);

@@ -225,3 +225,23 @@ def test_adaln_rejects_on_host(L):
     assert call(o=x + 16) == INVALID       # partial overlap with x
     assert call(o=sc - 16 * 256 * 2 + 16) == INVALID  # out runs into scale
     assert call(M=0) == 0
+
+
+def test_batch_rejects_cross_problem_overlaps_on_host(L):
+    """Problems of a batch run concurrently: one problem's y may not overlap
+    another problem's x, codes, residual or y (all rejected before any
+    device work)."""
+    M, N, K = 16, 256, 256
+    yb = M * N * 2
+
+    def args(x1=F + 0x400000, y1=F + 0x500000, p1=F + 0x100000):
+        arr = (tern.LinearArgs * 2)()
+        arr[0] = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, M, N, K)
+        arr[1] = tern.LinearArgs(x1, p1, F + 0x200000, None, y1, M, N, K)
+        return arr
+    assert L.tern_linear_batch(args(y1=F + 0x300000 + yb - 64), 2, None) == INVALID  # y1 runs into y0
+    assert L.tern_linear_batch(args(x1=F + 0x300000), 2, None) == INVALID  # x1 is y0
+    assert L.tern_linear_batch(args(p1=F + 0x500000 - 0x100), 2, None) == INVALID  # codes 1 overlap y1 (own check)
+    eps = (tern.Epilogue * 2)()
+    eps[1] = tern.Epilogue(0, 0, F + 0x300000, None)  # problem 1's residual is problem 0's y
+    assert L.tern_linear_batch_epilogue(args(), eps, 2, None) == INVALID
