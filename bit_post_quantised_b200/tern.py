@@ -148,8 +148,12 @@ def adaln_modulate(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, ep
     own row stride), e.g. slices of the modulation output; out may be x."""
     M, K = x.shape
     T = M if tokens_per_row is None else int(tokens_per_row)
+    if scale.stride(-1) != 1 or shift.stride(-1) != 1:
+        raise ValueError("scale and shift rows must be contiguous")
     if mod_ld is None:
         mod_ld = scale.stride(0) if scale.dim() == 2 else K
+        if shift.dim() == 2 and shift.stride(0) != mod_ld:
+            raise ValueError("scale and shift rows must be the same distance apart")
     if out is None:
         out = torch.empty_like(x)
     _check(lib().tern_adaln_modulate(_ptr(x), M, K, _ptr(scale), _ptr(shift), int(mod_ld), max(T, 1), float(eps),
