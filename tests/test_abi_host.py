@@ -14,6 +14,7 @@ import subprocess
 import sys
 
 import pytest
+import torch
 
 from bit_post_quantised_b200 import _build, tern
 
@@ -245,3 +246,15 @@ def test_batch_rejects_cross_problem_overlaps_on_host(L):
     eps = (tern.Epilogue * 2)()
     eps[1] = tern.Epilogue(0, 0, F + 0x300000, None)  # problem 1's residual is problem 0's y
     assert L.tern_linear_batch_epilogue(args(), eps, 2, None) == INVALID
+
+
+def test_adaln_binding_checks_row_layout():
+    """The binding passes scale and shift as rows mod_ld apart: rows that are
+    not contiguous, or scale and shift rows spaced differently, are refused
+    before the library is called."""
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    mod = torch.zeros(2, 6 * 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        tern.adaln_modulate(x, mod[:, 64:128].t().contiguous().t(), mod[:, :64])  # columns strided
+    with pytest.raises(ValueError):
+        tern.adaln_modulate(x, mod[:, 64:128], torch.zeros(2, 64, dtype=torch.bfloat16))  # 384 vs 64 apart
