@@ -35,6 +35,11 @@ Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
   + shift``, what FLUX.1's blocks feed to their first linears.  Like the
   epilogues, an operation between the quantised linears that the pages do
   not describe (Section 3.1), written from that model's definition.
+* ``fp8_e4m3_rne``, ``quantize_act_e4m3``, ``linear_act_e4m3`` -- the
+  activation quantisation the pages name as the missing latency lever
+  (Section 4): x per token row to FP8 E4M3 with an absmax scale, against the
+  same exact ternary weights.  The pages fix no format or granularity; this
+  is one reading, for a kernel that does not exist yet.
 
 bf16 tensors are passed as their raw uint16 bit patterns.
 """
@@ -315,3 +320,49 @@ def adaln_modulate(x_bits: np.ndarray, scale_bits: np.ndarray, shift_bits: np.nd
     v = (x - mean) / np.sqrt(var + eps)
     g = np.arange(M) // T
     return v * (1.0 + sc[g]) + sh[g]
+
+
+E4M3_MAX = 448.0
+
+
+def fp8_e4m3_rne(v) -> np.ndarray:
+    """Nearest FP8 E4M3 value of each float64 (1 sign, 4 exponent bits with
+    bias 7, 3 mantissa bits, subnormals down to 2^-9, no infinities), ties to
+    even, magnitudes above 448 saturated to 448 (the finite-saturating
+    conversion), as float64."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)  # a = m 2^ex, 0.5 <= m < 1, so floor(log2 a) = ex - 1 exactly
+    e = np.maximum(ex - 1, -6)  # below 2^-6 the spacing stays 2^-9
+    q = np.ldexp(1.0, e - 3)  # spacing of the binade: 3 mantissa bits
+    r = np.minimum(np.round(a / q) * q, E4M3_MAX)  # a / q is exact; np.round ties to even
+    return np.copysign(r, v)
+
+
+def quantize_act_e4m3(x_bits: np.ndarray):
+    """Per token row m: a_m = max_k |x[m,k]| / 448 and v = x / a_m, both
+    divisions in fp32 (the precision a kernel would decide in), then
+    xq = E4M3(v).  A zero row gets a_m = 1 and zero codes.  Returns
+    (xq [M, K] as float64 values, a [M] float64)."""
+    x = bf16_bits_to_f64(_c(x_bits, np.uint16)).astype(np.float32)
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    amax = np.max(np.abs(x), axis=1)
+    a = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    v = (x / a[:, None]).astype(np.float32)
+    return fp8_e4m3_rne(v.astype(np.float64)), a.astype(np.float64)
+
+
+def linear_act_e4m3(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None) -> np.ndarray:
+    """y[m,n] = a_m s_n sum_k xq[m,k] T[n,k] + b_n in float64 with the
+    E4M3-quantised activations of ``quantize_act_e4m3``."""
+    xq, a = quantize_act_e4m3(x_bits)
+    T = _c(T, np.int8)
+    s = _c(s, np.float64)
+    if T.shape[1] != xq.shape[1] or s.shape != (T.shape[0],):
+        raise ValueError("shape mismatch")
+    acc = xq @ T.astype(np.float64).T  # exact: multiples of 2^-9 below 2^33
+    y = acc * a[:, None] * s[None, :]
+    if b_bits is not None:
+        y = y + bf16_bits_to_f64(_c(b_bits, np.uint16))[None, :]
+    return y

@@ -485,3 +485,59 @@ def test_adaln_modulate_invariants_and_row_groups():
     assert np.allclose(v.mean(axis=1), 0.0, atol=1e-13) and np.allclose(v.var(axis=1), 1.0, rtol=1e-12)
     with pytest.raises(ValueError):
         oracle.adaln_modulate(x_bits, sc_bits[:1], sh_bits[:1], 0.0, T)
+
+
+def test_fp8_e4m3_rounding_against_torch_and_closed_forms():
+    """E4M3 rounding: torch's float8_e4m3fn conversion (a library routine) on
+    values up to 448 including subnormals and exact ties, the eight
+    mantissas of [1, 2), ties to even, the extremes, and saturation."""
+    rng = np.random.default_rng(13)
+    v = np.concatenate([rng.uniform(-448, 448, 4000), rng.uniform(-0.02, 0.02, 2000),
+                        rng.uniform(-2.0 ** -6, 2.0 ** -6, 1000)])
+    # exact midpoints between neighbours in several binades (ties)
+    for e in (-9, -7, -6, -3, 0, 4, 7):
+        for m in range(8):
+            lo = (8 + m) * 2.0 ** (e - 3) if e >= -6 else m * 2.0 ** -9
+            v = np.append(v, [lo + 2.0 ** (max(e, -6) - 4), -(lo + 2.0 ** (max(e, -6) - 4))])
+    v = v[np.abs(v) <= 448]
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.fp8_e4m3_rne(v.astype(np.float32).astype(np.float64)), ref)
+    assert list(oracle.fp8_e4m3_rne(1 + np.arange(8) / 8.0)) == list(1 + np.arange(8) / 8.0)
+    assert oracle.fp8_e4m3_rne(1.0625) == 1.0 and oracle.fp8_e4m3_rne(1.1875) == 1.25  # ties to even
+    assert oracle.fp8_e4m3_rne(2.0 ** -9) == 2.0 ** -9 and oracle.fp8_e4m3_rne(2.0 ** -10) == 0.0
+    assert oracle.fp8_e4m3_rne(448.0) == 448.0 and oracle.fp8_e4m3_rne(-1000.0) == -448.0
+
+
+def test_act_e4m3_linear_lossless_on_grid_and_bounded_otherwise():
+    """Rows whose values are E4M3 values times a power of two, with the
+    largest magnitude 448 times that power, quantise without loss, so the
+    linear equals the unquantised one exactly; otherwise each activation
+    moves by at most 2^-4 of its magnitude (3 mantissa bits) or one
+    subnormal step, and y by the matching bound.  The absmax element of a
+    row maps to +-448."""
+    rng = np.random.default_rng(14)
+    M, K, N = 5, 128, 64
+    grid = np.concatenate([(8 + np.arange(8)) * 2.0 ** (e - 3) for e in range(-6, 9)])
+    grid = grid[grid <= 448]
+    xq = rng.choice(grid, size=(M, K)) * rng.choice([-1.0, 1.0], size=(M, K))
+    xq[:, 0] = 448.0
+    x = xq * (2.0 ** -6)  # every value and the scale exact in bf16
+    x_bits = to_bf16_bits(x)
+    T = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    s = rng.uniform(0.01, 0.03, N)
+    got = oracle.linear_act_e4m3(x_bits, T, s)
+    assert np.array_equal(got, oracle.linear(x_bits, T, s))
+    q, a = oracle.quantize_act_e4m3(x_bits)
+    assert np.all(q[:, 0] == 448.0) and np.all(a == 2.0 ** -6)
+
+    xr = torch.randn(M, K, generator=torch.Generator().manual_seed(15)).to(torch.bfloat16)
+    xb = workloads.bf16_bits(xr)
+    q, a = oracle.quantize_act_e4m3(xb)
+    x64 = oracle.bf16_bits_to_f64(xb)
+    assert np.all(np.max(np.abs(q), axis=1) == 448.0)
+    err = np.abs(q * a[:, None] - x64)
+    assert np.all(err <= 2.0 ** -4 * np.abs(x64) * (1 + 1e-6) + 2.0 ** -9 * a[:, None])
+    y = oracle.linear_act_e4m3(xb, T, s)
+    y_ref = oracle.linear(xb, T, s)
+    bound = (err @ np.abs(T.astype(np.float64)).T) * s[None, :]
+    assert np.all(np.abs(y - y_ref) <= bound * (1 + 1e-9) + 1e-12)
