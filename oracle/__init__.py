@@ -35,7 +35,8 @@ Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
   + shift``, what FLUX.1's blocks feed to their first linears.  Like the
   epilogues, an operation between the quantised linears that the pages do
   not describe (Section 3.1), written from that model's definition.
-* ``fp8_e4m3_rne``, ``quantize_act_e4m3``, ``linear_act_e4m3`` -- the
+* ``fp8_e4m3_rne``, ``fp8_e4m3_bits``, ``quantize_act_e4m3``,
+  ``linear_act_e4m3`` -- the
   activation quantisation the pages name as the missing latency lever
   (Section 4): x per token row to FP8 E4M3 with an absmax scale, against the
   same exact ternary weights.  The pages fix no format or granularity; this
@@ -366,3 +367,20 @@ def linear_act_e4m3(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=Non
     if b_bits is not None:
         y = y + bf16_bits_to_f64(_c(b_bits, np.uint16))[None, :]
     return y
+
+
+def fp8_e4m3_bits(v) -> np.ndarray:
+    """The E4M3 byte of each value that is already an E4M3 value (as
+    returned by ``fp8_e4m3_rne``): sign bit 7, biased exponent bits 3-6
+    (bias 7; 0 for subnormals), mantissa bits 0-2.  -0 encodes as 0x80."""
+    v = np.asarray(v, dtype=np.float64)
+    if np.any(fp8_e4m3_rne(v) != v):
+        raise ValueError("value not representable in E4M3")
+    a = np.abs(v)
+    _, ex = np.frexp(a)
+    e = ex - 1  # floor(log2 a) for a > 0
+    normal = a >= 2.0 ** -6
+    exp_field = np.where(normal, e + 7, 0)
+    mant = np.where(normal, a / np.ldexp(1.0, e) - 1.0, a / 2.0 ** -6) * 8.0
+    bits = (np.signbit(v).astype(np.int64) << 7) | (exp_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    return bits.astype(np.uint8)

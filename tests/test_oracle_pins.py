@@ -541,3 +541,16 @@ def test_act_e4m3_linear_lossless_on_grid_and_bounded_otherwise():
     y_ref = oracle.linear(xb, T, s)
     bound = (err @ np.abs(T.astype(np.float64)).T) * s[None, :]
     assert np.all(np.abs(y - y_ref) <= bound * (1 + 1e-9) + 1e-12)
+
+
+def test_fp8_e4m3_bytes_against_torch():
+    """E4M3 encoding of every finite E4M3 value (all 254 non-NaN bytes,
+    through torch's float8_e4m3fn), and the codes +1 -> 0x38, -1 -> 0xB8,
+    0 -> 0x00 that ternary weights take in an FP8 MMA."""
+    b = torch.arange(256, dtype=torch.uint8)
+    b = b[(b & 0x7F) != 0x7F]  # the two NaN bytes
+    vals = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.fp8_e4m3_bits(vals), b.numpy())
+    assert list(oracle.fp8_e4m3_bits([1.0, -1.0, 0.0, 448.0, 2.0 ** -9])) == [0x38, 0xB8, 0x00, 0x7E, 0x01]
+    with pytest.raises(ValueError):
+        oracle.fp8_e4m3_bits([1.0625])
