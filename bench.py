@@ -93,8 +93,9 @@ def profiled_traffic(stem: str, workload: str):
 
 class ClockSampler:
     """Samples SM clocks and clock-event (throttle) reasons while the timed
-    region runs: NVML every 2 ms from a thread (reads only), else nvidia-smi
-    every 100 ms."""
+    region runs: NVML every 0.1 ms from a thread (reads only; a timed region
+    of a few milliseconds still gets tens of samples), else nvidia-smi every
+    100 ms."""
 
     # NVML clock-event reason bits
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
@@ -121,7 +122,7 @@ class ClockSampler:
                 break
             self.samples.append((float(sm), float(mx), {k for k, b in self.REASONS.items() if bits & b}))
             self.ready.set()
-            time.sleep(0.002)
+            time.sleep(0.0001)
 
     def __enter__(self):
         try:
@@ -184,7 +185,7 @@ class ClockSampler:
             reasons |= r
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(b for _, b, _ in self.samples),
                 "reasons": sorted(reasons), "samples": len(sm),
-                "source": "nvml 2 ms" if self.thread is not None else "nvidia-smi 100 ms"}
+                "source": "nvml 0.1 ms" if self.thread is not None else "nvidia-smi 100 ms"}
 
 
 # ------------------------------------------------------------ CPU oracle leg
@@ -388,6 +389,27 @@ def graph_time(calls, replays, stream):
     return e0.elapsed_time(e1) * 1e-3 / (replays * len(calls))
 
 
+def cublas_context_us(L, packs, x, b, stream):
+    """Dense bf16 cuBLAS (F.linear) on the dequantised weight T*s of the same
+    shape, as context: the weight rotates over enough copies (> 3x the 126 MB
+    L2) that it is read from HBM, like the ternary codes."""
+    import torch
+    import torch.nn.functional as F
+
+    from bit_post_quantised_b200 import tern
+
+    l2 = 126 * 2 ** 20
+    wbytes = 2 * L.N * L.K
+    copies = max(2, min(len(packs), -(-3 * l2 // wbytes) + 1))
+    Wds = [tern.dequantize(packs[i % len(packs)][0], packs[i % len(packs)][1], L.K, stream=stream)
+           for i in range(copies)]
+    torch.cuda.synchronize()
+    reps = max(2, 24 // copies)
+    t = graph_time([(lambda Wd=Wd: F.linear(x, Wd, b)) for Wd in Wds] * reps, 5, stream)
+    del Wds
+    return t * 1e6
+
+
 def side_table(device, peaks, stream):
     """Per-kernel figures for the other rows of the path (not the headline):
     the adaLN modulation GEMV sweep, the MLP layers, quantise/pack, the adaLN
@@ -402,7 +424,7 @@ def side_table(device, peaks, stream):
     rows = {}
     l2 = 126 * 2 ** 20
     for name in ["mod6_m1", "mod6_m4", "mod6_m16", "mod6_m64", "mod3_m1", "mod3_m4", "mod3_m16",
-                 "mod3_m64", "mlp_up", "mlp_down"]:
+                 "mod3_m64", "qkv", "mlp_up", "mlp_down"]:
         L = workloads.CONFIGS[name]
         x, W, b = (t.to(device) for t in workloads.make_inputs(L))
         copies = max(2, min(24, int(3 * l2 // max(1, L.packed_bytes)) + 1))
@@ -426,12 +448,7 @@ def side_table(device, peaks, stream):
             ta = graph_time(acts * reps, 5, stream)
             entry["gelu_fused_us"] = ta * 1e6
             entry["gelu_separate_pass_us_at_hbm_peak"] = 2 * 2 * L.M * L.N / peaks["hbm_gbs"] / 1e9 * 1e6
-        if name in ("mlp_up", "mlp_down", "mod6_m64"):
-            Wd = tern.dequantize(packs[0][0], packs[0][1], L.K, stream=stream)
-            torch.cuda.synchronize()
-            tc = graph_time([lambda: F.linear(x, Wd, b)] * 10, 5, stream)
-            entry["cublas_bf16_us"] = tc * 1e6
-            del Wd
+        entry["cublas_bf16_us"] = cublas_context_us(L, packs, x, b, stream)
         rows[name] = entry
         del packs
     # quantise/pack of the largest weight
@@ -505,11 +522,10 @@ def stack_rows(device, peaks, stream):
                 bias[L.N] = (torch.randn(L.N, device=device) * 0.01).to(torch.bfloat16)
             p = dict(x=buf(xs, (L.M, L.K), (L.M, L.K)), packed=packs[i][0], scales=packs[i][1], bias=bias[L.N],
                      y=buf(ys, (j, L.M, L.N), (L.M, L.N)))
-            if L.name.endswith(".mlp_up"):
-                p["act"] = tern.ACT_GELU_TANH
-            elif L.name.endswith(".qkv_mlp"):
-                p["act"], p["act_col0"] = tern.ACT_GELU_TANH, 3 * workloads.HIDDEN  # q, k, v, then the MLP
-            elif L.name.endswith((".proj", ".mlp_down", ".proj_out")):
+            e = workloads.block_epilogue(L.name)
+            if e.get("act") == "gelu_tanh":
+                p["act"], p["act_col0"] = tern.ACT_GELU_TANH, e["act_col0"]
+            elif e.get("gated_residual"):
                 # gated update of a residual stream, in place (adaLN-Zero); one
                 # buffer per problem, as the problems of a batch run concurrently
                 stream_buf = buf(ys, ("stream", j, L.M, L.N), (L.M, L.N))

@@ -115,3 +115,34 @@ def bf16_bits(t: torch.Tensor):
     import numpy as np
 
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def block_layers(block: str) -> List[Layer]:
+    """The layers of one block of ``flux_stack()``, e.g. "double0" or "single7"."""
+    return [L for L in flux_stack() if L.name.split(".")[0] == block]
+
+
+def block_epilogue(name: str, qk_norm: bool = False) -> dict:
+    """How one FLUX.1 block uses the output of its linear ``name``.
+
+    The pages quantise every linear of both block types (Section 3.1) and
+    describe nothing between them; this lists what FLUX.1's blocks do there,
+    as plain data (no arithmetic):
+      * act "gelu_tanh" from column act_col0: the MLP's first linear (all of
+        its columns), or the MLP part of a single block's fused projection
+        (after q, k and v: from column 3 * HIDDEN);
+      * gated_residual: the attention and MLP output projections update the
+        residual stream in place, scaled per channel by an adaLN-Zero gate;
+      * norm_cols (only with qk_norm): per-head RMS normalisation of q and k,
+        the first 2 * HIDDEN columns of a QKV projection.
+    """
+    e: dict = {}
+    if name.endswith(".mlp_up"):
+        e["act"], e["act_col0"] = "gelu_tanh", 0
+    elif name.endswith(".qkv_mlp"):
+        e["act"], e["act_col0"] = "gelu_tanh", 3 * HIDDEN
+    elif name.endswith((".proj", ".mlp_down", ".proj_out")):
+        e["gated_residual"] = True
+    if qk_norm and name.endswith((".qkv", ".qkv_mlp")):
+        e["norm_cols"] = (0, 2 * HIDDEN)
+    return e

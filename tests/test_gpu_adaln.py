@@ -79,20 +79,17 @@ def test_adaln_modulate_constant_rows_give_the_shift():
     assert_close(out, oracle.adaln_modulate(bits(x), bits(sc), bits(sh), EPS))
 
 
-def test_adaln_modulate_flux_image_stream_sampled():
+def test_adaln_modulate_flux_image_stream_full():
     """FLUX.1's double-block image stream at 1024x1024 (4096 tokens x 3072),
-    two images' modulation rows; the oracle on 64 sampled rows."""
+    two images' modulation rows; the oracle on every row."""
     M, K, T = 4096, 3072, 2048
     x = rand_bf16((M, K), 0.0, 1.0, seed=21).cuda()
     mod = rand_bf16((2, 6 * K), 0.0, 0.1, seed=22).cuda()
     out = tern.adaln_modulate(x, mod[:, K:2 * K], mod[:, :K], EPS, tokens_per_row=T)
     torch.cuda.synchronize()
     assert tern.device_status() == 0
-    rows = np.sort(np.random.default_rng(23).choice(M, 64, replace=False))
-    rt = torch.from_numpy(rows)
-    g = rt // T
-    ref = oracle.adaln_modulate(bits(x.cpu()[rt]), bits(mod.cpu()[g, K:2 * K]), bits(mod.cpu()[g, :K]), EPS, 1)
-    assert_close(out.cpu()[rt], ref)
+    ref = oracle.adaln_modulate(bits(x.cpu()), bits(mod.cpu()[:, K:2 * K]), bits(mod.cpu()[:, :K]), EPS, T)
+    assert_close(out.cpu(), ref)
 
 
 def test_adaln_modulate_empty_is_a_no_op():
