@@ -11,6 +11,9 @@ namespace tern {
 // Bits of the per-device status word.  Kernels OR bits into it (through the
 // pointer they are given) instead of trapping; the host reads and clears it.
 constexpr unsigned kStatusTimeout = 1u;
+// A kernel found its launch configuration inconsistent with its arguments
+// (a defect of the host code, never of the caller's data); it computed nothing.
+constexpr unsigned kStatusLaunchConfig = 2u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

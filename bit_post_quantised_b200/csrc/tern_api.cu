@@ -740,6 +740,8 @@ tern_status tern_get_device_status(tern_stream_t stream) {
       }
     return fail(TERN_ERR_TIMEOUT, "a device-side wait ran out of time");
   }
+  if (word & kStatusLaunchConfig)
+    return fail(TERN_ERR_LAUNCH_CONFIG, "a kernel found its launch configuration inconsistent and computed nothing");
   return TERN_OK;
 }
 
@@ -768,6 +770,7 @@ const char* tern_status_string(tern_status status) {
     case TERN_ERR_CUDA: return "CUDA error";
     case TERN_ERR_TIMEOUT: return "device wait timed out";
     case TERN_ERR_NO_DEVICE: return "no supported device";
+    case TERN_ERR_LAUNCH_CONFIG: return "inconsistent kernel launch configuration";
   }
   return "unknown status";
 }

@@ -135,8 +135,10 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   const int u0 = blockIdx.y, ustep = gridDim.y, units = batch.total_units;
   // With K split over a cluster the producer only joins the per-unit cluster
   // rendezvous after its whole stream, so each CTA must own a single unit.
+  // (The host never launches otherwise; the test is uniform over the grid,
+  // so every CTA leaves here and the host reads TERN_ERR_LAUNCH_CONFIG.)
   if (splits > 1 && ustep < units) {
-    if (threadIdx.x == 0) atomicOr(st, kStatusTimeout);
+    if (threadIdx.x == 0) atomicOr(st, kStatusLaunchConfig);
     return;
   }
 

@@ -20,7 +20,7 @@ _lib = None
 TERN_OK = 0
 STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPORTED_SHAPE",
                 -3: "TERN_ERR_MISALIGNED", -4: "TERN_ERR_CUDA", -5: "TERN_ERR_TIMEOUT",
-                -6: "TERN_ERR_NO_DEVICE"}
+                -6: "TERN_ERR_NO_DEVICE", -7: "TERN_ERR_LAUNCH_CONFIG"}
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
             "tern_linear_act", "tern_linear_epilogue", "tern_linear_batch", "tern_linear_batch_act",

@@ -67,12 +67,19 @@ typedef enum {
   TERN_ERR_MISALIGNED = -3,       /* a pointer breaks the alignment rule above */
   TERN_ERR_CUDA = -4,             /* a CUDA runtime call or launch failed */
   TERN_ERR_TIMEOUT = -5,          /* a bounded device wait ran out (device status) */
-  TERN_ERR_NO_DEVICE = -6         /* the current device is not an sm_100 GPU */
+  TERN_ERR_NO_DEVICE = -6,        /* the current device is not an sm_100 GPU */
+  TERN_ERR_LAUNCH_CONFIG = -7     /* a kernel found its launch configuration inconsistent
+                                     with its arguments and computed nothing: a defect of
+                                     the library's host code, not of the caller's data
+                                     (device status) */
 } tern_status;
 
 /* Bytes of the packed codes of an N x K ternary matrix: Np*K/4, Np = N rounded
  * up to a multiple of 128 (N*K/4 when N % 128 == 0).  Returns 0 for a shape
- * the layout does not support (N % 16, K % 64, or non-positive). */
+ * the layout does not support (N % 16, K % 64, or non-positive).  The four
+ * 2-bit codes per byte follow page "1.58-bit FLUX", Section 1 (weights
+ * "stored using 2-bit signed integers"); the padding to whole 128-channel
+ * slabs is this library's layout choice, not on the pages. */
 TERN_API size_t tern_packed_bytes(int64_t N, int64_t K);
 
 /*
@@ -219,7 +226,11 @@ TERN_API tern_status tern_linear_batch_epilogue(const tern_linear_args* args, co
 /*
  * Several independent ternary linears (for instance the per-stream adaLN
  * modulation GEMVs and projections of one FLUX block) with as few launches as
- * possible: problems with similar M share one grouped launch (M <= 8, M <= 16,
+ * possible.  Each problem is the layer of page "1.58-bit FLUX", Sections 1
+ * and 3.1 (every linear of both block types is ternary); batching them is not
+ * on the pages -- it is an interface choice of this library, made because a
+ * FLUX forward has 76 small modulation GEMVs whose launches would otherwise
+ * dominate their run time.  Problems with similar M share one grouped launch (M <= 8, M <= 16,
  * then the tcgen05 kernels).  `args` is host memory, read before the call
  * returns.  Every problem is validated before anything is launched; on an
  * error nothing runs.  count == 0 is a no-op.  Problems may share inputs
@@ -275,7 +286,9 @@ TERN_API tern_status tern_adaln_modulate(const void* x, int64_t M, int64_t K, co
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: TERN_ERR_TIMEOUT if any kernel's bounded wait ran out since
- * the last call, TERN_OK otherwise (TERN_ERR_CUDA if the sync itself failed). */
+ * the last call, else TERN_ERR_LAUNCH_CONFIG if a kernel refused an
+ * inconsistent launch configuration, TERN_OK otherwise (TERN_ERR_CUDA if the
+ * sync itself failed). */
 TERN_API tern_status tern_get_device_status(tern_stream_t stream);
 
 /* Wall-time limit of every device-side wait, in nanoseconds (default 1e9).

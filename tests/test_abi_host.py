@@ -62,6 +62,7 @@ def test_packed_bytes(L):
 def test_status_strings(L):
     assert tern.status_string(0) == "ok"
     assert "timed out" in tern.status_string(-5)
+    assert "launch configuration" in tern.status_string(-7)
     assert tern.status_string(123) == "unknown status"
 
 
