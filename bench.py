@@ -451,6 +451,29 @@ def side_table(device, peaks, stream):
         entry["cublas_bf16_us"] = cublas_context_us(L, packs, x, b, stream)
         rows[name] = entry
         del packs
+    # FP8 (E4M3) activations on the QKV shape: the per-token quantisation of x
+    # and the kind::f8f6f4 layer, against the FP8 tensor peak (the measured
+    # bf16 burst x 2, the nominal dense ratio)
+    L = workloads.CONFIGS["qkv"]
+    x, W, b = (t.to(device) for t in workloads.make_inputs(L))
+    packs = [tern.quantize_pack(W, workloads.EPS, stream=stream) for _ in range(24)]
+    xq, a = tern.quantize_act_e4m3(x, stream=stream)
+    y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=device)
+    t_lin = graph_time([(lambda p=p, s=s: tern.linear_e4m3(xq, a, p, s, b, out=y, stream=stream))
+                        for p, s in packs] * 2, 5, stream)
+    xs4 = [(torch.randn(L.M, L.K, device=device)).to(torch.bfloat16) for _ in range(6)]  # 151 MB > L2
+    t_q = graph_time([(lambda xx=xx: tern.quantize_act_e4m3(xx, xq=xq, a=a, stream=stream)) for xx in xs4] * 4, 5,
+                     stream)
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    qbytes = 2 * L.M * L.K + L.M * L.K + 4 * L.M
+    rows["qkv_fp8_activations"] = {
+        "M": L.M, "N": L.N, "K": L.K, "linear_us": t_lin * 1e6, "tflops": L.flop / t_lin / 1e12,
+        "fp8_peak_tflops": fp8_peak, "frac_of_fp8_peak": L.flop / t_lin / 1e12 / fp8_peak,
+        "peak_source": "measured bf16 burst x 2 (nominal dense FP8/BF16 ratio)",
+        "quantize_act_us": t_q * 1e6, "quantize_act_gbs": qbytes / t_q / 1e9,
+        "quantize_act_hbm_frac": qbytes / t_q / 1e9 / peaks["hbm_gbs"],
+        "step_us": (t_lin + t_q) * 1e6, "step_tflops": L.flop / (t_lin + t_q) / 1e12}
+    del packs, xs4, xq, a, y
     # quantise/pack of the largest weight
     N, K = 21504, 3072
     W = (torch.randn(N, K, device=device) * 0.02).to(torch.bfloat16)

@@ -104,5 +104,13 @@ int max_active_clusters_2sm();
 cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream);
 int max_active_clusters_2sm();
 int smem_bytes_2sm();
+// FP8 (E4M3) activations: per-token absmax quantisation of x (one warp per
+// row, k interleaved inside 16-element groups), and the CTA-pair tile kernel
+// with kind::f8f6f4 MMAs (one problem: N % 256 == 0, tmap_x = the 2-D E4M3 map
+// {K, M} with box {128, 128}, ws = the per-token scales).
+cudaError_t launch_quantize_act_e4m3(const __nv_bfloat16* x, int M, int K, uint8_t* xq, float* a,
+                                     cudaStream_t stream);
+cudaError_t launch_ternary_fp8(const Batch& batch, int pairs, cudaStream_t stream);
+
 
 }  // namespace tern

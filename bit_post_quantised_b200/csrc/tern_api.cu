@@ -141,6 +141,22 @@ tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_
   return TERN_OK;
 }
 
+// E4M3 x [M, K] bytes row-major: box = 128 k x 128 rows, 128-byte swizzle;
+// columns past K and rows past M read as zero.
+tern_status make_xq_map(CUtensorMap* map, const void* xq, int64_t M, int64_t K) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+  const cuuint64_t strides[1] = {cuuint64_t(K)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(xq), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled (E4M3 x) failed (%d)", int(r));
+  return TERN_OK;
+}
+
 // ------------------------------------------------------------ workspace
 struct Workspace {
   float* ws = nullptr;
@@ -714,6 +730,81 @@ tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, 
                                     static_cast<__nv_bfloat16*>(W_bf16_out),
                                     reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return TERN_OK;
+}
+
+tern_status tern_quantize_act_e4m3(const void* x_bf16, int64_t M, int64_t K, void* xq, float* a,
+                                   tern_stream_t stream) {
+  if (M < 0 || K < 0) return fail(TERN_ERR_INVALID_ARG, "negative size M=%lld K=%lld", (long long)M, (long long)K);
+  if (K == 0 || K % 64 != 0 || K > kMaxK || M > kMaxM)
+    return fail(TERN_ERR_UNSUPPORTED_SHAPE, "quantize_act_e4m3: need K %% 64 == 0, K <= 2^20, M <= 2^26 (M=%lld K=%lld)",
+                (long long)M, (long long)K);
+  if (M == 0) return TERN_OK;
+  if (!x_bf16 || !xq || !a) return fail(TERN_ERR_INVALID_ARG, "null x, xq or a");
+  if (!aligned(x_bf16, 16) || !aligned(xq, 16) || !aligned(a, 4))
+    return fail(TERN_ERR_MISALIGNED, "x and xq need 16-byte, a 4-byte alignment");
+  const size_t xb = size_t(M) * size_t(K) * 2, qb = size_t(M) * size_t(K), ab = size_t(M) * 4;
+  if (overlaps(xq, qb, x_bf16, xb) || overlaps(a, ab, x_bf16, xb) || overlaps(a, ab, xq, qb))
+    return fail(TERN_ERR_INVALID_ARG, "outputs overlap each other or x");
+  int dev;
+  DeviceState* ds;
+  tern_status s;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  cudaError_t e = launch_quantize_act_e4m3(static_cast<const __nv_bfloat16*>(x_bf16), int(M), int(K),
+                                           static_cast<uint8_t*>(xq), a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_act_e4m3 launch");
+  return TERN_OK;
+}
+
+tern_status tern_linear_e4m3(const void* xq, const float* a, int64_t M, int64_t K, const void* packed,
+                             const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                             tern_stream_t stream) {
+  tern_status s = check_nk(N, K);
+  if (s != TERN_OK) return s;
+  if (N % 256 != 0) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "linear_e4m3: need N %% 256 == 0, got N=%lld", (long long)N);
+  if (M < 0) return fail(TERN_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+  if (M > kMaxM) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "M above 2^26 (M=%lld)", (long long)M);
+  if (M == 0) return TERN_OK;
+  if (!xq || !a || !packed || !scales || !y_bf16) return fail(TERN_ERR_INVALID_ARG, "null xq, a, packed, scales or y");
+  if (!aligned(xq, 16) || !aligned(packed, 16) || !aligned(y_bf16, 16) || !aligned(scales, 4) || !aligned(a, 4) ||
+      (bias_bf16 && !aligned(bias_bf16, 2)))
+    return fail(TERN_ERR_MISALIGNED, "xq, packed and y need 16-byte, a and scales 4-byte, bias 2-byte alignment");
+  const size_t yb = size_t(M) * size_t(N) * 2;
+  if (overlaps(y_bf16, yb, xq, size_t(M) * size_t(K)) || overlaps(y_bf16, yb, a, size_t(M) * 4) ||
+      overlaps(y_bf16, yb, packed, packed_size(N, K)) || overlaps(y_bf16, yb, scales, size_t(N) * 4) ||
+      overlaps(y_bf16, yb, bias_bf16, bias_bf16 ? size_t(N) * 2 : 0))
+    return fail(TERN_ERR_INVALID_ARG, "y overlaps an input");
+  int dev;
+  DeviceState* ds;
+  if ((s = current_device(&dev, &ds)) != TERN_OK) return s;
+  if (ds->clusters_2sm <= 0) return fail(TERN_ERR_NO_DEVICE, "the device cannot co-schedule CTA pairs");
+  static Batch batch;  // built under the lock below; ~4 KiB, copied into the launch
+  static std::mutex batch_mu;
+  std::lock_guard<std::mutex> lock(batch_mu);
+  std::memset(static_cast<void*>(&batch), 0, sizeof batch);
+  Problem& p = batch.p[0];
+  if ((s = make_xq_map(&p.tmap_x, xq, M, K)) != TERN_OK) return s;
+  p.packed = static_cast<const uint8_t*>(packed);
+  p.scales = scales;
+  p.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  p.y = static_cast<__nv_bfloat16*>(y_bf16);
+  p.ws = const_cast<float*>(a);  // the per-token scales
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.n_tiles = int(N / 256);
+  p.m_tiles = int((M + 255) / 256);
+  p.splits = 1;
+  p.chunks_per_split = int(K / 64);
+  const int64_t tiles = int64_t(p.n_tiles) * p.m_tiles;
+  if (tiles > (int64_t(1) << 31) - 1) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "too many tiles");
+  batch.count = 1;
+  batch.total_units = int(tiles);
+  batch.wait_limit_ns = g_wait_limit_ns.load();
+  batch.status = ds->status;
+  cudaError_t e = launch_ternary_fp8(batch, int(std::min<int64_t>(tiles, ds->clusters_2sm)),
+                                     reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ternary_fp8 launch");
   return TERN_OK;
 }
 

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
             "tern_linear_act", "tern_linear_epilogue", "tern_linear_batch", "tern_linear_batch_act",
-            "tern_linear_batch_epilogue", "tern_adaln_modulate",
+            "tern_linear_batch_epilogue", "tern_adaln_modulate", "tern_quantize_act_e4m3", "tern_linear_e4m3",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -92,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.tern_linear_batch.restype = st
         L.tern_adaln_modulate.argtypes = [vp, i64, i64, vp, vp, i64, i64, ctypes.c_float, vp, vp]
         L.tern_adaln_modulate.restype = st
+        L.tern_quantize_act_e4m3.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.tern_quantize_act_e4m3.restype = st
+        L.tern_linear_e4m3.argtypes = [vp, vp, i64, i64, vp, vp, vp, i64, vp, vp]
+        L.tern_linear_e4m3.restype = st
         L.tern_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
         L.tern_dequantize.restype = st
         L.tern_get_device_status.argtypes = [vp]
@@ -269,6 +273,31 @@ def linear_batch_epilogue(problems: Sequence[dict], stream=None) -> None:
         args[i] = _linear_args(p)
         epis[i] = _epilogue(p)
     _check(lib().tern_linear_batch_epilogue(args, epis, len(problems), _stream(stream)))
+
+
+def quantize_act_e4m3(x: torch.Tensor, xq: Optional[torch.Tensor] = None, a: Optional[torch.Tensor] = None,
+                      stream=None):
+    """tern_quantize_act_e4m3: x bf16 [M,K] -> (xq uint8 [M,K] E4M3 bytes in the
+    interleaved k order of include/tern.h, a fp32 [M] per-token scales)."""
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+    if a is None:
+        a = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().tern_quantize_act_e4m3(_ptr(x), M, K, _ptr(xq), _ptr(a), _stream(stream)))
+    return xq, a
+
+
+def linear_e4m3(xq: torch.Tensor, a: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
+    """tern_linear_e4m3: y = a_m * s_n * sum_k xq[m,k] T[n,k] + b_n -> bf16 [M,N]."""
+    M, K = xq.shape
+    N = scales.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+    _check(lib().tern_linear_e4m3(_ptr(xq), _ptr(a), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
+                                  _stream(stream)))
+    return out
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional[torch.Tensor] = None,

@@ -284,6 +284,38 @@ TERN_API tern_status tern_adaln_modulate(const void* x, int64_t M, int64_t K, co
                                 int64_t mod_ld, int64_t tokens_per_row, float eps, void* out,
                                 tern_stream_t stream);
 
+/*
+ * FP8 (E4M3) activations for the ternary linear (page "1.58-bit FLUX",
+ * Section 4: the method keeps activations at 16 bits and names quantising them
+ * as the step that would turn the 2-bit weights into a latency gain; the pages
+ * fix no format, so this is one reading of it).  Per token row m:
+ *     a_m = max_k |x[m,k]| / 448   (fp32, IEEE division; 1 for an all-zero row)
+ *     xq[m,k] = E4M3(x[m,k] / a_m) (fp32 IEEE division, round to nearest even,
+ *                                  saturating at +-448; subnormals kept)
+ * and the layer  y[m,n] = a_m * s_n * sum_k xq[m,k] * T[n,k] + b_n  with fp32
+ * accumulation (the ternary weights are exact E4M3 values), rounded once to
+ * bf16.  The only new error against tern_linear is the activation rounding
+ * (at most 2^-4 relative per element).
+ *
+ * tern_quantize_act_e4m3: x [M, K] bf16 (16-byte aligned) -> xq [M, K] bytes
+ * (16-byte aligned) and a [M] fp32 (4-byte aligned), all device memory owned
+ * by the caller; K % 64 == 0.  Layout of xq: row-major, but inside every group
+ * of 16 consecutive k the two halves are interleaved -- byte 16g + 2i holds
+ * E4M3 of k = 16g + i and byte 16g + 2i + 1 holds k = 16g + 8 + i (i < 8) --
+ * the order tern_linear_e4m3's kernel expands the weights in.  One launch.
+ */
+TERN_API tern_status tern_quantize_act_e4m3(const void* x_bf16, int64_t M, int64_t K, void* xq, float* a,
+                                            tern_stream_t stream);
+
+/* The layer on E4M3 activations from tern_quantize_act_e4m3: xq [M, K] in its
+ * interleaved layout and a [M]; packed, scales, bias and y as tern_linear.
+ * N % 256 == 0 (CTA-pair tiles of 256 channels; TERN_ERR_UNSUPPORTED_SHAPE
+ * otherwise), K % 64 == 0, M >= 0.  y must not overlap an input.  One launch;
+ * no workspace. */
+TERN_API tern_status tern_linear_e4m3(const void* xq, const float* a, int64_t M, int64_t K, const void* packed,
+                                      const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
+                                      tern_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: TERN_ERR_TIMEOUT if any kernel's bounded wait ran out since
  * the last call, else TERN_ERR_LAUNCH_CONFIG if a kernel refused an

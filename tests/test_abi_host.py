@@ -259,3 +259,38 @@ def test_adaln_binding_checks_row_layout():
         tern.adaln_modulate(x, mod[:, 64:128].t().contiguous().t(), mod[:, :64])  # columns strided
     with pytest.raises(ValueError):
         tern.adaln_modulate(x, mod[:, 64:128], torch.zeros(2, 64, dtype=torch.bfloat16))  # 384 vs 64 apart
+
+
+def test_quantize_act_e4m3_rejects_on_host(L):
+    q = lambda x=F, M=16, K=256, xq=F + 0x1000000, a=F + 0x2000000: L.tern_quantize_act_e4m3(
+        ctypes.c_void_p(x), M, K, ctypes.c_void_p(xq), ctypes.c_void_p(a), None)
+    assert q(K=100) == SHAPE
+    assert q(K=0) == SHAPE
+    assert q(M=-1) == INVALID
+    assert q(M=1 << 27) == SHAPE
+    assert q(x=0) == INVALID
+    assert q(a=0) == INVALID
+    assert q(x=F + 2) == MISALIGNED
+    assert q(xq=F + 0x1000008) == MISALIGNED
+    assert q(a=F + 0x2000002) == MISALIGNED
+    assert q(xq=F + 0x100) == INVALID   # xq overlaps x
+    assert q(a=F + 0x1000010) == INVALID  # a overlaps xq
+    assert q(M=0, x=0, xq=0, a=0) == OK  # empty: nothing to do, nothing checked
+
+
+def test_linear_e4m3_rejects_on_host(L):
+    f = lambda xq=F, a=F + 0x80000, M=16, K=256, P=F + 0x100000, S=F + 0x200000, b=None, N=256, y=F + 0x300000: \
+        L.tern_linear_e4m3(ctypes.c_void_p(xq), ctypes.c_void_p(a), M, K, ctypes.c_void_p(P), ctypes.c_void_p(S),
+                           None if b is None else ctypes.c_void_p(b), N, ctypes.c_void_p(y), None)
+    assert f(N=128) == SHAPE      # the FP8 kernel tiles 256 channels per CTA pair
+    assert f(N=100) == SHAPE
+    assert f(K=96) == SHAPE
+    assert f(M=-1) == INVALID
+    assert f(a=0) == INVALID
+    assert f(xq=0) == INVALID
+    assert f(xq=F + 4) == MISALIGNED
+    assert f(a=F + 0x80002) == MISALIGNED
+    assert f(y=F + 0x300008) == MISALIGNED
+    assert f(y=F) == INVALID          # y aliases xq
+    assert f(y=F + 0x80000) == INVALID  # y aliases a
+    assert f(M=0, xq=0, a=0, y=0) == OK
