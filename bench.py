@@ -44,6 +44,9 @@ def parse_args():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="layer the step runs on (default: the QKV headline; others for profiling)")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-kernel side table")
+    ap.add_argument("--fp8", action="store_true",
+                    help="run the step on FP8 (E4M3) activations: quantise/pack W, quantise x per token "
+                         "row, the kind::f8f6f4 layer (not the headline; no CPU baseline, no side table)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU oracle sample budget (0 skips the CPU baseline, for profiling runs)")
     return ap.parse_args()
@@ -268,11 +271,12 @@ DESCRIPTIONS = {"qkv": "FLUX.1-dev double-block image-stream QKV, 1024x1024 imag
                 "tiny": "tiny ternary linear"}
 
 
-def workload_config(layer):
+def workload_config(layer, fp8=False):
     what = DESCRIPTIONS.get(layer.name, f"FLUX.1-dev adaLN modulation GEMV ({layer.name})")
     return {"workload": f"{what}: x [{layer.M},{layer.K}] bf16, W [{layer.N},{layer.K}] ternary, bias bf16",
             "M": layer.M, "K": layer.K, "N": layer.N, "eps": 1e-5,
-            "step": "tern_quantize_pack(W) + tern_linear(x)",
+            "step": ("tern_quantize_pack(W) + tern_quantize_act_e4m3(x) + tern_linear_e4m3" if fp8 else
+                     "tern_quantize_pack(W) + tern_linear(x)"),
             "accumulate": "fp32",
             "l2": "two rotating input sets of 164 MB each (> 126 MB L2)"}
 
@@ -355,6 +359,8 @@ def make_sets(layer, rank, n_sets, device):
             "packed": torch.empty(layer.N * layer.K // 4, dtype=torch.uint8, device=device),
             "scales": torch.empty(layer.N, dtype=torch.float32, device=device),
             "y": torch.empty(layer.M, layer.N, dtype=torch.bfloat16, device=device),
+            "xq": torch.empty(layer.M, layer.K, dtype=torch.uint8, device=device),
+            "a": torch.empty(layer.M, dtype=torch.float32, device=device),
             "cpu": (x, W, b),
         })
     return sets
@@ -609,14 +615,26 @@ def run_tern(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(K)]
 
+    def layer_call(st):
+        if args.fp8:
+            tern.quantize_act_e4m3(st["x"], xq=st["xq"], a=st["a"], stream=stream)
+            tern.linear_e4m3(st["xq"], st["a"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        else:
+            tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+
     def step(i, events=None):
         st = sets[i % len(sets)]
         if events:
             events[0].record(stream)
         tern.quantize_pack(st["W"], workloads.EPS, packed=st["packed"], scales=st["scales"], stream=stream)
+        if args.fp8:
+            tern.quantize_act_e4m3(st["x"], xq=st["xq"], a=st["a"], stream=stream)
         if events:
             events[1].record(stream)
-        tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        if args.fp8:
+            tern.linear_e4m3(st["xq"], st["a"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        else:
+            tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
         if events:
             events[2].record(stream)
 
@@ -676,7 +694,7 @@ def run_tern(args):
         if used[j]:
             stream.wait_event(ev_out[j])  # step i - nset's y has left the device
         tern.quantize_pack(st["W"], workloads.EPS, packed=st["packed"], scales=st["scales"], stream=stream)
-        tern.linear(st["x"], st["packed"], st["scales"], st["b"], out=st["y"], stream=stream)
+        layer_call(st)
         ev_comp[j].record(stream)
         s_out.wait_event(ev_comp[j])
         with torch.cuda.stream(s_out):
@@ -709,14 +727,21 @@ def run_tern(args):
     tensor_bound = flop / (peaks["bf16_tflops"] * 1e12) >= layer.algorithmic_bytes / (peaks["hbm_gbs"] * 1e9)
     kname, kstem = linear_kernel(layer)
     traffic = profiled_traffic(kstem, layer.name)
+    if args.fp8:
+        # FP8 tensor peak: the measured bf16 burst x 2 (the nominal dense ratio)
+        peaks = dict(peaks, bf16_tflops=2.0 * peaks["bf16_tflops"], source=peaks["source"] + " bf16 x 2 (FP8)")
+        kname, kstem = "ternary_fp8_pair_kernel", "ternary_fp8"
+        traffic = profiled_traffic(kstem, layer.name)
+        tensor_bound = True
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, FLUX.1-dev QKV shapes)",
-        "config": workload_config(layer),
+        "vs_baseline": None, "dtype": "e4m3 x, ternary w" if args.fp8 else "bf16",
+        "data": "synthetic (seeded, FLUX.1-dev QKV shapes)",
+        "config": workload_config(layer, args.fp8),
         "roofline": ({"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                       "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                      "kernel": f"{kname} (tern_linear)",
+                      "kernel": f"{kname} ({'tern_linear_e4m3' if args.fp8 else 'tern_linear'})",
                       "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)"}
                      if tensor_bound else
                      {"bound": "hbm", "achieved": layer.algorithmic_bytes / t_lin / 1e9,
@@ -729,10 +754,10 @@ def run_tern(args):
         "quantize_pack_gbs": (2 * layer.N * layer.K + layer.packed_bytes + 4 * layer.N) / t_quant / 1e9,
         "e2e": {"value": job_throughput(world, K, flop, e2e_elapsed), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * K * world,
+        "gpu_launches": (3 if args.fp8 else 2) * K * world,
         "clocks": clocks.summary(),
     }
-    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0 and not args.fp8:
         line["cpu_baseline"] = cpu_baseline(layer, *sets[0]["cpu"], budget_s=args.cpu_seconds)
         if not args.no_extras:
             try:

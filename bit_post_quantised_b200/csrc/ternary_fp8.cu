@@ -11,17 +11,20 @@
 //
 // Two kernels:
 //   * quantize_act_e4m3_kernel: one warp per token row; the row's absolute
-//     maximum, a_m = max / 448 and x / a_m in fp32 with IEEE division, each
-//     rounded to E4M3 to nearest even with saturation (cvt.rn.satfinite).
+//     maximum, a_m = max / 448 (IEEE fp32 division) and x / a_m rounded to
+//     fp32 exactly as IEEE division would (an fp64 multiply by the fp64
+//     reciprocal; the kernel states why that is exact for bf16 x), then to
+//     E4M3 to nearest even with saturation (cvt.rn.satfinite).
 //     Inside every 16-element group of k the two halves are interleaved:
 //     byte 2i holds k = i and byte 2i + 1 holds k = 8 + i (i < 8).  That is
 //     the k order in which the weight expansion below is cheapest; the MMA
 //     sums over k, so the same order on both operands changes nothing.
 //   * ternary_fp8_pair_kernel: the CTA-pair tile kernel of the bf16 path
 //     (256 channels x 256 tokens per pair, tcgen05 cta_group::2, weights
-//     decoded into TMEM as the A operand) with 128-k stages of one 2-D TMA box
-//     of E4M3 x (128 tokens x 128 bytes per CTA) and 4 KiB of codes, four
-//     K = 32 MMAs per stage.  A code shifted so its two bits land on bits 7
+//     decoded into TMEM as the A operand) with 256-k stages of two 2-D TMA
+//     boxes of E4M3 x (128 tokens x 128 bytes each per CTA) and 8 KiB of
+//     codes, eight K = 32 MMAs per stage (1024 tensor cycles between two
+//     barrier handshakes, as in a bf16 stage).  A code shifted so its two bits land on bits 7
 //     and 6 of a byte is the E4M3 value 2t (0x40 = 2, 0xC0 = -2, 0 = 0; the
 //     unused pattern 10 reads as -0): one shift and one AND yield four bytes,
 //     the codes of k = 2q, 8 + 2q, 2q + 1 and 9 + 2q of a 16-k word for
@@ -58,45 +61,86 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 
 }  // namespace
 
-// One warp per token row, eight rows per CTA.  K % 64 == 0; x, xq 16-byte
-// aligned rows.
-__global__ void __launch_bounds__(256) quantize_act_e4m3_kernel(const uint16_t* __restrict__ x, int M, int K,
+// One warp per token row, eight rows per CTA (four CTAs per SM for K <= 3072,
+// so the 4096 rows of a FLUX image stream run in one wave).  K % 64 == 0; x,
+// xq 16-byte aligned rows.  NV > 0: the row is held in registers (lane l keeps the
+// 16-element groups l, l + 32, ..., NV per lane, K <= 512 NV), so x is read
+// once; NV == 0: any K, the row is read twice (the second time mostly from
+// L2).
+template <int NV>
+__global__ void __launch_bounds__(256, NV > 6 ? 2 : 4) quantize_act_e4m3_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                  uint8_t* __restrict__ xq, float* __restrict__ a) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= M) return;
   const uint16_t* xr = x + size_t(row) * K;
-  const int groups = K >> 4;  // 16-element groups of the row
-  float mx = 0.f;
-  for (int g = lane; g < groups; g += 32) {
-    const uint4 v0 = *reinterpret_cast<const uint4*>(xr + 16 * g);
-    const uint4 v1 = *reinterpret_cast<const uint4*>(xr + 16 * g + 8);
-    float f0[8], f1[8];
-    bf16x8_to_f32(v0, f0);
-    bf16x8_to_f32(v1, f1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fmaxf(fabsf(f0[i]), fabsf(f1[i])));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const float am = mx > 0.f ? __fdiv_rn(mx, kE4M3Max) : 1.0f;
-  if (lane == 0) a[row] = am;
   uint8_t* qr = xq + size_t(row) * K;
-  for (int g = lane; g < groups; g += 32) {  // the row again, mostly from L1/L2
-    const uint4 v0 = *reinterpret_cast<const uint4*>(xr + 16 * g);
-    const uint4 v1 = *reinterpret_cast<const uint4*>(xr + 16 * g + 8);
+  const int groups = K >> 4;  // 16-element groups of the row
+  // x / a_m rounded to fp32 as IEEE division would, from one fp64 multiply
+  // by the fp64 reciprocal r = RN64(1 / a_m).  x is a bf16 (8 significant
+  // bits) and a_m an fp32 (24), so x / a_m is never exactly halfway between
+  // two fp32 numbers, and when it is not, it lies at least 2^-49 (relative)
+  // from such a midpoint; RN64(x r) is within 2^-52 (relative) of x / a_m,
+  // so rounding it to fp32 gives RN32(x / a_m).  (Where x / a_m falls into
+  // the fp32 subnormals the E4M3 code is a signed zero either way.)
+  auto q32 = [](float v, double r) { return __double2float_rn(double(v) * r); };
+  // bytes 4j .. 4j + 3 of a group's output = k 2j, 8 + 2j, 2j + 1, 9 + 2j
+  auto emit = [&](int g, const uint4& v0, const uint4& v1, double r) {
     float f0[8], f1[8];
     bf16x8_to_f32(v0, f0);
     bf16x8_to_f32(v1, f1);
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      // bytes 4j .. 4j + 3 = k 2j, 8 + 2j, 2j + 1, 9 + 2j
-      const uint16_t lo = e4m3x2(__fdiv_rn(f1[2 * j], am), __fdiv_rn(f0[2 * j], am));
-      const uint16_t hi = e4m3x2(__fdiv_rn(f1[2 * j + 1], am), __fdiv_rn(f0[2 * j + 1], am));
+      const uint16_t lo = e4m3x2(q32(f1[2 * j], r), q32(f0[2 * j], r));
+      const uint16_t hi = e4m3x2(q32(f1[2 * j + 1], r), q32(f0[2 * j + 1], r));
       w[j] = uint32_t(lo) | (uint32_t(hi) << 16);
     }
     *reinterpret_cast<uint4*>(qr + 16 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+  };
+  auto absmax8 = [](const uint4& v) {
+    // |bf16| as bits: clear the sign; the largest magnitude has the largest bits
+    const uint32_t m = 0x7FFF7FFFu;
+    const uint32_t a0 = max(max((v.x & m) & 0xFFFFu, (v.x & m) >> 16), max((v.y & m) & 0xFFFFu, (v.y & m) >> 16));
+    const uint32_t a1 = max(max((v.z & m) & 0xFFFFu, (v.z & m) >> 16), max((v.w & m) & 0xFFFFu, (v.w & m) >> 16));
+    return max(a0, a1);
+  };
+  uint32_t mb = 0;  // the bits of the largest magnitude so far (bf16 magnitudes order as integers)
+  if constexpr (NV > 0) {
+    uint4 v[NV][2];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int g = lane + 32 * i;
+      if (g < groups) {
+        v[i][0] = *reinterpret_cast<const uint4*>(xr + 16 * g);
+        v[i][1] = *reinterpret_cast<const uint4*>(xr + 16 * g + 8);
+      } else {
+        v[i][0] = v[i][1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) mb = max(mb, max(absmax8(v[i][0]), absmax8(v[i][1])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float mx = __uint_as_float(mb << 16);
+    const float am = mx > 0.f ? __fdiv_rn(mx, kE4M3Max) : 1.0f;
+    if (lane == 0) a[row] = am;
+    const double r = 1.0 / double(am);
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      if (lane + 32 * i < groups) emit(lane + 32 * i, v[i][0], v[i][1], r);
+  } else {
+    for (int g = lane; g < groups; g += 32)
+      mb = max(mb, max(absmax8(*reinterpret_cast<const uint4*>(xr + 16 * g)),
+                       absmax8(*reinterpret_cast<const uint4*>(xr + 16 * g + 8))));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float mx = __uint_as_float(mb << 16);
+    const float am = mx > 0.f ? __fdiv_rn(mx, kE4M3Max) : 1.0f;
+    if (lane == 0) a[row] = am;
+    const double r = 1.0 / double(am);
+    for (int g = lane; g < groups; g += 32)  // the row again, mostly from L2
+      emit(g, *reinterpret_cast<const uint4*>(xr + 16 * g), *reinterpret_cast<const uint4*>(xr + 16 * g + 8), r);
   }
 }
 
@@ -105,14 +149,15 @@ namespace {
 struct F8Cfg {
   static constexpr int kTokPair = 256;            // UMMA N: tokens per pair tile
   static constexpr int kTokCta = 128;             // x rows each CTA loads
-  static constexpr int kBK = 128;                 // k per stage
-  static constexpr int kXBytes = kTokCta * 128;   // 128 rows x 128 E4M3, 128-byte swizzle
+  static constexpr int kChunks = 4;               // 64-k chunks per stage: 256 k
+  static constexpr int kXBox = kTokCta * 128;     // 128 rows x 128 E4M3 bytes, 128-byte swizzle
+  static constexpr int kXBytes = 2 * kXBox;       // two boxes: k 0-127 and 128-255 of the stage
   static constexpr int kCSub = 128 * 16;          // codes of 128 channels x 64 k
-  static constexpr int kCBytes = 2 * kCSub;
-  static constexpr int kStageBytes = kXBytes + kCBytes;  // 20 KiB
-  static constexpr int kStages = 10;
-  static constexpr int kASlots = 8;               // decoded-weight slots in TMEM
-  static constexpr int kACols = kBK / 4;          // 32-bit TMEM columns per slot (four E4M3)
+  static constexpr int kCBytes = kChunks * kCSub;
+  static constexpr int kStageBytes = kXBytes + kCBytes;  // 40 KiB
+  static constexpr int kStages = 5;
+  static constexpr int kASlots = 4;               // decoded-weight slots in TMEM, one stage each
+  static constexpr int kACols = kChunks * 16;     // 32-bit TMEM columns per slot (four E4M3)
   static constexpr int kDCols = kTokPair;         // one fp32 accumulator
   static constexpr int kACol0 = kDCols;
   static constexpr int kTmemCols = 512;
@@ -130,43 +175,54 @@ struct F8Cfg {
   static_assert(kSmemBytes <= 220 * 1024, "shared memory");
 };
 
-// Four (or, for a 64-k tail, two) K = 32 MMAs of one stage and two commits,
-// issued by the lane elect.sync picks in the converged MMA warp.  A: the
-// stage's TMEM slot, step j at a + 8 j; B: the stage's x box, step j adds 32
-// bytes (2 in the descriptor's address field).
+// The K = 32 MMAs of one stage (2 per 64-k chunk: NMMA = 2, 4, 6 or 8) and two
+// commits, issued by the lane elect.sync picks in the converged MMA warp, as
+// one block (uniform operands; per-MMA arithmetic in a single-lane branch
+// measured several times slower on the bf16 kernels).  A: the stage's TMEM
+// slot, MMA j at a + 8 j.  B: the stage's two x boxes; MMA j reads 32 bytes
+// at 32 (j % 4) of box j / 4 (descriptor address units of 16 bytes: + 2 per
+// MMA, + 1024 for the second 16 KiB box).
+#define F8_MMA(AR, ER, P) "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [" AR "], " ER ", %3, " P ";\n\t"
+#define F8_COMMITS                                                                                       \
+  "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%5], %7;\n\t" \
+  "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%6], %7;\n\t}"
+#define F8_PROLOGUE                                                                              \
+  "{\n\t.reg .pred p, q, t;\n\t.reg .b64 e1, e2, e3, e4, e5, e6, e7;\n\t"                     \
+  ".reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"                                                   \
+  "elect.sync _|p, 0xffffffff;\n\tsetp.ne.b32 q, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"           \
+  "add.s64 e1, %2, 2;\n\tadd.s64 e2, %2, 4;\n\tadd.s64 e3, %2, 6;\n\tadd.s64 e4, %2, 1024;\n\t" \
+  "add.s64 e5, %2, 1026;\n\tadd.s64 e6, %2, 1028;\n\tadd.s64 e7, %2, 1030;\n\t"                \
+  "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\tadd.u32 a4, %1, 32;\n\t" \
+  "add.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+#define F8_M01 F8_MMA("%1", "%2", "q") F8_MMA("a1", "e1", "t")
+#define F8_M23 F8_MMA("a2", "e2", "t") F8_MMA("a3", "e3", "t")
+#define F8_M45 F8_MMA("a4", "e4", "t") F8_MMA("a5", "e5", "t")
+#define F8_M67 F8_MMA("a6", "e6", "t") F8_MMA("a7", "e7", "t")
+#define F8_ARGS                                                                                  \
+  ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "h"(both) : "memory"
+
 template <int NMMA>
 __device__ __forceinline__ void mma_stage_f8(uint32_t d, uint32_t a, uint64_t desc, uint32_t idesc, uint32_t acc,
                                              uint32_t bar0, uint32_t bar1) {
-  static_assert(NMMA == 2 || NMMA == 4, "a stage is one or two 64-k halves");
+  static_assert(NMMA == 2 || NMMA == 4 || NMMA == 6 || NMMA == 8, "two MMAs per 64-k chunk");
   const uint16_t both = 0x3;
-  if constexpr (NMMA == 4)
-    asm volatile(
-        "{\n\t.reg .pred p, q, t;\n\t.reg .b64 e1, e2, e3;\n\t.reg .b32 a1, a2, a3;\n\t"
-        "elect.sync _|p, 0xffffffff;\n\t"
-        "setp.ne.b32 q, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
-        "add.s64 e1, %2, 2;\n\tadd.s64 e2, %2, 4;\n\tadd.s64 e3, %2, 6;\n\t"
-        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [%1], %2, %3, q;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [a1], e1, %3, t;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [a2], e2, %3, t;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [a3], e3, %3, t;\n\t"
-        "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%5], %7;\n\t"
-        "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%6], %7;\n\t}"
-        ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "h"(both)
-        : "memory");
+  if constexpr (NMMA == 8)
+    asm volatile(F8_PROLOGUE F8_M01 F8_M23 F8_M45 F8_M67 F8_COMMITS F8_ARGS);
+  else if constexpr (NMMA == 6)
+    asm volatile(F8_PROLOGUE F8_M01 F8_M23 F8_M45 F8_COMMITS F8_ARGS);
+  else if constexpr (NMMA == 4)
+    asm volatile(F8_PROLOGUE F8_M01 F8_M23 F8_COMMITS F8_ARGS);
   else
-    asm volatile(
-        "{\n\t.reg .pred p, q, t;\n\t.reg .b64 e1;\n\t.reg .b32 a1;\n\t"
-        "elect.sync _|p, 0xffffffff;\n\t"
-        "setp.ne.b32 q, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
-        "add.s64 e1, %2, 2;\n\tadd.u32 a1, %1, 8;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [%1], %2, %3, q;\n\t"
-        "@p tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], [a1], e1, %3, t;\n\t"
-        "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%5], %7;\n\t"
-        "@p tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%6], %7;\n\t}"
-        ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "h"(both)
-        : "memory");
+    asm volatile(F8_PROLOGUE F8_M01 F8_COMMITS F8_ARGS);
 }
+#undef F8_MMA
+#undef F8_COMMITS
+#undef F8_PROLOGUE
+#undef F8_M01
+#undef F8_M23
+#undef F8_M45
+#undef F8_M67
+#undef F8_ARGS
 
 // The E4M3 bytes of 2t for the 16 codes of one code word, as four 32-bit
 // TMEM columns: column q holds k = 2q, 8 + 2q, 2q + 1, 9 + 2q of the word's
@@ -262,9 +318,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------ TMA producer (one lane)
-    if (lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    // Stage it is issued by lane it % S (each lane owns one ring slot): one
+    // thread issues a copy only every ~280 SM cycles, and a stage is three
+    // copies.
+    if (lane == 0)
       for (int pi = 0; pi < batch.count; ++pi) prefetch_tensormap(&batch.p[pi].tmap_x);
+    __syncwarp();
+    if (lane < S) {
       int it = 0;
       bool ok = true;
       for (int u = u0; u < units && ok; u += ustep) {
@@ -273,21 +334,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
         const int kc_total = P.K >> 6;
         const uint8_t* codes = P.packed + size_t(2 * nt + int(rank)) * kc_total * C::kCSub;
         const int row = mt * C::kTokPair + int(rank) * C::kTokCta;
-        for (int kc = 0; kc < kc_total; kc += 2, ++it) {
-          const int s = it % S;
+        for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
+          if (it % S != lane) continue;
+          const int s = lane;
           ok = mbar_wait(smem_u32(&empty_bar[s]), ((it / S) & 1) ^ 1, lim, st);
           if (!ok) break;
-          const int nsub = min(2, kc_total - kc);
+          const int nch = min(C::kChunks, kc_total - kc);
           const uint32_t stage = smem_base + s * C::kStageBytes;
           const uint32_t fb = smem_u32(&full_bar[s]);
-          // 128 k of E4M3 x (zero past K and past M) and the stage's codes.
-          mbar_arrive_expect_tx(fb, C::kXBytes + nsub * C::kCSub);
+          // 256 k of E4M3 x as two 128-byte-wide boxes (zero past K and past
+          // M) and the stage's codes, one block.
+          mbar_arrive_expect_tx(fb, C::kXBytes + nch * C::kCSub);
           tma_load_2d(stage, &P.tmap_x, kc * 64, row, fb);
-          tma_load_bulk(stage + C::kXBytes, codes + size_t(kc) * C::kCSub, nsub * C::kCSub, fb);
+          tma_load_2d(stage + C::kXBox, &P.tmap_x, kc * 64 + 128, row, fb);
+          tma_load_bulk(stage + C::kXBytes, codes + size_t(kc) * C::kCSub, nch * C::kCSub, fb);
         }
       }
-      // No copy may still be landing in shared memory when the CTA exits.
-      for (int i = it > S ? it - S : 0; i < it; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1, lim, st);
+      // No copy this lane issued may still be landing when the CTA exits.
+      if (it > lane) {
+        const int last = lane + ((it - 1 - lane) / S) * S;  // this lane's last stage
+        mbar_wait(smem_u32(&full_bar[lane]), (last / S) & 1, lim, st);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -302,7 +369,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
         ok = warp_wait_f8(smem_u32(&accempty_bar), (lt & 1) ^ 1, lim, st, lane);
         if (!ok) break;
         tc_fence_after();
-        for (int kc = 0; kc < kc_total; kc += 2, ++it) {
+        for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
           const int s = it % S, a = it % A;
           ok = warp_wait_f8(smem_u32(&afull_bar[a]), (it / A) & 1, lim, st, lane);
           if (!ok) break;
@@ -310,7 +377,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
           const uint32_t a_tmem = tmem_u + C::kACol0 + a * C::kACols;
           const uint64_t desc = sw128_kmajor_desc(smem_base + s * C::kStageBytes);
           const uint32_t bar0 = smem_u32(&empty_bar[s]), bar1 = smem_u32(&aempty_bar[a]);
-          if (kc + 1 < kc_total)
+          const int nch = min(C::kChunks, kc_total - kc);
+          if (nch == 4)
+            mma_stage_f8<8>(tmem_u, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1);
+          else if (nch == 3)
+            mma_stage_f8<6>(tmem_u, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1);
+          else if (nch == 2)
             mma_stage_f8<4>(tmem_u, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1);
           else
             mma_stage_f8<2>(tmem_u, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1);
@@ -335,7 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
     for (int u = u0; u < units && ok; u += ustep) {
       int mt, nt;
       const int kc_total = unit_problem(u, &mt, &nt).K >> 6;
-      for (int kc = 0; kc < kc_total; kc += 2, ++it) {
+      for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
         const int s = it % S, a = it % A;
         bool got = true;
         if (lane == 0) {
@@ -347,23 +419,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint8_t* cp = smem_gen + s * C::kStageBytes + C::kXBytes + r * 16;
-        uint32_t t[32];
-        const uint4 v0 = *reinterpret_cast<const uint4*>(cp);
-        decode_word_e4m3(v0.x, t + 0);
-        decode_word_e4m3(v0.y, t + 4);
-        decode_word_e4m3(v0.z, t + 8);
-        decode_word_e4m3(v0.w, t + 12);
-        if (kc + 1 < kc_total) {
-          const uint4 v1 = *reinterpret_cast<const uint4*>(cp + C::kCSub);
-          decode_word_e4m3(v1.x, t + 16);
-          decode_word_e4m3(v1.y, t + 20);
-          decode_word_e4m3(v1.z, t + 24);
-          decode_word_e4m3(v1.w, t + 28);
-        } else {
+        const uint32_t dst = tmem + lane_off + C::kACol0 + a * C::kACols;
+        // Two 128-k halves of the stage, 32 columns each (a half past K is
+        // not written: its MMAs are not issued).
 #pragma unroll
-          for (int i = 16; i < 32; ++i) t[i] = 0u;  // never read: the tail stage issues two MMAs
-        }
-        tmem_st32(tmem + lane_off + C::kACol0 + a * C::kACols, t);
+        for (int h = 0; h < 2; ++h)
+          if (kc + 2 * h < kc_total) {
+            uint32_t t[32];
+            const uint4 v0 = *reinterpret_cast<const uint4*>(cp + (2 * h) * C::kCSub);
+            decode_word_e4m3(v0.x, t + 0);
+            decode_word_e4m3(v0.y, t + 4);
+            decode_word_e4m3(v0.z, t + 8);
+            decode_word_e4m3(v0.w, t + 12);
+            if (kc + 2 * h + 1 < kc_total) {
+              const uint4 v1 = *reinterpret_cast<const uint4*>(cp + (2 * h + 1) * C::kCSub);
+              decode_word_e4m3(v1.x, t + 16);
+              decode_word_e4m3(v1.y, t + 20);
+              decode_word_e4m3(v1.z, t + 24);
+              decode_word_e4m3(v1.w, t + 28);
+            } else {
+#pragma unroll
+              for (int i = 16; i < 32; ++i) t[i] = 0u;  // past K: never read
+            }
+            tmem_st32(dst + 32 * h, t);
+          }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -394,30 +473,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
       const float ahi = lane + 32 < rows ? ascale[row0 + 32 + lane] : 0.f;
       if (!warp_wait_f8(smem_u32(&accfull_bar), lt & 1, lim, st, lane)) break;
       tc_fence_after();
-      // y = acc * (a_m s_n / 2) + b_n, packed to bf16x2 while the
-      // accumulator is read; it is released before the stores.
-      uint32_t out[kCols / 2];
+      // The accumulator goes to registers and is released at once (the next
+      // tile's MMAs wait for it); y = acc * (a_m s_n / 2) + b_n comes after.
+      float f[kCols];
 #pragma unroll
       for (int c0 = 0; c0 < kCols; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + part * kCols + c0, v);
-        tmem_wait_ld();
-        const float ah = c0 == 0 ? alo : ahi;
+        tmem_wait_ld();  // the registers hold the values only after the wait
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float a0 = __shfl_sync(0xffffffffu, ah, j);
-          const float a1 = __shfl_sync(0xffffffffu, ah, j + 1);
-          out[(c0 + j) / 2] = pack_bf16x2_rn(fmaf(__uint_as_float(v[j]), sc * a0, bi),
-                                             fmaf(__uint_as_float(v[j + 1]), sc * a1, bi));
-        }
+        for (int j = 0; j < 32; ++j) f[c0 + j] = __uint_as_float(v[j]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(accempty_leader);  // the next tile's MMAs may start
       uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
 #pragma unroll
-      for (int c = 0; c < kCols; ++c)
-        if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+      for (int c = 0; c < kCols; ++c) {
+        const float am = __shfl_sync(0xffffffffu, c < 32 ? alo : ahi, c & 31);
+        const float y = fmaf(f[c], sc * am, bi);
+        if (c < rows) yp[size_t(c) * P.N] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+      }
     }
   }
 
@@ -433,7 +509,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
 cudaError_t launch_quantize_act_e4m3(const __nv_bfloat16* x, int M, int K, uint8_t* xq, float* a,
                                      cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
-  quantize_act_e4m3_kernel<<<(M + 7) / 8, 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(x), M, K, xq, a);
+  const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+  const dim3 grid((M + 7) / 8);
+  if (K <= 512 * 2) quantize_act_e4m3_kernel<2><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
+  else if (K <= 512 * 4) quantize_act_e4m3_kernel<4><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
+  else if (K <= 512 * 6) quantize_act_e4m3_kernel<6><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
+  else if (K <= 512 * 8) quantize_act_e4m3_kernel<8><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
+  else quantize_act_e4m3_kernel<0><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
   return cudaGetLastError();
 }
 

@@ -95,6 +95,20 @@ def test_quantize_act_special_rows():
     assert list(nat[1, :4]) == [0x7E, 0x38, 0x3A, 0xC4]  # 448, 1.0, 1.25, -3.0
 
 
+def test_quantize_act_scales_across_the_exponent_range():
+    """Rows whose magnitudes span bf16's exponent range (1e-38 .. 1e38, bf16
+    subnormals included) and random mantissas, so that x / a_m and its fp32
+    rounding are exercised far from 1: every byte must still match the
+    oracle's fp32 division."""
+    M, K = 512, 1024
+    g = torch.Generator().manual_seed(31)
+    mant = torch.rand(M, K, generator=g) * 2 - 1
+    expo = torch.randint(-130, 127, (M, 1), generator=g).float()
+    spread = torch.randint(-20, 1, (M, K), generator=g).float()
+    x = (mant * torch.pow(2.0, (expo + spread).clamp(-133, 127))).to(torch.bfloat16)
+    check_act(x)
+
+
 def test_quantize_act_empty_is_a_no_op():
     x = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
     xq, a = tern.quantize_act_e4m3(x)
