@@ -27,6 +27,7 @@ struct alignas(64) Problem {
   const __nv_bfloat16* gate;      // [N] or null (gate 1)
   int norm_col0, norm_col1;       // RMS-normalised columns (128-column groups), empty if equal
   float norm_eps;
+  int ldy;                        // elements between rows of y (and of the residual), >= N
   const __nv_bfloat16* norm_weight;  // [N] or null (weight 1)
 };
 static_assert(sizeof(Problem) == 256, "Problem layout");

@@ -109,11 +109,11 @@ EncodeTiledFn encode_fn() {
 
 // x [M, K] bf16 row-major; box = 64 k x tok rows; 128-byte swizzle; rows past
 // M read as zero.
-tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int tok) {
+tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx, int tok) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
-  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+  const cuuint64_t strides[1] = {cuuint64_t(ldx) * 2};
   const cuuint32_t box[2] = {64, cuuint32_t(tok)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
@@ -127,11 +127,12 @@ tern_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, in
 // {64, rows, chunks} lands as [chunk][token][64 k] with 128-byte swizzle, so
 // one copy brings several 64-k chunks; tokens past M and chunks past K read
 // as zero.
-tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_t K, int rows, int chunks) {
+tern_status make_x_map_chunks(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx, int rows,
+                              int chunks) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(TERN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[3] = {64, cuuint64_t(M), cuuint64_t(K / 64)};
-  const cuuint64_t strides[2] = {cuuint64_t(K) * 2, 128};
+  const cuuint64_t strides[2] = {cuuint64_t(ldx) * 2, 128};
   const cuuint32_t box[3] = {64, cuuint32_t(rows), cuuint32_t(chunks)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box,
@@ -212,6 +213,41 @@ constexpr int64_t kMaxM = int64_t(1) << 26;
 int64_t n_slabs(int64_t N) { return (N + 127) / 128; }
 size_t packed_size(int64_t N, int64_t K) { return size_t(n_slabs(N)) * 128 * size_t(K) / 4; }
 
+// One problem with its row strides in elements: x rows ldx apart, y (and the
+// residual) rows ldy apart.  The dense entry points pass ldx = K, ldy = N.
+struct LinArgs : tern_linear_args {
+  int64_t ldx = 0, ldy = 0;
+};
+LinArgs dense_args(const tern_linear_args& a) {
+  LinArgs l;
+  static_cast<tern_linear_args&>(l) = a;
+  l.ldx = a.K;
+  l.ldy = a.N;
+  return l;
+}
+
+// Whether two row-strided byte regions (rows, bytes per row, bytes between
+// rows) share a byte.  Exact when the strides are equal (two views of one
+// parent tensor, e.g. column slices of a concatenation buffer); otherwise
+// any intersection of their spans counts.
+bool regions_overlap(const void* a, int64_t ra, size_t wa, size_t lda, const void* b, int64_t rb, size_t wb,
+                     size_t ldb) {
+  if (!a || !b || ra <= 0 || rb <= 0 || wa == 0 || wb == 0) return false;
+  const size_t na = size_t(ra - 1) * lda + wa, nb = size_t(rb - 1) * ldb + wb;
+  if (!overlaps(a, na, b, nb)) return false;
+  if (lda != ldb || ra == 1 || rb == 1) return true;  // conservative
+  uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  if (pa > pb) {
+    std::swap(pa, pb);
+    std::swap(ra, rb);
+    std::swap(wa, wb);
+  }
+  const size_t d = size_t(pb - pa), q = d / lda, rem = d % lda;
+  // b's row r starts in a's row q + r at byte rem and may run into row q + r + 1.
+  if (rem < wa && int64_t(q) < ra) return true;
+  return rem + wb > lda && int64_t(q) + 1 < ra;
+}
+
 tern_status check_nk(int64_t N, int64_t K) {
   if (N < 0 || K < 0) return fail(TERN_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
   if (N == 0 || K == 0 || N % 16 != 0 || K % 64 != 0)
@@ -222,21 +258,26 @@ tern_status check_nk(int64_t N, int64_t K) {
   return TERN_OK;
 }
 
-tern_status check_linear(const tern_linear_args& a) {
+tern_status check_linear(const LinArgs& a) {
   tern_status s = check_nk(a.N, a.K);
   if (s != TERN_OK) return s;
   if (a.M < 0) return fail(TERN_ERR_INVALID_ARG, "negative M=%lld", (long long)a.M);
   if (a.M > kMaxM) return fail(TERN_ERR_UNSUPPORTED_SHAPE, "M above 2^26 (M=%lld)", (long long)a.M);
+  if (a.ldx < a.K || a.ldy < a.N || a.ldx % 8 != 0 || a.ldy % 8 != 0 || a.ldx > (int64_t(1) << 30) ||
+      a.ldy > (int64_t(1) << 30))
+    return fail(TERN_ERR_INVALID_ARG, "row strides need ldx >= K, ldy >= N, both multiples of 8 and <= 2^30 "
+                "(ldx=%lld K=%lld ldy=%lld N=%lld)", (long long)a.ldx, (long long)a.K, (long long)a.ldy,
+                (long long)a.N);
   if (!a.packed || !a.scales || (a.M > 0 && (!a.x || !a.y)))
     return fail(TERN_ERR_INVALID_ARG, "null x, packed, scales or y");
   if (!aligned(a.x, 16) || !aligned(a.packed, 16) || !aligned(a.y, 16) || !aligned(a.scales, 4) ||
       (a.bias && !aligned(a.bias, 2)))
     return fail(TERN_ERR_MISALIGNED, "x, packed and y need 16-byte, scales 4-byte, bias 2-byte alignment");
-  const size_t ybytes = size_t(a.M) * size_t(a.N) * 2;
-  if (overlaps(a.y, ybytes, a.x, size_t(a.M) * size_t(a.K) * 2) ||
-      overlaps(a.y, ybytes, a.packed, packed_size(a.N, a.K)) ||
-      overlaps(a.y, ybytes, a.scales, size_t(a.N) * 4) ||
-      overlaps(a.y, ybytes, a.bias, a.bias ? size_t(a.N) * 2 : 0))
+  const size_t yw = size_t(a.N) * 2, yld = size_t(a.ldy) * 2;
+  if (regions_overlap(a.y, a.M, yw, yld, a.x, a.M, size_t(a.K) * 2, size_t(a.ldx) * 2) ||
+      regions_overlap(a.y, a.M, yw, yld, a.packed, 1, packed_size(a.N, a.K), packed_size(a.N, a.K)) ||
+      regions_overlap(a.y, a.M, yw, yld, a.scales, 1, size_t(a.N) * 4, size_t(a.N) * 4) ||
+      regions_overlap(a.y, a.M, yw, yld, a.bias, a.bias ? 1 : 0, size_t(a.N) * 2, size_t(a.N) * 2))
     return fail(TERN_ERR_INVALID_ARG, "y overlaps an input");
   return TERN_OK;
 }
@@ -245,19 +286,21 @@ static_assert(kActNone == TERN_ACT_NONE && kActGeluTanh == TERN_ACT_GELU_TANH, "
 
 // (The epilogue of one problem is a tern_epilogue; all zero is the plain layer.)
 
-tern_status check_epilogue(const tern_epilogue& e, const tern_linear_args& a) {
+tern_status check_epilogue(const tern_epilogue& e, const LinArgs& a) {
   if (e.act != TERN_ACT_NONE && e.act != TERN_ACT_GELU_TANH)
     return fail(TERN_ERR_INVALID_ARG, "unknown activation %d", e.act);
   if (e.act_col0 < 0 || e.act_col0 > a.N)
     return fail(TERN_ERR_INVALID_ARG, "act_col0=%lld outside [0, N=%lld]", (long long)e.act_col0, (long long)a.N);
   if (!aligned(e.residual, 2) || !aligned(e.gate, 2))
     return fail(TERN_ERR_MISALIGNED, "residual and gate need 2-byte alignment");
-  const size_t ybytes = size_t(a.M) * size_t(a.N) * 2;
-  // The residual may be y itself (an in-place update: each element is read
-  // before the same thread writes it); any other overlap with y would race.
-  if (e.residual && e.residual != a.y && overlaps(e.residual, ybytes, a.y, ybytes))
+  const size_t yw = size_t(a.N) * 2, yld = size_t(a.ldy) * 2;
+  // The residual has y's layout (rows ldy apart) and may be y itself (an
+  // in-place update: each element is read before the same thread writes
+  // it); any other overlap with y would race.
+  if (e.residual && e.residual != a.y && regions_overlap(e.residual, a.M, yw, yld, a.y, a.M, yw, yld))
     return fail(TERN_ERR_INVALID_ARG, "residual overlaps y without being y");
-  if (overlaps(e.gate, e.gate ? size_t(a.N) * 2 : 0, a.y, ybytes)) return fail(TERN_ERR_INVALID_ARG, "gate overlaps y");
+  if (regions_overlap(e.gate, e.gate ? 1 : 0, yw, yw, a.y, a.M, yw, yld))
+    return fail(TERN_ERR_INVALID_ARG, "gate overlaps y");
   if (e.norm_col0 < 0 || e.norm_col1 < e.norm_col0 || e.norm_col1 > a.N || e.norm_col0 % 128 || e.norm_col1 % 128)
     return fail(TERN_ERR_INVALID_ARG, "norm columns [%lld, %lld) must be 128-aligned within [0, N=%lld]",
                 (long long)e.norm_col0, (long long)e.norm_col1, (long long)a.N);
@@ -265,7 +308,7 @@ tern_status check_epilogue(const tern_epilogue& e, const tern_linear_args& a) {
     if (!(e.norm_eps > 0.f) || !std::isfinite(e.norm_eps))
       return fail(TERN_ERR_INVALID_ARG, "norm_eps must be finite and > 0");
     if (!aligned(e.norm_weight, 2)) return fail(TERN_ERR_MISALIGNED, "norm_weight needs 2-byte alignment");
-    if (overlaps(e.norm_weight, e.norm_weight ? size_t(a.N) * 2 : 0, a.y, ybytes))
+    if (regions_overlap(e.norm_weight, e.norm_weight ? 1 : 0, yw, yw, a.y, a.M, yw, yld))
       return fail(TERN_ERR_INVALID_ARG, "norm_weight overlaps y");
   }
   return TERN_OK;
@@ -307,10 +350,10 @@ int pick_tok(int64_t M) {
 }
 
 // Fills everything of a Problem except unit_begin; returns its CTA count.
-tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, Problem* p,
+tern_status fill_problem(const LinArgs& a, int tok, int splits_wanted, Problem* p,
                          int64_t* ctas) {
   std::memset(static_cast<void*>(p), 0, sizeof(Problem));
-  tern_status s = make_x_map(&p->tmap_x, a.x, a.M, a.K, tok);
+  tern_status s = make_x_map(&p->tmap_x, a.x, a.M, a.K, a.ldx, tok);
   if (s != TERN_OK) return s;
   p->packed = static_cast<const uint8_t*>(a.packed);
   p->scales = a.scales;
@@ -319,6 +362,7 @@ tern_status fill_problem(const tern_linear_args& a, int tok, int splits_wanted, 
   p->M = int(a.M);
   p->N = int(a.N);
   p->K = int(a.K);
+  p->ldy = int(a.ldy);
   p->n_tiles = int(n_slabs(a.N));
   p->m_tiles = int((a.M + tok - 1) / tok);
   const int kc_total = int(a.K / 64);
@@ -345,10 +389,10 @@ int pair_tok(const tern_linear_args& a, const DeviceState* ds) {
 bool tok_is_pair(int tok) { return tok == 256; }
 
 // Fills a Problem for the pair-tile kernel except unit_begin; returns its tiles.
-tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int64_t* tiles) {
+tern_status fill_problem_2sm(const LinArgs& a, int tok, Problem* p, int64_t* tiles) {
   std::memset(static_cast<void*>(p), 0, sizeof(Problem));
   const bool pair = tok_is_pair(tok);
-  tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, pair ? tok / 2 : tok, 2);
+  tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, a.ldx, pair ? tok / 2 : tok, 2);
   if (s != TERN_OK) return s;
   p->packed = static_cast<const uint8_t*>(a.packed);
   p->scales = a.scales;
@@ -357,6 +401,7 @@ tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int
   p->M = int(a.M);
   p->N = int(a.N);
   p->K = int(a.K);
+  p->ldy = int(a.ldy);
   p->n_tiles = int(a.N / (pair ? 256 : 128));
   p->m_tiles = int((a.M + tok - 1) / tok);
   p->splits = 1;
@@ -368,7 +413,7 @@ tern_status fill_problem_2sm(const tern_linear_args& a, int tok, Problem* p, int
 
 // Launches the problems `idx` of `args` (all with pair_tok == tok) on the
 // pair-tile kernel, up to kMaxProblems per launch.
-tern_status launch_2sm_group(const tern_linear_args* args, const tern_epilogue* epis, const std::vector<int>& idx, int tok,
+tern_status launch_2sm_group(const LinArgs* args, const tern_epilogue* epis, const std::vector<int>& idx, int tok,
                              Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
@@ -398,7 +443,7 @@ tern_status launch_2sm_group(const tern_linear_args* args, const tern_epilogue* 
 // Launches the problems `idx` of `args` (all with M <= 8 nt) on the GEMV
 // kernel, up to kMaxProblems per launch.  K is split over a cluster of up to
 // eight CTAs when the launch has fewer 128-channel slabs than the GPU has SMs.
-tern_status launch_gemv_group(const tern_linear_args* args, const tern_epilogue* epis, const std::vector<int>& idx, int nt,
+tern_status launch_gemv_group(const LinArgs* args, const tern_epilogue* epis, const std::vector<int>& idx, int nt,
                               Batch& batch, const DeviceState* ds, cudaStream_t cs) {
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
@@ -406,9 +451,9 @@ tern_status launch_gemv_group(const tern_linear_args* args, const tern_epilogue*
     int64_t min_chunks = int64_t(1) << 40;
     int n = 0;
     for (size_t g = g0; g < idx.size() && n < kMaxProblems; ++g, ++n) {
-      const tern_linear_args& a = args[idx[g]];
+      const LinArgs& a = args[idx[g]];
       Problem* p = &batch.p[n];
-      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, 8 * nt, nt == 1 ? 16 : 8);
+      tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, a.ldx, 8 * nt, nt == 1 ? 16 : 8);
       if (s != TERN_OK) return s;
       p->packed = static_cast<const uint8_t*>(a.packed);
       p->scales = a.scales;
@@ -417,6 +462,7 @@ tern_status launch_gemv_group(const tern_linear_args* args, const tern_epilogue*
       p->M = int(a.M);
       p->N = int(a.N);
       p->K = int(a.K);
+      p->ldy = int(a.ldy);
       p->n_tiles = int(n_slabs(a.N));
       p->m_tiles = 1;
       set_epilogue(p, epis, idx[g]);
@@ -530,7 +576,7 @@ tern_status tern_adaln_modulate(const void* x, int64_t M, int64_t K, const void*
 namespace tern {
 namespace {
 
-tern_status linear_impl(const tern_linear_args& a, const tern_epilogue& epi, tern_stream_t stream) {
+tern_status linear_impl(const LinArgs& a, const tern_epilogue& epi, tern_stream_t stream) {
   const int64_t M = a.M, N = a.N, K = a.K;
   tern_status s = check_linear(a);
   if (s != TERN_OK) return s;
@@ -580,7 +626,7 @@ tern_status linear_impl(const tern_linear_args& a, const tern_epilogue& epi, ter
   return TERN_OK;
 }
 
-tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, int count, tern_stream_t stream) {
+tern_status batch_impl(const LinArgs* args, const tern_epilogue* epis, int count, tern_stream_t stream) {
   for (int i = 0; i < count; ++i) {
     tern_status s = check_linear(args[i]);
     if (s == TERN_OK && epis) s = check_epilogue(epis[i], args[i]);
@@ -594,20 +640,25 @@ tern_status batch_impl(const tern_linear_args* args, const tern_epilogue* epis, 
   // Problems of one launch run concurrently: no problem's y may overlap any
   // buffer of another problem (its inputs, its residual or its y).
   for (int i = 0; i < count; ++i) {
-    const tern_linear_args& a = args[i];
+    const LinArgs& a = args[i];
     if (a.M == 0) continue;
-    const size_t ya = size_t(a.M) * size_t(a.N) * 2;
+    const size_t wa = size_t(a.N) * 2, lda = size_t(a.ldy) * 2;
     for (int j = 0; j < count; ++j) {
-      const tern_linear_args& b = args[j];
+      const LinArgs& b = args[j];
       if (j == i || b.M == 0) continue;
-      const size_t yb = size_t(b.M) * size_t(b.N) * 2;
+      const size_t wb = size_t(b.N) * 2, ldb = size_t(b.ldy) * 2;
       const void* res = epis ? epis[j].residual : nullptr;
       const void* gate = epis ? epis[j].gate : nullptr;
       const void* nw = epis ? epis[j].norm_weight : nullptr;
-      if (overlaps(a.y, ya, b.y, yb) || overlaps(a.y, ya, b.x, size_t(b.M) * size_t(b.K) * 2) ||
-          overlaps(a.y, ya, b.packed, packed_size(b.N, b.K)) || overlaps(a.y, ya, b.scales, size_t(b.N) * 4) ||
-          overlaps(a.y, ya, b.bias, b.bias ? size_t(b.N) * 2 : 0) || overlaps(a.y, ya, res, res ? yb : 0) ||
-          overlaps(a.y, ya, gate, gate ? size_t(b.N) * 2 : 0) || overlaps(a.y, ya, nw, nw ? size_t(b.N) * 2 : 0))
+      const size_t pb = packed_size(b.N, b.K);
+      if (regions_overlap(a.y, a.M, wa, lda, b.y, b.M, wb, ldb) ||
+          regions_overlap(a.y, a.M, wa, lda, b.x, b.M, size_t(b.K) * 2, size_t(b.ldx) * 2) ||
+          regions_overlap(a.y, a.M, wa, lda, b.packed, 1, pb, pb) ||
+          regions_overlap(a.y, a.M, wa, lda, b.scales, 1, size_t(b.N) * 4, size_t(b.N) * 4) ||
+          regions_overlap(a.y, a.M, wa, lda, b.bias, b.bias ? 1 : 0, wb, wb) ||
+          regions_overlap(a.y, a.M, wa, lda, res, res ? b.M : 0, wb, ldb) ||
+          regions_overlap(a.y, a.M, wa, lda, gate, gate ? 1 : 0, wb, wb) ||
+          regions_overlap(a.y, a.M, wa, lda, nw, nw ? 1 : 0, wb, wb))
         return fail(TERN_ERR_INVALID_ARG, "problem %d's y overlaps a buffer of problem %d", i, j);
     }
   }
@@ -672,7 +723,8 @@ extern "C" {
 tern_status tern_linear(const void* x_bf16, int64_t M, int64_t K, const void* packed,
                         const float* scales, const void* bias_bf16, int64_t N, void* y_bf16,
                         tern_stream_t stream) {
-  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, tern_epilogue{}, stream);
+  return linear_impl(dense_args(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}), tern_epilogue{},
+                     stream);
 }
 
 tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, const void* packed,
@@ -681,20 +733,22 @@ tern_status tern_linear_act(const void* x_bf16, int64_t M, int64_t K, const void
   tern_epilogue spec{};
   spec.act = act;
   spec.act_col0 = act_col0;
-  return linear_impl(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}, spec, stream);
+  return linear_impl(dense_args(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K}), spec, stream);
 }
 
 tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream) {
   if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
-  return batch_impl(args, nullptr, count, stream);
+  std::vector<LinArgs> lin(size_t(std::max(count, 0)));
+  for (int i = 0; i < count; ++i) lin[i] = dense_args(args[i]);
+  return batch_impl(lin.data(), nullptr, count, stream);
 }
 
 tern_status tern_linear_batch_act(const tern_linear_act_args* args, int count, tern_stream_t stream) {
   if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
-  std::vector<tern_linear_args> lin(size_t(std::max(count, 0)));
+  std::vector<LinArgs> lin(size_t(std::max(count, 0)));
   std::vector<tern_epilogue> epis(size_t(std::max(count, 0)));
   for (int i = 0; i < count; ++i) {
-    lin[i] = args[i].linear;
+    lin[i] = dense_args(args[i].linear);
     epis[i] = tern_epilogue{};
     epis[i].act = args[i].act;
     epis[i].act_col0 = args[i].act_col0;
@@ -704,13 +758,38 @@ tern_status tern_linear_batch_act(const tern_linear_act_args* args, int count, t
 
 tern_status tern_linear_epilogue(const tern_linear_args* args, const tern_epilogue* epilogue, tern_stream_t stream) {
   if (!args) return fail(TERN_ERR_INVALID_ARG, "null args");
-  return linear_impl(*args, epilogue ? *epilogue : tern_epilogue{}, stream);
+  return linear_impl(dense_args(*args), epilogue ? *epilogue : tern_epilogue{}, stream);
 }
 
 tern_status tern_linear_batch_epilogue(const tern_linear_args* args, const tern_epilogue* epilogues, int count,
                                        tern_stream_t stream) {
   if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
-  return batch_impl(args, epilogues, count, stream);
+  std::vector<LinArgs> lin(size_t(std::max(count, 0)));
+  for (int i = 0; i < count; ++i) lin[i] = dense_args(args[i]);
+  return batch_impl(lin.data(), epilogues, count, stream);
+}
+
+namespace {
+LinArgs strided_args(const tern_linear_strided_args& a) {
+  LinArgs l = dense_args(a.linear);
+  l.ldx = a.ldx;
+  l.ldy = a.ldy;
+  return l;
+}
+}  // namespace
+
+tern_status tern_linear_strided(const tern_linear_strided_args* args, const tern_epilogue* epilogue,
+                                tern_stream_t stream) {
+  if (!args) return fail(TERN_ERR_INVALID_ARG, "null args");
+  return linear_impl(strided_args(*args), epilogue ? *epilogue : tern_epilogue{}, stream);
+}
+
+tern_status tern_linear_batch_strided(const tern_linear_strided_args* args, const tern_epilogue* epilogues,
+                                      int count, tern_stream_t stream) {
+  if (count < 0 || (count > 0 && !args)) return fail(TERN_ERR_INVALID_ARG, "bad count or null args");
+  std::vector<LinArgs> lin(size_t(std::max(count, 0)));
+  for (int i = 0; i < count; ++i) lin[i] = strided_args(args[i]);
+  return batch_impl(lin.data(), epilogues, count, stream);
 }
 
 tern_status tern_dequantize(const void* packed, const float* scales, int64_t N, int64_t K,
@@ -792,6 +871,7 @@ tern_status tern_linear_e4m3(const void* xq, const float* a, int64_t M, int64_t 
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
+  p.ldy = int(N);
   p.n_tiles = int(N / 256);
   p.m_tiles = int((M + 255) / 256);
   p.splits = 1;
@@ -911,7 +991,7 @@ tern_status noalloc_scratch(int dev, unsigned char** out) {
 extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* packed,
                                            const float* scales, const void* bias_bf16, int64_t N,
                                            void* y_bf16, tern_stream_t stream) {
-  const tern_linear_args a{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K};
+  const LinArgs a = dense_args(tern_linear_args{x_bf16, packed, scales, bias_bf16, y_bf16, M, N, K});
   tern_status s = check_linear(a);
   if (s != TERN_OK) return s;
   if (M == 0) return TERN_OK;

@@ -487,12 +487,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(accempty_leader);  // the next tile's MMAs may start
-      uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+      uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
 #pragma unroll
       for (int c = 0; c < kCols; ++c) {
         const float am = __shfl_sync(0xffffffffu, c < 32 ? alo : ahi, c & 31);
         const float y = fmaf(f[c], sc * am, bi);
-        if (c < rows) yp[size_t(c) * P.N] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+        if (c < rows) yp[size_t(c) * P.ldy] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
       }
     }
   }

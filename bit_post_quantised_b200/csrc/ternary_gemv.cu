@@ -96,6 +96,7 @@ struct GemvProb {
   __nv_bfloat16* y;
   int unit_begin, M, N, K, chunks_per_split;
   int act, act_col0;  // epilogue activation and its first column
+  int ldy;            // elements between rows of y and of the residual
   const uint16_t* residual;  // [M, N] or null
   const uint16_t* gate;      // [N] or null
 };
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
     g.chunks_per_split = q.chunks_per_split;
     g.act = q.act;
     g.act_col0 = q.act_col0;
+    g.ldy = q.ldy;
     g.residual = reinterpret_cast<const uint16_t*>(q.residual);
     g.gate = reinterpret_cast<const uint16_t*>(q.gate);
   }
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int t = 8 * nb + 2 * c + (e & 1);
             const int nn = n_out + (e >> 1) * 8;
-            rv[nb][e] = (P.residual && live && t < P.M) ? bf16_bits_to_float(P.residual[size_t(t) * P.N + nn]) : 0.f;
+            rv[nb][e] = (P.residual && live && t < P.M) ? bf16_bits_to_float(P.residual[size_t(t) * P.ldy + nn]) : 0.f;
           }
 #pragma unroll
         for (int nb = 0; nb < NT; ++nb)
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
             if (live && t < P.M) {
               const float v = fmaf(d[nb][e], e >> 1 ? s1 : s0, e >> 1 ? b1 : b0);
               const float a = apply_act(v, P.act, nn, P.act_col0);
-              P.y[size_t(t) * P.N + nn] = __float2bfloat16_rn(fmaf(e >> 1 ? g1 : g0, a, rv[nb][e]));
+              P.y[size_t(t) * P.ldy + nn] = __float2bfloat16_rn(fmaf(e >> 1 ? g1 : g0, a, rv[nb][e]));
             }
           }
       }

@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
     const int col_end = min(TOK, col_begin + kColsPerHalf);
     const int n = n_tile * 128 + r;
     const int M = P.M, N = P.N;
+    const size_t ld = size_t(P.ldy);  // elements between rows of y and of the residual
     const bool live = n < N;  // channels past N (the last slab's zero-code rows) are not stored
     const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
     if (P.splits == 1) {
@@ -192,12 +193,12 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
         float rv[16];  // residual loads of the group first (it may be y itself)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          rv[j] = (res && live && row0 + c0 + j < M) ? bf16_bits_to_float(res[size_t(row0 + c0 + j) * N + n]) : 0.f;
+          rv[j] = (res && live && row0 + c0 + j < M) ? bf16_bits_to_float(res[size_t(row0 + c0 + j) * ld + n]) : 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = row0 + c0 + j;
           if (live && m < M)
-            P.y[size_t(m) * N + n] = __float2bfloat16_rn(
+            P.y[size_t(m) * ld + n] = __float2bfloat16_rn(
                 fmaf(gt, apply_act(fmaf(__uint_as_float(v[j]), sc, bi), P.act, n, P.act_col0), rv[j]));
         }
       }
@@ -230,8 +231,8 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
             float acc = 0.f;
             for (int sp = 0; sp < P.splits; ++sp)
               acc += __ldcg(P.ws + ((size_t(sp) * tiles + tile) * TOK + c) * 128 + r);
-            P.y[size_t(m) * N + n] = __float2bfloat16_rn(
-                epilogue_value(fmaf(acc, sc, bi), P.act, n, P.act_col0, res, size_t(m) * N + n, gt));
+            P.y[size_t(m) * ld + n] = __float2bfloat16_rn(
+                epilogue_value(fmaf(acc, sc, bi), P.act, n, P.act_col0, res, size_t(m) * ld + n, gt));
           }
         }
         if (dw == 0 && lane == 0) P.counters[tile] = 0;  // ready for the next launch

@@ -415,16 +415,16 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
             const uint32_t bar = smem_u32(&res_bar[ew]);
             const uint32_t dst = smem_base + C::kStages * C::kStageBytes + ew * C::kResWarpBytes;
             // 16-byte aligned: res is, N is a multiple of 128 and n - lane of 32
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(res + size_t(row0) * P.N + (n - lane));
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(res + size_t(row0) * P.ldy + (n - lane));
             if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(rows) * 64u);
             __syncwarp();
-            for (int c = lane; c < rows; c += 32) tma_load_bulk(dst + c * 64, src + size_t(c) * P.N * 2, 64, bar);
+            for (int c = lane; c < rows; c += 32) tma_load_bulk(dst + c * 64, src + size_t(c) * P.ldy * 2, 64, bar);
             staged = true;
           }
         } else if (res) {
           // Otherwise bring the residual rows into L2, so the loads after the
           // release do not wait for HBM.
-          for (int c = 0; c < rows; ++c) prefetch_l2(res + size_t(row0 + c) * P.N + n);
+          for (int c = 0; c < rows; ++c) prefetch_l2(res + size_t(row0 + c) * P.ldy + n);
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accfull_bar[ab]), (lt / AB) & 1, lim, st))) {
@@ -473,8 +473,8 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         // 2(l % 16) + 1 of token 2i + l / 16) for 4-byte stores.
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = min(kCols, P.M - row0);
-        const int ld = P.N;
-        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + (n - lane) + 2 * (lane & 15);
+        const int ld = P.ldy;
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + (n - lane) + 2 * (lane & 15);
         const uint32_t sel = (lane >> 4) ? 0x7632u : 0x5410u;
 #pragma unroll
         for (int i = 0; i < kCols / 2; ++i) {
@@ -522,10 +522,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         }
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = min(kCols, P.M - row0);
-        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
-          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+          if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
       } else if (EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1) {
         // RMS normalisation: the CTA's 128 channels are one group (n - r and
         // the bounds are multiples of 128), so every warp of the CTA takes
@@ -566,9 +566,9 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         ++norm_it;
         if (!__all_sync(0xffffffffu, ok_n)) break;
         const float w = P.norm_weight ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.norm_weight)[n]) : 1.f;
-        const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
+        const int act = P.act, act_col0 = P.act_col0, ld = P.ldy;  // c * ld < 2^28
         const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
-        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const uint16_t* rp = res ? res + size_t(row0) * P.ldy + n : nullptr;
         const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
         uint32_t out[kCols / 2];  // the finished values, bf16x2; stored after the release
 #pragma unroll
@@ -597,10 +597,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
-        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
-          if (c < rows) yp[size_t(c) * P.N] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+          if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
       } else {
         // Residual and gate (with or without the activation): fp32 until the
         // store, everything after the release.
@@ -618,10 +618,10 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = min(kCols, P.M - row0);
-        const int act = P.act, act_col0 = P.act_col0, ld = P.N;  // c * ld < 2^28
-        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.N + n;
+        const int act = P.act, act_col0 = P.act_col0, ld = P.ldy;  // c * ld < 2^28
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
         const uint16_t* res = reinterpret_cast<const uint16_t*>(P.residual);
-        const uint16_t* rp = res ? res + size_t(row0) * P.N + n : nullptr;
+        const uint16_t* rp = res ? res + size_t(row0) * P.ldy + n : nullptr;
         const float gt = P.gate ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.gate)[n]) : 1.f;
 #pragma unroll
         for (int c = 0; c < kCols; ++c) f[c] = apply_act(f[c], act, n, act_col0);

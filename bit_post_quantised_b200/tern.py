@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "TERN_OK", -1: "TERN_ERR_INVALID_ARG", -2: "TERN_ERR_UNSUPPOR
 
 EXPORTED = ("tern_packed_bytes", "tern_quantize_pack", "tern_linear", "tern_linear_noalloc",
             "tern_linear_act", "tern_linear_epilogue", "tern_linear_batch", "tern_linear_batch_act",
-            "tern_linear_batch_epilogue", "tern_adaln_modulate", "tern_quantize_act_e4m3", "tern_linear_e4m3",
+            "tern_linear_batch_epilogue", "tern_linear_strided", "tern_linear_batch_strided",
+            "tern_adaln_modulate", "tern_quantize_act_e4m3", "tern_linear_e4m3",
             "tern_dequantize", "tern_get_device_status", "tern_set_wait_limit_ns",
             "tern_selftest_wait_timeout", "tern_status_string", "tern_last_error")
 
@@ -45,6 +46,11 @@ class LinearArgs(ctypes.Structure):
 class LinearActArgs(ctypes.Structure):
     """Mirror of tern_linear_act_args."""
     _fields_ = [("linear", LinearArgs), ("act", ctypes.c_int), ("act_col0", ctypes.c_int64)]
+
+
+class LinearStridedArgs(ctypes.Structure):
+    """Mirror of tern_linear_strided_args."""
+    _fields_ = [("linear", LinearArgs), ("ldx", ctypes.c_int64), ("ldy", ctypes.c_int64)]
 
 
 class Epilogue(ctypes.Structure):
@@ -89,6 +95,11 @@ def lib() -> ctypes.CDLL:
         L.tern_linear_batch_epilogue.argtypes = [ctypes.POINTER(LinearArgs), ctypes.POINTER(Epilogue), ctypes.c_int,
                                                  vp]
         L.tern_linear_batch_epilogue.restype = st
+        L.tern_linear_strided.argtypes = [ctypes.POINTER(LinearStridedArgs), ctypes.POINTER(Epilogue), vp]
+        L.tern_linear_strided.restype = st
+        L.tern_linear_batch_strided.argtypes = [ctypes.POINTER(LinearStridedArgs), ctypes.POINTER(Epilogue),
+                                                ctypes.c_int, vp]
+        L.tern_linear_batch_strided.restype = st
         L.tern_linear_batch.restype = st
         L.tern_adaln_modulate.argtypes = [vp, i64, i64, vp, vp, i64, i64, ctypes.c_float, vp, vp]
         L.tern_adaln_modulate.restype = st
@@ -298,6 +309,41 @@ def linear_e4m3(xq: torch.Tensor, a: torch.Tensor, packed: torch.Tensor, scales:
     _check(lib().tern_linear_e4m3(_ptr(xq), _ptr(a), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
                                   _stream(stream)))
     return out
+
+
+def _strided_args(p: dict) -> LinearStridedArgs:
+    x, y = p["x"], p["y"]
+    if x.stride(1) != 1 or y.stride(1) != 1:
+        raise ValueError("x and y rows must be contiguous (stride 1 along the last dimension)")
+    M, K = x.shape
+    N = p["scales"].shape[0]
+    lin = LinearArgs(x.data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
+                     None if p.get("bias") is None else p["bias"].data_ptr(), y.data_ptr(), M, N, K)
+    return LinearStridedArgs(lin, x.stride(0), y.stride(0))
+
+
+def linear_strided(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, bias: Optional[torch.Tensor],
+                   out: torch.Tensor, stream=None, **epilogue):
+    """tern_linear_strided: x and out may be row-strided views (for instance
+    column slices of wider tensors); their row strides are passed as ldx and
+    ldy.  Keyword arguments are the epilogue's (act, act_col0, residual,
+    gate, norm_col0, norm_col1, norm_weight, norm_eps); a residual has out's
+    row stride."""
+    a = _strided_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
+    e = _epilogue(epilogue)
+    _check(lib().tern_linear_strided(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
+    return out
+
+
+def linear_batch_strided(problems: Sequence[dict], stream=None) -> None:
+    """tern_linear_batch_strided over dicts as linear_batch_epilogue's, with x
+    and y possibly row-strided views."""
+    n = max(1, len(problems))
+    args, epis = (LinearStridedArgs * n)(), (Epilogue * n)()
+    for i, p in enumerate(problems):
+        args[i] = _strided_args(p)
+        epis[i] = _epilogue(p)
+    _check(lib().tern_linear_batch_strided(args, epis, len(problems), _stream(stream)))
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional[torch.Tensor] = None,

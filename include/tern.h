@@ -240,6 +240,32 @@ TERN_API tern_status tern_linear_batch_epilogue(const tern_linear_args* args, co
  */
 TERN_API tern_status tern_linear_batch(const tern_linear_args* args, int count, tern_stream_t stream);
 
+/*
+ * Row-strided x and y (page "1.58-bit FLUX", Sections 1 and 3.1: the same
+ * ternary layer; strides are this library's interface choice, so that a
+ * linear can read a column slice of a wider activation and write its output
+ * into a slice of a concatenation buffer -- e.g. the attention and MLP parts
+ * of a single FLUX block feeding its output projection -- without a copy).
+ * x[m, k] is at x + m*ldx + k and y[m, n] at y + m*ldy + n (elements); the
+ * residual of an epilogue has y's layout (rows ldy apart; it may be y
+ * itself).  ldx >= K, ldy >= N, both multiples of 8 (16 bytes) and <= 2^30;
+ * x and y 16-byte aligned.  y may share a parent tensor with x or with
+ * another problem's buffers as long as no element is shared: regions with
+ * equal strides are checked element-exactly, regions with different strides
+ * must not intersect at all.  Everything else is as tern_linear_epilogue /
+ * tern_linear_batch_epilogue (ldx = K, ldy = N gives exactly those calls).
+ */
+typedef struct {
+  tern_linear_args linear;
+  int64_t ldx; /* elements between rows of x */
+  int64_t ldy; /* elements between rows of y (and of the residual) */
+} tern_linear_strided_args;
+
+TERN_API tern_status tern_linear_strided(const tern_linear_strided_args* args, const tern_epilogue* epilogue,
+                                         tern_stream_t stream);
+TERN_API tern_status tern_linear_batch_strided(const tern_linear_strided_args* args, const tern_epilogue* epilogues,
+                                               int count, tern_stream_t stream);
+
 /* One problem of tern_linear_batch_act: a linear and its epilogue activation. */
 typedef struct {
   tern_linear_args linear;

@@ -294,3 +294,41 @@ def test_linear_e4m3_rejects_on_host(L):
     assert f(y=F) == INVALID          # y aliases xq
     assert f(y=F + 0x80000) == INVALID  # y aliases a
     assert f(M=0, xq=0, a=0, y=0) == OK
+
+
+PASSES = "passes"  # accepted by every host-side check
+
+
+def _no_gpu() -> bool:
+    return not torch.cuda.is_available()
+
+
+def call_strided(L, x=F, ldx=256, M=16, K=256, packed=F + 0x1000000, scales=F + 0x2000000, bias=None, N=256,
+                 y=F + 0x3000000, ldy=256, residual=None):
+    a = tern.LinearStridedArgs(tern.LinearArgs(x, packed, scales, bias, y, M, N, K), ldx, ldy)
+    e = tern.Epilogue(0, 0, residual, None, 0, 0, None, 0.0)
+    return L.tern_linear_strided(ctypes.byref(a), ctypes.byref(e), None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(ldx=128), INVALID), (dict(ldy=200), INVALID), (dict(ldx=260), INVALID), (dict(ldy=268), INVALID),
+    (dict(ldx=(1 << 30) + 8), INVALID),
+    # y rows interleaved with x rows of one parent tensor (equal strides, disjoint columns): passes the host checks
+    (dict(x=F, y=F + 512, ldx=512, ldy=512, N=256), PASSES),
+    # ... but the columns overlap by one 16-byte group
+    (dict(x=F, y=F + 496, ldx=512, ldy=512, N=256), INVALID),
+    # different strides whose spans intersect: rejected
+    (dict(x=F, y=F + 512, ldx=512, ldy=768, N=256), INVALID),
+    # a residual with y's stride in the other half of each row of y's parent: fine; inside y's columns: not
+    (dict(y=F + 0x3000000, ldy=512, residual=F + 0x3000000 + 512), PASSES),
+    (dict(y=F + 0x3000000, ldy=512, residual=F + 0x3000000 + 256), INVALID),
+])
+def test_strided_linear_checks_on_host(L, kw, expected):
+    if expected == PASSES:
+        # The fake pointers must never reach a launch: only where no GPU can
+        # run one does the call get past the host checks (to the device query).
+        if not _no_gpu():
+            pytest.skip("a call that passes the host checks would launch on this machine's GPU")
+        assert call_strided(L, **kw) in (-4, -6)  # TERN_ERR_CUDA / TERN_ERR_NO_DEVICE from the device query
+    else:
+        assert call_strided(L, **kw) == expected
