@@ -395,6 +395,44 @@ def graph_time(calls, replays, stream):
     return e0.elapsed_time(e1) * 1e-3 / (replays * len(calls))
 
 
+def interleaved_time(call_lists, rounds, stream):
+    """Device time per call of several launch lists, each captured in its own
+    CUDA graph, replayed in turn round after round (median over rounds).
+    Under the power cap the SM clock drifts over tens of milliseconds, so
+    cases timed one after another see different clocks; taking turns gives
+    every case the same mix of them (a fused epilogue is compared with the
+    plain layer this way)."""
+    import statistics
+
+    import torch
+
+    graphs = []
+    for calls in call_lists:
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for c in calls:  # warm-up on the capture stream
+                c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in calls:
+                c()
+        graphs.append(g)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    times = [[] for _ in graphs]
+    for _ in range(rounds):
+        for i, g in enumerate(graphs):
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            times[i].append(e0.elapsed_time(e1) * 1e-3 / len(call_lists[i]))
+    del graphs
+    return [statistics.median(t) for t in times]
+
+
 def cublas_context_us(L, packs, x, b, stream):
     """Dense bf16 cuBLAS (F.linear) on the dequantised weight T*s of the same
     shape, as context: the weight rotates over enough copies (> 3x the 126 MB
@@ -440,20 +478,36 @@ def side_table(device, peaks, stream):
         y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=device)
         calls = [(lambda p=p, s=s: tern.linear(x, p, s, b, out=y)) for p, s in packs]
         reps = max(2, 64 // copies)
-        t = graph_time(calls * reps, 5, stream)
+        fused = None
+        if name == "mlp_up":
+            # FLUX's MLP activation fused into the epilogue
+            fused = [(lambda p=p, s=s: tern.linear_act(x, p, s, b, tern.ACT_GELU_TANH, 0, out=y)) for p, s in packs]
+        elif name == "qkv":
+            # per-head RMS normalisation of q and k (the first 2 * HIDDEN
+            # columns) fused into the epilogue
+            nw = (1 + 0.1 * torch.randn(L.N, device=device)).to(torch.bfloat16)
+            fused = [(lambda p=p, s=s: tern.linear_epilogue(x, p, s, b, norm_cols=(0, 2 * workloads.HIDDEN),
+                                                            norm_weight=nw, norm_eps=1e-6, out=y))
+                     for p, s in packs]
+        if fused is None:
+            t = graph_time(calls * reps, 5, stream)
+        else:
+            t, tf = interleaved_time([calls * (reps // 2 or 1), fused * (reps // 2 or 1)], 8, stream)
         flop_t = 2.0 * L.M * L.N * L.K / peaks["bf16_tflops"] / 1e12
         byte_t = L.algorithmic_bytes / peaks["hbm_gbs"] / 1e9
         entry = {"M": L.M, "N": L.N, "K": L.K, "us": t * 1e6, "tflops": L.flop / t / 1e12,
                  "packed_gbs": L.packed_bytes / t / 1e9, "roofline_frac": max(flop_t, byte_t) / t,
                  "bound": "tensor" if flop_t > byte_t else "hbm"}
         if name == "mlp_up":
-            # FLUX's MLP activation fused into the epilogue, against the HBM
-            # time a separate bf16 GELU pass over y would need (read + write)
-            acts = [(lambda p=p, s=s: tern.linear_act(x, p, s, b, tern.ACT_GELU_TANH, 0, out=y))
-                    for p, s in packs]
-            ta = graph_time(acts * reps, 5, stream)
-            entry["gelu_fused_us"] = ta * 1e6
+            # against the HBM time a separate bf16 GELU pass over y would
+            # need (read + write); plain and fused timed in turns
+            entry["gelu_fused_us"] = tf * 1e6
             entry["gelu_separate_pass_us_at_hbm_peak"] = 2 * 2 * L.M * L.N / peaks["hbm_gbs"] / 1e9 * 1e6
+        elif name == "qkv":
+            # against the HBM time a separate pass over q and k would need
+            entry["qk_norm_fused_us"] = tf * 1e6
+            entry["qk_norm_separate_pass_us_at_hbm_peak"] = (2 * 2 * L.M * 2 * workloads.HIDDEN / peaks["hbm_gbs"]
+                                                              / 1e9 * 1e6)
         entry["cublas_bf16_us"] = cublas_context_us(L, packs, x, b, stream)
         rows[name] = entry
         del packs

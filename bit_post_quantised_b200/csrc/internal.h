@@ -92,10 +92,12 @@ int smem_bytes_for_tok(int tok);
 // (pair, cta_group::2; tok 256 for M > 64) or of 128 channels on single CTAs
 // (!pair; tok 64 for 16 < M <= 64).  Problems use n_tiles = N / (256 or 128),
 // m_tiles = ceil(M / tok), splits = 1 and a 3-D x tensor map {64 k, M,
-// K / 64} whose box is {64, tok / 2 or tok rows, 2 chunks}; ctas_or_pairs
-// work units run at once.
+// K / 64} whose box is {64, tok / 2 or tok rows, x_chunks_2sm(tok) chunks}
+// (the 64-k chunks of one pipeline stage); ctas_or_pairs work units run at
+// once.
 cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream);
 int max_active_clusters_2sm();
+int x_chunks_2sm(int tok);
 // Small-M kernel (M <= 8 nt tokens, nt in {1, 2}), persistent over work
 // units (problem, 128-channel slab): grid (splits, ctas) with clusters of
 // `splits` CTAs along k (splits > 1 needs ctas == total_units); problems use
@@ -103,8 +105,6 @@ int max_active_clusters_2sm();
 // chunks_per_split 64-k chunks per CTA and a 3-D x tensor map {64 k, M,
 // K / 64} whose box is {64, min(M, 8 nt), 16 (nt = 1) or 8 chunks}.
 cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream);
-int max_active_clusters_2sm();
-int smem_bytes_2sm();
 // FP8 (E4M3) activations: per-token absmax quantisation of x (one warp per
 // row, k interleaved inside 16-element groups), and the CTA-pair tile kernel
 // with kind::f8f6f4 MMAs (one problem: N % 256 == 0, tmap_x = the 2-D E4M3 map

@@ -103,6 +103,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// Both phases, as mbar_wait each: the first two polls go out back to back,
+// so when both phases are already complete (the usual case) the wait costs
+// one poll's latency instead of two.
+__device__ __forceinline__ bool mbar_wait_both(uint32_t bar0, uint32_t parity0, uint32_t bar1, uint32_t parity1,
+                                               uint64_t limit_ns, unsigned int* status) {
+  const bool d0 = mbar_try_wait(bar0, parity0);
+  const bool d1 = mbar_try_wait(bar1, parity1);
+  if (d0 && d1) return true;
+  return (d0 || mbar_wait(bar0, parity0, limit_ns, status)) && (d1 || mbar_wait(bar1, parity1, limit_ns, status));
+}
+
 // Asks for the 128-byte line holding `p` to be brought into L2 (no register
 // result, no ordering).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
@@ -385,6 +396,22 @@ __device__ __forceinline__ void mma_stage(uint32_t d, uint32_t a, uint64_t desc,
   else
     asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(2) TERN_COMMIT2("%5") TERN_COMMIT2("%6") "}"
                  ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(bar0), "r"(bar1), "l"(chunk2), "h"(both)
+                 : "memory");
+}
+// The first 128 k of a longer stage: eight MMAs like mma_stage<8>, no
+// commit (the commits after the stage's last block cover them: a commit
+// tracks every tcgen05 op its thread issued before it, and elect.sync picks
+// the same lane of the converged warp each time).
+template <bool PAIR>
+__device__ __forceinline__ void mma_stage_open(uint32_t d, uint32_t a, uint64_t desc, uint32_t idesc, uint32_t acc,
+                                               uint64_t chunk2) {
+  if constexpr (!PAIR)
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(1) TERN_STAGE_HI(1) "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "l"(chunk2)
+                 : "memory");
+  else
+    asm volatile(TERN_STAGE_PROLOGUE TERN_STAGE_LO(2) TERN_STAGE_HI(2) "}"
+                 ::"r"(d), "r"(a), "l"(desc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "l"(chunk2)
                  : "memory");
 }
 #undef TERN_STAGE_PROLOGUE

@@ -6,8 +6,10 @@
 // absmean rule of BitNet b1.58, per output channel n:
 //   s_n = mean_k |W[n,k]| + eps,   T[n,k] = RoundClip(W[n,k] / s_n, -1, +1).
 // With round-to-nearest-even, RoundClip gives +-1 exactly when
-// |W[n,k]| / s_n > 1/2, i.e. |W[n,k]| > s_n / 2; s_n / 2 is exact in fp32, so
-// the kernel decides every code exactly for the fp32 s_n it stores.
+// |W[n,k]| / s_n > 1/2, i.e. |W[n,k]| > s_n / 2.  For a bf16 W that holds
+// exactly when |W| exceeds s_n / 2 truncated to bf16, so the kernel decides
+// every code exactly for the fp32 s_n it stores (two bf16x2 compares per
+// pair of values).
 //
 // One warp owns one row.  It sums |w| over 16-byte loads: eight values in
 // fp32 (a pairwise tree, error <= 3 ulp of the group), the groups in fp64,
@@ -42,15 +44,67 @@ __device__ __forceinline__ float abs_sum8(const uint4& v) {
 
 // Codes of the two bf16 values of a 32-bit word (k in the low half, k + 1 in
 // the high half) at bits 0-1 and 16-17, given the bf16 threshold thr16 =
-// the top 16 bits of the fp32 s/2.  For a bf16 magnitude m (15 bits),
-// m > thr16 exactly when |w| > s/2 (|w| is a bf16; thr16 is s/2 rounded
-// down to bf16).  Per half, 0x8000 + thr16 - m stays in [1, 0xFFFF], so its
+// s/2 truncated to bf16 (the top 16 bits of s/2 halved toward zero in fp32:
+// exact for normal s, and still the truncation for subnormal s, where the
+// halving drops a bit).  For a bf16 magnitude m (15 bits), m > thr16 exactly
+// when |w| > s/2 (|w| is a bf16).  Per half, 0x8000 + thr16 - m stays in [1, 0xFFFF], so its
 // bit 15 is clear exactly when m > thr16, with no borrow into the other half.
 __device__ __forceinline__ uint32_t code_pair(uint32_t w, uint32_t thr_pair) {
   const uint32_t mag = w & 0x7FFF7FFFu;
   const uint32_t nz = (~((thr_pair | 0x80008000u) - mag) >> 15) & 0x00010001u;
   const uint32_t neg = (w >> 15) & 0x00010001u;
   return nz | ((nz & neg) << 1);
+}
+
+// The codes of a lane's eight values (one 16-byte group: k = 8i .. 8i + 7)
+// ORed into their places in the 16-k code word, from two bf16x2 compares per
+// 32-bit word: w > t and w < -t, t = s/2 rounded down to bf16 (thr_pos; thr_neg
+// is -t).  For a bf16 w, w > t exactly when w > s/2 (t <= s/2 < the next bf16
+// above t), so the compares decide every code exactly, like code_pair, with
+// two compares and two LOP3s per word instead of ten integer operations.  A
+// compare writes 0xFFFF into each half where it holds; the code bits of the
+// word's two values go to bits (2p, 2p + 1) of each half, p = the pair's index
+// in the 16-k word, through the masks k1 (0x00010001 << 2p: sign-free bit) and
+// k3 (0x00030003 << 2p: both bits, -1 = 0b11).  Needs t normal (the compare
+// may treat subnormal operands as zero); the caller takes code_pair otherwise.
+__device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_lt_mask(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.lt.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+struct CodeMasks {
+  uint32_t k1[4], k3[4];
+  __device__ __forceinline__ explicit CodeMasks(int j0) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      k1[e] = 0x00010001u << (2 * (j0 + e));
+      k3[e] = 0x00030003u << (2 * (j0 + e));
+    }
+  }
+};
+__device__ __forceinline__ uint32_t group_codes(const uint4& v, uint32_t thr_pos, uint32_t thr_neg,
+                                                const CodeMasks& m) {
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  uint32_t word = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    word |= bf16x2_gt_mask(w4[e], thr_pos) & m.k1[e];
+    word |= bf16x2_lt_mask(w4[e], thr_neg) & m.k3[e];
+  }
+  return word;
+}
+// The same word through code_pair (any threshold).
+__device__ __forceinline__ uint32_t group_codes_int(const uint4& v, uint32_t thr_pair, int j0) {
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  uint32_t word = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) word |= code_pair(w4[e], thr_pair) << (2 * (j0 + e));
+  return word;
 }
 
 // The padding rows n = N .. Np - 1 of the last 128-channel slab (N % 128
@@ -93,19 +147,19 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   const float s = float(acc / double(K) + double(eps));
   if (lane == 0) scales[n] = s;
-  const uint32_t thr16 = __float_as_uint(0.5f * s) >> 16;
+  const uint32_t thr16 = __float_as_uint(__fmul_rz(0.5f, s)) >> 16;  // trunc(s / 2), exact for any s
   const uint32_t thr_pair = thr16 | (thr16 << 16);
+  const bool normal_thr = thr16 >= 0x0080u;  // t is a normal bf16 (uniform over the warp)
 
   // ---- codes
   uint8_t* slab = packed + size_t(n >> 7) * size_t(K >> 6) * 2048 + size_t(n & 127) * 16;
   const int j0 = (lane & 1) * 4;  // pair index of k = 8i inside its 16-k word (i has lane's parity)
+  const CodeMasks cm(j0);
 #pragma unroll
   for (int t = 0; t < NV; ++t) {
     const int i = lane + 32 * t;
-    const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) word |= code_pair(w4[e], thr_pair) << (2 * (j0 + e));
+    uint32_t word = normal_thr ? group_codes(v[t], thr_pair, thr_pair | 0x80008000u, cm)
+                               : group_codes_int(v[t], thr_pair, j0);
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
     if (i < n8 && (i & 1) == 0)
       *reinterpret_cast<uint32_t*>(slab + size_t(i >> 3) * 2048 + ((i & 7) >> 1) * 4) = word;
@@ -140,10 +194,12 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   const float s = float(acc / double(K) + double(eps));
   if (lane == 0) scales[n] = s;
-  const uint32_t thr16 = __float_as_uint(0.5f * s) >> 16;
+  const uint32_t thr16 = __float_as_uint(__fmul_rz(0.5f, s)) >> 16;  // trunc(s / 2), exact for any s
   const uint32_t thr_pair = thr16 | (thr16 << 16);
+  const bool normal_thr = thr16 >= 0x0080u;
   uint8_t* slab = packed + size_t(n >> 7) * size_t(K >> 6) * 2048 + size_t(n & 127) * 16;
   const int j0 = (lane & 1) * 4;
+  const CodeMasks cm(j0);
   for (int base = 0; base < n8; base += 32 * NV) {
     uint4 v[NV];
 #pragma unroll
@@ -154,10 +210,8 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 #pragma unroll
     for (int t = 0; t < NV; ++t) {
       const int i = base + lane + 32 * t;
-      const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) word |= code_pair(w4[e], thr_pair) << (2 * (j0 + e));
+      uint32_t word = normal_thr ? group_codes(v[t], thr_pair, thr_pair | 0x80008000u, cm)
+                                 : group_codes_int(v[t], thr_pair, j0);
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
       if (i < n8 && (i & 1) == 0)
         *reinterpret_cast<uint32_t*>(slab + size_t(i >> 3) * 2048 + ((i & 7) >> 1) * 4) = word;

@@ -392,7 +392,7 @@ bool tok_is_pair(int tok) { return tok == 256; }
 tern_status fill_problem_2sm(const LinArgs& a, int tok, Problem* p, int64_t* tiles) {
   std::memset(static_cast<void*>(p), 0, sizeof(Problem));
   const bool pair = tok_is_pair(tok);
-  tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, a.ldx, pair ? tok / 2 : tok, 2);
+  tern_status s = make_x_map_chunks(&p->tmap_x, a.x, a.M, a.K, a.ldx, pair ? tok / 2 : tok, x_chunks_2sm(tok));
   if (s != TERN_OK) return s;
   p->packed = static_cast<const uint8_t*>(a.packed);
   p->scales = a.scales;
@@ -1029,7 +1029,10 @@ extern "C" tern_status tern_linear_noalloc(const void* x_bf16, int64_t M, int64_
     p.ws = reinterpret_cast<float*>(scratch);
     p.counters = reinterpret_cast<int*>(scratch + kNoAllocPartialBytes);
     // The array keeps whatever the previous call (or a timed-out one) left:
-    // the arrival counters must start at zero.
+    // the arrival counters must start at zero.  The kernel resets each
+    // counter it used, but a launch that failed or timed out may not have;
+    // this clear on every call is what covers that case, so it stays even
+    // though it is redundant after a clean launch.
     cudaError_t e = cudaMemsetAsync(p.counters, 0, size_t(tiles) * sizeof(int), cs);
     if (e != cudaSuccess) return cuda_fail(e, "no-alloc counter clear");
   }

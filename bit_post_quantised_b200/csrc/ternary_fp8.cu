@@ -236,12 +236,6 @@ __device__ __forceinline__ void decode_word_e4m3(uint32_t w, uint32_t* out) {
   out[3] = w & 0xC0C0C0C0u;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
-  uint32_t d;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
 // One lane waits (bounded) and the warp barrier orders the others after it.
 __device__ __forceinline__ bool warp_wait_f8(uint32_t bar, uint32_t parity, uint64_t lim, unsigned int* st,
                                              int lane) {

@@ -38,6 +38,12 @@
 //     then), then y = acc * s + b rounded to bf16 and stored.  A residual
 //     epilogue copies each warp's residual slice into shared memory while
 //     the tile's MMAs run, so after the release it reads shared memory only.
+// The 64-token tiles (16 < M <= 64) run on single CTAs (cta_group::1, 128
+// channels x 64 tokens) with the same roles, eight decoder warps (two
+// groups of four taking alternate stages), eight epilogue warps, two
+// accumulators and 256-k stages (40 KiB, 5 stages, 4 with a residual
+// epilogue; 3 TMEM slots of 128 columns): sixteen MMAs per handshake
+// instead of eight.
 // Work is persistent: cluster c takes tiles c, c + #clusters, ...  No TMA
 // multicast is used: every copy reads this GPU's global memory into the
 // issuing CTA's own shared memory.
@@ -68,15 +74,19 @@ struct Cfg2 {
   static constexpr int kTokCta = PAIR ? TOK / 2 : TOK;  // x rows each CTA loads
   static constexpr int kChCta = 128;              // channels (TMEM lanes) per CTA
   static constexpr int kChTile = PAIR ? 256 : 128;  // channels per tile
-  static constexpr int kBK = 128;                 // k per stage
+  // 64-k chunks per stage.  Every stage costs its handshakes (copy landed,
+  // slot decoded, MMAs done: several hundred cycles, measured) however many
+  // MMAs it feeds, and an N = 64 MMA is short, so the 64-token tiles take
+  // 256 k per stage; the pair tiles' N = 256 MMAs hide them at 128 k.
+  static constexpr int kChunks = TOK >= 256 ? 2 : 4;
+  static constexpr int kBK = 64 * kChunks;        // k per stage
   static constexpr int kXBox = kTokCta * 128;     // one 64 k x kTokCta row box, 128-byte swizzle
-  static constexpr int kXBytes = 2 * kXBox;
+  static constexpr int kXBytes = kChunks * kXBox;
   static constexpr int kCSub = 128 * 16;          // codes of 128 channels x 64 k
-  static constexpr int kCBytes = 2 * kCSub;
+  static constexpr int kCBytes = kChunks * kCSub;
   static constexpr int kStageBytes = kXBytes + kCBytes;
   static constexpr bool kResStaged = EPI == 2;
-  static constexpr int kStages = kStageBytes > 24 * 1024 ? (kResStaged ? 4 : 6) : 8;
-  static constexpr int kASlots = 4;               // decoded-weight slots in TMEM
+  static constexpr int kStages = TOK >= 256 ? (kResStaged ? 4 : 6) : (kResStaged ? 4 : 5);
   static constexpr int kACols = kBK / 2;          // 32-bit TMEM columns per slot (bf16x2)
   static constexpr int kDCols = TOK;              // one accumulator
   // Two accumulators (the epilogue of a tile overlaps the next tile's MMAs)
@@ -84,6 +94,9 @@ struct Cfg2 {
   static constexpr int kAccBufs = TOK >= 256 ? 1 : 2;
   static constexpr int kACol0 = kAccBufs * kDCols;
   static constexpr int kTmemCols = 512;
+  // Decoded-weight slots in TMEM: what the accumulators leave, at most four
+  // (4 x 128 k at N = 256, 3 x 256 k at N = 64).
+  static constexpr int kASlots = (kTmemCols - kACol0) / kACols < 4 ? (kTmemCols - kACol0) / kACols : 4;
   // A narrow tile makes the MMAs of a stage short, so decoding needs more warps.
   static constexpr int kDecWarps = TOK >= 256 ? 4 : 8;
   // Epilogue warps: kEpiWarps / 4 per TMEM lane quarter, each draining
@@ -229,7 +242,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int a = 0; a < A; ++a) {
-      mbar_init(smem_u32(&afull_bar[a]), C::kCtas * C::kDecWarps);
+      mbar_init(smem_u32(&afull_bar[a]), C::kCtas * 4);  // one decoder warp per lane quarter per CTA
       mbar_init(smem_u32(&aempty_bar[a]), 1);
     }
     for (int b = 0; b < AB; ++b) {
@@ -274,16 +287,16 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         const uint8_t* codes =
             t.P->packed + size_t(t.n_tile * C::kCtas + int(rank)) * kc_total * C::kCSub;
         const int row = t.m_tile * C::kTokPair + int(rank) * C::kTokCta;
-        for (int kc = 0; kc < kc_total; kc += 2, ++it) {
+        for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
           if (it % L != lane) continue;
           const int s = it % S;
           ok = mbar_wait(smem_u32(&empty_bar[s]), ((it / S) & 1) ^ 1, lim, st);
           if (!ok) break;
-          const int nsub = min(2, kc_total - kc);
+          const int nsub = min(C::kChunks, kc_total - kc);
           const uint32_t stage = smem_base + s * C::kStageBytes;
           const uint32_t fb = smem_u32(&full_bar[s]);
-          // One 3-D box brings both 64-k chunks of x (the second reads as
-          // zero past K); the codes of the stage are one contiguous block.
+          // One 3-D box brings all 64-k chunks of x of the stage (those past
+          // K read as zero); the codes of the stage are one contiguous block.
           mbar_arrive_expect_tx(fb, C::kXBytes + nsub * C::kCSub);
           tma_load_3d(stage, &t.P->tmap_x, 0, row, kc, fb);
           tma_load_bulk(stage + C::kXBytes, codes + size_t(kc) * C::kCSub, nsub * C::kCSub, fb);
@@ -308,19 +321,33 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_u + ab * C::kDCols;
-        for (int kc = 0; kc < kc_total; kc += 2, ++it) {
+        for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
           const int s = it % S, a = it % A;
           ok = __shfl_sync(0xffffffffu, mbar_wait(smem_u32(&afull_bar[a]), (it / A) & 1, lim, st), 0);
           if (!ok) break;
           tc_fence_after();
           // The whole warp computes the (uniform) operands; one lane issues.
-          const uint32_t a_tmem = tmem_u + C::kACol0 + a * C::kACols;
-          const uint64_t desc = sw128_kmajor_desc(smem_base + s * C::kStageBytes);
+          uint32_t a_tmem = tmem_u + C::kACol0 + a * C::kACols;
+          uint64_t desc = sw128_kmajor_desc(smem_base + s * C::kStageBytes);
           const uint32_t bar0 = smem_u32(&empty_bar[s]), bar1 = smem_u32(&aempty_bar[a]);
-          if (kc + 1 < kc_total)
-            mma_stage<8, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1, uint64_t(C::kXBox >> 4));
+          constexpr uint64_t kChunk2 = uint64_t(C::kXBox >> 4);  // next 64-k chunk of x, 16-byte units
+          int left = kc_total - kc;  // 64-k chunks this stage still holds
+          uint32_t acc = kc != 0;
+          if constexpr (C::kChunks == 4) {
+            // 256-k stage: the first 128 k (when the stage has more) without
+            // a commit, then the rest with the stage's two commits.
+            if (left > 2) {
+              mma_stage_open<PAIR>(d_tmem, a_tmem, desc, C::kIdesc, acc, kChunk2);
+              a_tmem += 64;
+              desc += 2 * kChunk2;
+              acc = 1;
+              left -= 2;
+            }
+          }
+          if (left >= 2)
+            mma_stage<8, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, acc, bar0, bar1, kChunk2);
           else
-            mma_stage<4, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, kc != 0, bar0, bar1, uint64_t(C::kXBox >> 4));
+            mma_stage<4, PAIR>(d_tmem, a_tmem, desc, C::kIdesc, acc, bar0, bar1, kChunk2);
         }
         if (ok) T::commit_all(smem_u32(&accfull_bar[ab]));  // converged warp: the issuing lane
         __syncwarp();
@@ -331,11 +358,16 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     }
   } else if (warp < C::kEpiWarp0) {
     // ------------------------------------------------------ decoders
-    // With four decoder warps each thread expands both 64-k halves of its
-    // row; with eight, warps 2-5 take the first half and warps 6-9 the second.
-    constexpr int kSubs = 8 / C::kDecWarps;  // 64-k halves per decoder warp
+    // Each thread expands every 64-k chunk of its channel row of a stage.
+    // With eight decoder warps, warps 2-5 take the even stages and warps 6-9
+    // the odd ones: a stage's decode is a chain of latencies (two barrier
+    // polls of ~200 cycles each even when the phase is complete, shared
+    // loads, tcgen05.st and its wait), so two stages in flight double the
+    // rate at which slots fill; splitting one stage's chunks over both
+    // groups instead left every stage paying the whole chain.
+    constexpr int kGroups = C::kDecWarps / 4;
+    const int group = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may touch
-    const int sub0 = kSubs == 2 ? 0 : (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t afull_leader0 = T::leader_addr(smem_u32(&afull_bar[0]));
@@ -343,18 +375,17 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
     bool ok = true;
     for (int u = u0; u < units && ok; u += ustep) {
       const int kc_total = tile_of(batch, u).P->K >> 6;
-      for (int kc = 0; kc < kc_total; kc += 2, ++it) {
+      for (int kc = 0; kc < kc_total; kc += C::kChunks, ++it) {
+        if (kGroups > 1 && it % kGroups != group) continue;
         const int s = it % S, a = it % A;
-        bool got = mbar_wait(smem_u32(&full_bar[s]), (it / S) & 1, lim, st);
-        got = got && mbar_wait(smem_u32(&aempty_bar[a]), ((it / A) & 1) ^ 1, lim, st);
-        ok = __all_sync(0xffffffffu, got);
+        ok = __all_sync(0xffffffffu, mbar_wait_both(smem_u32(&full_bar[s]), (it / S) & 1, smem_u32(&aempty_bar[a]),
+                                                    ((it / A) & 1) ^ 1, lim, st));
         if (!ok) break;
         tc_fence_after();
         const uint8_t* cp = smem_gen + s * C::kStageBytes + C::kXBytes + r * 16;
         const uint32_t dst = tmem + lane_off + C::kACol0 + a * C::kACols;
 #pragma unroll
-        for (int h = 0; h < kSubs; ++h) {
-          const int sub = sub0 + h;
+        for (int sub = 0; sub < C::kChunks; ++sub) {
           if (kc + sub < kc_total) {
             uint32_t t[32];
             const uint4 v = *reinterpret_cast<const uint4*>(cp + sub * C::kCSub);
@@ -390,8 +421,18 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
       const int n = t.n_tile * C::kChTile + int(rank) * C::kChCta + r;
       const float sc = 0.5f * P.scales[n];  // A held 2t
       const float bi = P.bias ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.bias)[n]) : 0.f;
-      bool plain = true;  // the same for the whole problem
-      if constexpr (EPI > 0) plain = P.act == kActNone && !P.residual && !P.gate && P.norm_col0 == P.norm_col1;
+      // Per tile (the same for every warp of the CTA): a tile whose 128
+      // channels get no epilogue step (no residual or gate, no activation
+      // or normalisation on them: the v columns of a QKV with q/k norm, the
+      // attention columns of a single block's fused projection) takes the
+      // plain epilogue, and one with only an activation the activation
+      // epilogue, whatever else the launch carries.
+      bool plain = true, act_only = false;
+      if constexpr (EPI > 0) {
+        const int n0 = n - r;  // the CTA's first channel
+        act_only = !P.residual && !P.gate && !(n0 >= P.norm_col0 && n0 < P.norm_col1);
+        plain = act_only && (P.act == kActNone || n0 + 127 < P.act_col0);
+      }
       // Residual, gate and activation ("early", EPI == 2): this warp's slice
       // of the tile's residual (its 32 channels of kCols tokens, 64 bytes per
       // token) is copied into shared memory while the tile's MMAs run; after
@@ -483,7 +524,7 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
           const int c = 2 * i + (lane >> 4);
           if (c < rows) *reinterpret_cast<uint32_t*>(yp + c * ld) = __byte_perm(a, b, sel);
         }
-      } else if (plain || EPI == 1) {
+      } else if (plain || EPI == 1 || act_only) {
         uint32_t out[kCols / 2];  // bf16x2: tokens (2c, 2c + 1) of this half
         if (plain) {
 #pragma unroll
@@ -526,13 +567,76 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c)
           if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+      } else if (EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1 && !P.residual && !P.gate &&
+                 (P.act == kActNone || n - r + 127 < P.act_col0)) {
+        // RMS normalisation with nothing else on these channels (FLUX's q/k
+        // norm; the CTA's 128 channels are one group and the condition is
+        // the same for every warp of the CTA).  y = acc * s + b is rounded
+        // to bf16 as it leaves TMEM -- as the unfused layer stores q and k in
+        // bf16 and normalises those -- so the accumulator is released after
+        // one read, like the plain epilogue's; the sums of squares of the
+        // rounded values, their exchange across the four lane quarters and
+        // the scaling all run after the release, overlapping the next
+        // tile's MMAs.  Two bf16 roundings: within 3 * 2^-9 relative.
+        uint32_t out[kCols / 2];  // bf16x2: tokens (2i, 2i + 1) of this lane's channel
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + ab * C::kDCols + half * kCols + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            out[c0 / 2 + j] = pack_bf16x2(fmaf(__uint_as_float(v[2 * j]), sc, bi),
+                                          fmaf(__uint_as_float(v[2 * j + 1]), sc, bi));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) T::arrive_leader(accempty_leader0 + ab * 8);
+        const float w = P.norm_weight ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(P.norm_weight)[n]) : 1.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += 32) {
+          float sq[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float lo = __uint_as_float(out[c0 / 2 + j] << 16), hi = __uint_as_float(out[c0 / 2 + j] & 0xFFFF0000u);
+            sq[2 * j] = lo * lo;
+            sq[2 * j + 1] = hi * hi;
+          }
+          warp_reduce_scatter<32>(sq, lane);  // token c0 + lane, this warp's 32 channels
+          norm_part[(half * 4 + quarter) * kCols + c0 + lane] = sq[0];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&norm_bar[2 * half]));
+        bool ok_n = mbar_wait(smem_u32(&norm_bar[2 * half]), norm_it & 1, lim, st);
+        if (quarter == 0 && ok_n)
+          for (int c = lane; c < kCols; c += 32) {
+            const float tot = (norm_part[(half * 4 + 0) * kCols + c] + norm_part[(half * 4 + 1) * kCols + c]) +
+                              (norm_part[(half * 4 + 2) * kCols + c] + norm_part[(half * 4 + 3) * kCols + c]);
+            norm_inv[half * kCols + c] = rsqrtf(tot * (1.0f / 128.0f) + P.norm_eps);
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&norm_bar[2 * half + 1]));
+        ok_n = mbar_wait(smem_u32(&norm_bar[2 * half + 1]), norm_it & 1, lim, st) && ok_n;
+        ++norm_it;
+        if (!__all_sync(0xffffffffu, ok_n)) break;
+#pragma unroll
+        for (int j = 0; j < kCols / 2; ++j) {
+          const float lo = __uint_as_float(out[j] << 16), hi = __uint_as_float(out[j] & 0xFFFF0000u);
+          out[j] = pack_bf16x2(lo * (norm_inv[half * kCols + 2 * j] * w), hi * (norm_inv[half * kCols + 2 * j + 1] * w));
+        }
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
+        uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
+#pragma unroll
+        for (int c = 0; c < kCols; ++c)
+          if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
       } else if (EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1) {
-        // RMS normalisation: the CTA's 128 channels are one group (n - r and
-        // the bounds are multiples of 128), so every warp of the CTA takes
-        // this branch for the tile.  The per-token sums of squares need all
-        // four lane quarters, so the accumulator is held (read twice from
-        // TMEM) until the normalised, activated and combined values are
-        // stored; registers hold 32 columns at a time.
+        // RMS normalisation combined with an activation, a residual or a
+        // gate on the same channels: fp32 throughout with one rounding.  The
+        // per-token sums of squares need all four lane quarters, so the
+        // accumulator is held (read twice from TMEM) until the normalised,
+        // activated and combined values are stored; registers hold 32
+        // columns at a time.
         constexpr int kChunk = 32;
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = min(kCols, P.M - row0);
@@ -653,12 +757,12 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
 
 // Pair tiles run as clusters of two CTAs; single-CTA tiles without clusters.
 template <int TOK, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<TOK, true>::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<TOK, true, EPI>::kThreads, 1)
     ternary_pair_kernel(const __grid_constant__ Batch batch) {
   tile_kernel_body<TOK, true, EPI>(batch);
 }
 template <int TOK, int EPI>
-__global__ void __launch_bounds__(Cfg2<TOK, false>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg2<TOK, false, EPI>::kThreads, 1)
     ternary_tile_kernel(const __grid_constant__ Batch batch) {
   tile_kernel_body<TOK, false, EPI>(batch);
 }
@@ -715,6 +819,8 @@ cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas
   }
   return cudaErrorInvalidValue;
 }
+
+int x_chunks_2sm(int tok) { return tok == 256 ? Cfg2<256, true>::kChunks : Cfg2<64, false>::kChunks; }
 
 int max_active_clusters_2sm() {
   if (configure_tile<256, true, 0>() != cudaSuccess || configure_tile<256, true, 1>() != cudaSuccess ||

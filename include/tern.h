@@ -208,6 +208,11 @@ typedef struct {
    * attention head of FLUX.1's q or k) on columns [norm_col0, norm_col1),
    * both multiples of 128 (equal: none), applied first, to v itself:
    *     v <- v / sqrt(mean over the token's group of v^2 + norm_eps) * norm_weight[n].
+   * Where a normalised group has no activation, residual or gate on its
+   * columns (FLUX.1's q/k norm), v is rounded to bf16 before it is
+   * normalised, as the unfused layer stores q and k in bf16 and normalises
+   * those: two roundings, within 3 * 2^-9 relative; otherwise fp32 and one
+   * rounding as above.
    * Only where the layer runs on the tcgen05 tile kernels (N % 256 == 0 and
    * M > 16); elsewhere a requested normalisation is TERN_ERR_UNSUPPORTED_SHAPE. */
   int64_t norm_col0, norm_col1;

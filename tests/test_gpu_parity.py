@@ -109,6 +109,34 @@ def test_quantize_pack_special_rows():
     assert (T[1] == 1).all()
 
 
+def test_quantize_pack_tiny_thresholds_eps_zero():
+    """eps = 0 and rows of tiny magnitudes, so that s_n / 2 falls below the
+    smallest normal bf16 (the kernel then decides the codes with integer
+    compares instead of bf16 ones), or right at it, or just above; bf16
+    subnormal weights among them.  Codes must equal the oracle's |w| > s_n / 2
+    for the GPU's s_n exactly; s_n as the oracle's mean."""
+    N, K = 128, 192
+    g = torch.Generator().manual_seed(17)
+    W = torch.zeros(N, K)
+    tiny = 2.0 ** -126  # smallest normal fp32 / bf16
+    for n in range(N):
+        mag = tiny * 2.0 ** (n % 12 - 8)  # s/2 from ~2^-135 (subnormal) to ~2^-124
+        W[n] = torch.randn(K, generator=g) * mag
+    W = W.to(torch.bfloat16)
+    packed, scales = tern.quantize_pack(W.cuda(), 0.0)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    Wb = bits(W)
+    s_gpu = scales.cpu().double().numpy()
+    s_ref = oracle.absmean_scales(Wb, 0.0)
+    # fp32 subnormal scales carry fewer digits: one rounding of the fp32 grid
+    assert np.all(np.abs(s_gpu - s_ref) <= 1e-6 * s_ref + 2.0 ** -149)
+    T_gpu, bad = oracle.unpack_tiled(packed.cpu().numpy(), N, K)
+    assert bad == 0
+    assert np.array_equal(T_gpu, oracle.ternarize(Wb, s_gpu))
+    assert (T_gpu != 0).any(axis=1).all()  # every row has codes on both sides of the threshold
+
+
 @pytest.mark.parametrize("N,K", [(9216, 3072), (12288, 3072), (3072, 12288), (21504, 3072), (3072, 15360),
                                  (18432, 3072)])
 def test_quantize_pack_flux_shapes(N, K):
@@ -155,10 +183,13 @@ def test_linear_pair_tiles(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(17, 256, 64), (24, 768, 192), (31, 512, 3072), (32, 256, 448),
-                                   (33, 1280, 320), (48, 256, 128), (64, 2560, 576)])
+                                   (33, 1280, 320), (48, 256, 128), (64, 2560, 576), (40, 512, 256),
+                                   (56, 256, 1280)])
 def test_linear_pair_tiles_narrow(M, N, K):
-    """16 < M <= 64 with N % 256 == 0 runs on CTA pairs with 64-token tiles
-    (double-buffered accumulators, eight decoder warps)."""
+    """16 < M <= 64 with N % 256 == 0 runs the 64-token tcgen05 tiles (one
+    CTA per 128 channels, double-buffered accumulators, eight decoder warps,
+    256-k stages): K covers every tail of a stage (64, 128 and 192 k left)
+    and whole stages."""
     run_linear_case(M, N, K, seed=3 * M + N + K)
 
 

@@ -5,10 +5,12 @@ running under global-mode CUDA graph capture, engines that own all device
 memory in a preplanned arena, latency-critical loops where an allocation could
 synchronise the device).  Its split-K scratch is a static device array of the
 library instead of a workspace allocated on first use.  It must give the same
-y as tern_linear within the parity tolerance of the other tests, on two calls
-in a row (the second one finds the first one's partial sums and counters in
-the shared array), whether this file runs alone in a fresh process or after
-every other test.  This file is named so that pytest collects it last.
+y as tern_linear bit for bit (the same kernels with the same tile and split
+choice; the last CTA of a tile adds the split partial sums in split order),
+on two calls in a row (the second one finds the first one's partial sums and
+counters in the shared array), whether this file runs alone in a fresh
+process or after every other test.  This file is named so that pytest
+collects it last.
 """
 from __future__ import annotations
 
@@ -59,6 +61,7 @@ def test_noalloc_matches_linear_on_two_calls(M, N, K):
         torch.cuda.synchronize()
         assert tern.device_status() == 0
         assert_close(y, y_ref)
+        assert torch.equal(y, y_ref)
 
 
 def test_noalloc_back_to_back_different_shapes():
@@ -71,3 +74,4 @@ def test_noalloc_back_to_back_different_shapes():
     assert tern.device_status() == 0
     for y, r in zip(outs, refs):
         assert_close(y, r)
+        assert torch.equal(y, r)
