@@ -169,6 +169,12 @@ def adaln_modulate(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, ep
         mod_ld = scale.stride(0) if scale.dim() == 2 else K
         if shift.dim() == 2 and shift.stride(0) != mod_ld:
             raise ValueError("scale and shift rows must be the same distance apart")
+    G = -(-M // max(T, 1)) if M else 0
+    for name, t in (("scale", scale), ("shift", shift)):
+        rows = t.shape[0] if t.dim() == 2 else 1
+        if t.shape[-1] < K or (G and (G - 1) * int(mod_ld) + K > (rows - 1) * int(mod_ld) + t.shape[-1]):
+            raise ValueError(f"{name} holds fewer than the {G} modulation rows of {K} values that "
+                             f"{M} rows at {T} tokens per row need")
     if out is None:
         out = torch.empty_like(x)
     _check(lib().tern_adaln_modulate(_ptr(x), M, K, _ptr(scale), _ptr(shift), int(mod_ld), max(T, 1), float(eps),

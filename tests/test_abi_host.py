@@ -332,3 +332,15 @@ def test_strided_linear_checks_on_host(L, kw, expected):
         assert call_strided(L, **kw) in (-4, -6)  # TERN_ERR_CUDA / TERN_ERR_NO_DEVICE from the device query
     else:
         assert call_strided(L, **kw) == expected
+
+
+@pytest.mark.parametrize("T,rows", [(1000, 2), (2303, 2), (4607, 1), (1, 4607)])
+def test_adaln_binding_checks_modulation_rows(T, rows):
+    """The binding refuses scale/shift views with fewer modulation rows than
+    ceil(M / tokens_per_row) before anything reaches the library (the C ABI
+    sees only pointers and cannot).  Host tensors: nothing is launched."""
+    M, K = 4608, 3072
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    mod = torch.zeros(rows, 6 * K, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="modulation rows"):
+        tern.adaln_modulate(x, mod[:, K:2 * K], mod[:, :K], 1e-6, tokens_per_row=T)
