@@ -182,6 +182,15 @@ def adaln_modulate(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, ep
     return out
 
 
+def _dense(*ts) -> None:
+    """The dense entry points take row-major tensors without gaps; a view
+    with a row stride goes through linear_strided / linear_batch_strided."""
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("x, y and residual must be dense row-major here; row-strided views go through "
+                             "linear_strided / linear_batch_strided")
+
+
 def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
            bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None):
     """tern_linear: y = (x . T^T) * s + b, x bf16 [M,K] -> y bf16 [M,N]."""
@@ -189,6 +198,7 @@ def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     N = scales.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _dense(x, out)
     _check(lib().tern_linear(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
                              _stream(stream)))
     return out
@@ -204,6 +214,7 @@ def linear_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     N = scales.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _dense(x, out)
     _check(lib().tern_linear_noalloc(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N,
                                      _ptr(out), _stream(stream)))
     return out
@@ -213,6 +224,7 @@ def linear_batch(problems: Sequence[dict], stream=None) -> None:
     """tern_linear_batch over dicts with keys x, packed, scales, bias (or None), y."""
     arr = (LinearArgs * max(1, len(problems)))()
     for i, p in enumerate(problems):
+        _dense(p["x"], p["y"])
         M, K = p["x"].shape
         N = p["scales"].shape[0]
         arr[i] = LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
@@ -230,6 +242,7 @@ def linear_act(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     N = scales.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _dense(x, out)
     _check(lib().tern_linear_act(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, act, act_col0,
                                  _ptr(out), _stream(stream)))
     return out
@@ -240,6 +253,7 @@ def linear_batch_act(problems: Sequence[dict], stream=None) -> None:
     none) and act_col0 (default 0)."""
     arr = (LinearActArgs * max(1, len(problems)))()
     for i, p in enumerate(problems):
+        _dense(p["x"], p["y"])
         M, K = p["x"].shape
         N = p["scales"].shape[0]
         arr[i] = LinearActArgs(LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
@@ -250,13 +264,16 @@ def linear_batch_act(problems: Sequence[dict], stream=None) -> None:
 
 
 def _linear_args(p: dict) -> LinearArgs:
+    _dense(p["x"], p["y"])
     M, K = p["x"].shape
     N = p["scales"].shape[0]
     return LinearArgs(p["x"].data_ptr(), p["packed"].data_ptr(), p["scales"].data_ptr(),
                       None if p.get("bias") is None else p["bias"].data_ptr(), p["y"].data_ptr(), M, N, K)
 
 
-def _epilogue(p: dict) -> Epilogue:
+def _epilogue(p: dict, strided: bool = False) -> Epilogue:
+    if not strided:
+        _dense(p.get("residual"))
     return Epilogue(p.get("act", ACT_NONE), p.get("act_col0", 0), _ptr(p.get("residual")), _ptr(p.get("gate")),
                     p.get("norm_col0", 0), p.get("norm_col1", 0), _ptr(p.get("norm_weight")),
                     p.get("norm_eps", 0.0))
@@ -336,7 +353,7 @@ def linear_strided(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, 
     gate, norm_col0, norm_col1, norm_weight, norm_eps); a residual has out's
     row stride."""
     a = _strided_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
-    e = _epilogue(epilogue)
+    e = _epilogue(epilogue, strided=True)
     _check(lib().tern_linear_strided(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
     return out
 
@@ -348,7 +365,7 @@ def linear_batch_strided(problems: Sequence[dict], stream=None) -> None:
     args, epis = (LinearStridedArgs * n)(), (Epilogue * n)()
     for i, p in enumerate(problems):
         args[i] = _strided_args(p)
-        epis[i] = _epilogue(p)
+        epis[i] = _epilogue(p, strided=True)
     _check(lib().tern_linear_batch_strided(args, epis, len(problems), _stream(stream)))
 
 
