@@ -562,6 +562,7 @@ def side_table(device, peaks, stream):
                                         "torch_unfused_us": tu * 1e6}
     del xs_, outs_, mod
     rows.update(stack_rows(device, peaks, stream))
+    rows.update(forward_rows(device, peaks, stream))
     return rows
 
 
@@ -640,6 +641,54 @@ def stack_rows(device, peaks, stream):
         "batched_us": t_batch * 1e6, "batched_packed_gbs": mod_bytes / t_batch / 1e9,
         "one_call_each_us": t_each * 1e6, "hbm_frac_batched": mod_bytes / t_batch / 1e9 / peaks["hbm_gbs"]}
     return out
+
+
+def forward_rows(device, peaks, stream):
+    """The blocks of a FLUX.1-shaped forward at 1024x1024 (19 double + 38
+    single, seeded random weights, synthetic activations): every linear
+    ternary through the library with its fused epilogues, attention and
+    rotary embedding from torch; against the same blocks in bf16 with dense
+    weights (T*s) through cuBLAS and torch's unfused operations, the bf16
+    model of the pages' Table 3 comparison.  The two are timed in turns
+    (CUDA events, medians of 3)."""
+    import statistics
+
+    import torch
+
+    from bit_post_quantised_b200 import flux, workloads
+
+    cfg = workloads.FluxConfig()
+    model = flux.TernaryFlux(cfg, device=device)
+    img, txt, vec, ids = (t.to(device) for t in workloads.flux_inputs(cfg))
+    dense = flux.dense_weights(model)
+    runs = {"ternary": lambda: model.forward(img, txt, vec, ids),
+            "dense_bf16": lambda: flux.dense_forward(model, dense, img, txt, vec, ids)}
+    for f in runs.values():
+        f()
+    torch.cuda.synchronize()
+    times = {k: [] for k in runs}
+    for _ in range(3):
+        for k, f in runs.items():
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            e1.synchronize()
+            times[k].append(e0.elapsed_time(e1))
+    fl = flux.forward_flop(cfg)
+    packed = sum(q[n][0].numel() for q in model.blocks.values() for n in q if not n.endswith("norm_w"))
+    dense_b = sum(d[n][0].numel() * 2 for d in dense.values() for n in d if not n.endswith("norm_w"))
+    t_ter, t_den = statistics.median(times["ternary"]), statistics.median(times["dense_bf16"])
+    del dense, model
+    torch.cuda.empty_cache()
+    return {"flux_forward_blocks": {
+        "blocks": f"{cfg.n_double} double + {cfg.n_single} single, {cfg.img_tokens} image + {cfg.txt_tokens} text tokens",
+        "ternary_ms": t_ter, "dense_bf16_ms": t_den, "speedup_vs_dense_bf16": t_den / t_ter,
+        "linear_gflop": fl["linear"] / 1e9, "attention_gflop": fl["attention"] / 1e9,
+        "ternary_tflops": (fl["linear"] + fl["attention"]) / (t_ter * 1e-3) / 1e12,
+        "block_weight_gb_ternary": packed / 1e9, "block_weight_gb_bf16": dense_b / 1e9,
+        "outside": "attention (torch SDPA), rotary embedding, SiLU: torch; all linears: this library"}}
 
 
 def gpu_id_for_smi(local: int) -> str:

@@ -146,3 +146,87 @@ def block_epilogue(name: str, qk_norm: bool = False) -> dict:
     if qk_norm and name.endswith((".qkv", ".qkv_mlp")):
         e["norm_cols"] = (0, 2 * HIDDEN)
     return e
+
+
+# --------------------------------------------------------------------- blocks
+HEAD_DIM = 128
+ROPE_AXES = (16, 56, 56)
+NORM_W_STD = 0.1
+
+
+@dataclasses.dataclass(frozen=True)
+class FluxConfig:
+    """A FLUX.1-shaped transformer: hidden width, MLP width, heads of 128,
+    an image token grid (64 x 64 for a 1024 x 1024 image: 2 x 2 patches of
+    its 128 x 128 latent), text tokens, and the block counts."""
+    hidden: int = HIDDEN
+    mlp: int = MLP
+    img_h: int = 64
+    img_w: int = 64
+    txt_tokens: int = TXT_TOKENS
+    n_double: int = N_DOUBLE
+    n_single: int = N_SINGLE
+    in_channels: int = 64
+    context_dim: int = 4096
+    seed: int = 77
+
+    @property
+    def img_tokens(self) -> int:
+        return self.img_h * self.img_w
+
+    @property
+    def heads(self) -> int:
+        return self.hidden // HEAD_DIM
+
+
+FLUX_SMALL = FluxConfig(hidden=256, mlp=1024, img_h=8, img_w=8, txt_tokens=24, n_double=1, n_single=1,
+                        in_channels=64, context_dim=256)
+
+
+def flux_block_shapes(cfg: FluxConfig, kind: str):
+    """(name, N, K) of every ternary linear of one block, "double" or "single"."""
+    C, F = cfg.hidden, cfg.mlp
+    if kind == "double":
+        out = []
+        for s in ("img", "txt"):
+            out += [(f"{s}.mod", 6 * C, C), (f"{s}.qkv", 3 * C, C), (f"{s}.proj", C, C),
+                    (f"{s}.mlp_up", F, C), (f"{s}.mlp_down", C, F)]
+        return out
+    return [("mod", 3 * C, C), ("linear1", 3 * C + F, C), ("linear2", C, C + F)]
+
+
+def flux_block_weights(cfg: FluxConfig, kind: str, index: int, device=None):
+    """Seeded bf16 parameters of one block: for every ternary linear
+    (W [N, K] ~ N(0, 0.02), b [N] ~ N(0, 0.01)), and the q/k RMS norm weights
+    ([128] ~ 1 + N(0, 0.1); per stream in a double block).  Drawn on
+    `device` (CPU by default) from a generator seeded by the block."""
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed * 1000003 + (0 if kind == "double" else 500) + index)
+
+    def normal(shape, std, mean=0.0):
+        return (torch.randn(shape, generator=gen, device=dev) * std + mean).to(torch.bfloat16)
+
+    p = {}
+    for name, N, K in flux_block_shapes(cfg, kind):
+        p[name] = (normal((N, K), W_STD), normal((N,), B_STD))
+    for s in (("img.", "txt.") if kind == "double" else ("",)):
+        p[s + "q_norm"] = normal((HEAD_DIM,), NORM_W_STD, 1.0)
+        p[s + "k_norm"] = normal((HEAD_DIM,), NORM_W_STD, 1.0)
+    return p
+
+
+def flux_inputs(cfg: FluxConfig, seed: int = 5):
+    """Seeded CPU inputs of the block stack: img [Li, C], txt [Lt, C], vec
+    [1, C] (bf16, N(0, 1)) and the token positions ids [Lt + Li, 3] (text
+    tokens at 0, image token (0, row, column)), text first."""
+    gen = torch.Generator().manual_seed(seed)
+    C = cfg.hidden
+    img = _normal((cfg.img_tokens, C), 1.0, gen)
+    txt = _normal((cfg.txt_tokens, C), 1.0, gen)
+    vec = _normal((1, C), 1.0, gen)
+    ids = torch.zeros(cfg.txt_tokens + cfg.img_tokens, 3)
+    r = torch.arange(cfg.img_h).repeat_interleave(cfg.img_w)
+    c = torch.arange(cfg.img_w).repeat(cfg.img_h)
+    ids[cfg.txt_tokens:, 1] = r.float()
+    ids[cfg.txt_tokens:, 2] = c.float()
+    return img, txt, vec, ids
