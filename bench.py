@@ -646,8 +646,8 @@ def stack_rows(device, peaks, stream):
 def forward_rows(device, peaks, stream):
     """The blocks of a FLUX.1-shaped forward at 1024x1024 (19 double + 38
     single, seeded random weights, synthetic activations): every linear
-    ternary through the library with its fused epilogues, attention and
-    rotary embedding from torch; against the same blocks in bf16 with dense
+    ternary through the library with its fused epilogues (the rotary
+    embedding in the q/k epilogue), attention from torch; against the same blocks in bf16 with dense
     weights (T*s) through cuBLAS and torch's unfused operations, the bf16
     model of the pages' Table 3 comparison.  The two are timed in turns
     (CUDA events, medians of 3)."""
@@ -688,7 +688,8 @@ def forward_rows(device, peaks, stream):
         "linear_gflop": fl["linear"] / 1e9, "attention_gflop": fl["attention"] / 1e9,
         "ternary_tflops": (fl["linear"] + fl["attention"]) / (t_ter * 1e-3) / 1e12,
         "block_weight_gb_ternary": packed / 1e9, "block_weight_gb_bf16": dense_b / 1e9,
-        "outside": "attention (torch SDPA), rotary embedding, SiLU: torch; all linears: this library"}}
+        "outside": "attention (torch SDPA) and SiLU: torch; all linears (with q/k norm and rotary embedding, "
+                   "GELU, gated residual in their epilogues) and the adaLN pass: this library"}}
 
 
 def gpu_id_for_smi(local: int) -> str:

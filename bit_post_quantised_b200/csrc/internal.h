@@ -15,7 +15,11 @@ struct alignas(64) Problem {
   const float* scales;      // [N]
   const __nv_bfloat16* bias;  // [N] or null
   __nv_bfloat16* y;         // [M, N]
-  float* ws;                // split-K partials [splits][tiles][TOK][128] (splits > 1)
+  union {
+    float* ws;              // ternary_mma: split-K partials [splits][tiles][TOK][128] (splits > 1);
+                            // ternary_fp8: the E4M3 row scales a [M]
+    const float* rope;      // ternary_mma2: (cos, sin) per token row and channel pair [M][64][2], or null
+  };
   int* counters;            // one arrival counter per output tile (splits > 1), zero at rest
   int M, N, K;
   int n_tiles, m_tiles, splits;

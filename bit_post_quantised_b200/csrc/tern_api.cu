@@ -311,6 +311,17 @@ tern_status check_epilogue(const tern_epilogue& e, const LinArgs& a) {
     if (regions_overlap(e.norm_weight, e.norm_weight ? 1 : 0, yw, yw, a.y, a.M, yw, yld))
       return fail(TERN_ERR_INVALID_ARG, "norm_weight overlaps y");
   }
+  if (e.rope_cs) {
+    if (e.norm_col0 == e.norm_col1)
+      return fail(TERN_ERR_INVALID_ARG, "the rotary embedding applies to normalised columns: none requested");
+    if (e.residual || e.gate || (e.act != TERN_ACT_NONE && e.act_col0 < e.norm_col1))
+      return fail(TERN_ERR_INVALID_ARG, "the rotary embedding needs no activation, residual or gate on the "
+                                        "normalised columns");
+    if (!aligned(e.rope_cs, 8)) return fail(TERN_ERR_MISALIGNED, "rope_cs needs 8-byte alignment");
+    const size_t rw = 64 * 2 * sizeof(float);
+    if (regions_overlap(e.rope_cs, a.M, rw, rw, a.y, a.M, yw, yld))
+      return fail(TERN_ERR_INVALID_ARG, "rope_cs overlaps y");
+  }
   return TERN_OK;
 }
 
@@ -336,6 +347,10 @@ void set_epilogue(Problem* p, const tern_epilogue* epis, int i) {
   p->norm_col1 = int(epis[i].norm_col1);
   p->norm_eps = epis[i].norm_eps;
   p->norm_weight = static_cast<const __nv_bfloat16*>(epis[i].norm_weight);
+  // Shares its slot with the split-K workspace of the fallback kernel, which
+  // never carries a normalisation (and so never a rotation): set only when
+  // given.
+  if (epis[i].rope_cs) p->rope = epis[i].rope_cs;
 }
 
 // Up to 16 tokens run on the register-fed GEMV kernel, in n8 blocks.

@@ -619,13 +619,29 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         ok_n = mbar_wait(smem_u32(&norm_bar[2 * half + 1]), norm_it & 1, lim, st) && ok_n;
         ++norm_it;
         if (!__all_sync(0xffffffffu, ok_n)) break;
+        const int row0 = t.m_tile * C::kTokPair + half * kCols;
+        const int rows = min(kCols, P.M - row0);
+        // Rotary embedding (the same for the whole problem): channel pair
+        // (2p, 2p + 1) of the group turns by the angle of pair p of its row;
+        // the partner channel is the neighbouring lane.  Even channel:
+        // a cos - b sin, odd: a cos + b sin (b the partner's value).
+        const float2* rcs = reinterpret_cast<const float2*>(P.rope);
+        const int pair = (n & 127) >> 1;
+        const float sgn = (n & 1) ? 1.f : -1.f;
 #pragma unroll
         for (int j = 0; j < kCols / 2; ++j) {
           const float lo = __uint_as_float(out[j] << 16), hi = __uint_as_float(out[j] & 0xFFFF0000u);
-          out[j] = pack_bf16x2(lo * (norm_inv[half * kCols + 2 * j] * w), hi * (norm_inv[half * kCols + 2 * j + 1] * w));
+          float a0 = lo * (norm_inv[half * kCols + 2 * j] * w), a1 = hi * (norm_inv[half * kCols + 2 * j + 1] * w);
+          if (rcs) {
+            const float b0 = __shfl_xor_sync(0xffffffffu, a0, 1), b1 = __shfl_xor_sync(0xffffffffu, a1, 1);
+            const int m0 = row0 + 2 * j;
+            const float2 c0 = m0 < P.M ? __ldg(rcs + size_t(m0) * 64 + pair) : make_float2(1.f, 0.f);
+            const float2 c1 = m0 + 1 < P.M ? __ldg(rcs + size_t(m0 + 1) * 64 + pair) : make_float2(1.f, 0.f);
+            a0 = fmaf(a0, c0.x, sgn * b0 * c0.y);
+            a1 = fmaf(a1, c1.x, sgn * b1 * c1.y);
+          }
+          out[j] = pack_bf16x2(a0, a1);
         }
-        const int row0 = t.m_tile * C::kTokPair + half * kCols;
-        const int rows = min(kCols, P.M - row0);
         uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
 #pragma unroll
         for (int c = 0; c < kCols; ++c)

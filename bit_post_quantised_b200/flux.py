@@ -1,7 +1,7 @@
 """FLUX.1's transformer blocks on the ternary linear layer: every linear of
-both block types runs through the C ABI (batched, with the fused epilogues);
-attention, rotary embedding, SiLU and the unquantised input/output
-projections are torch operations around it.
+both block types runs through the C ABI (batched, with the fused epilogues:
+q/k norm and rotary embedding, GELU, gated residual); attention and SiLU are
+torch operations around it.
 
 Page "1.58-bit FLUX" (arXiv 2412.18653): Section 3.1 quantises every linear
 layer of FLUX.1's double-stream and single-stream blocks, and Table 3
@@ -12,11 +12,11 @@ describe nothing between the linears; the block structure here is FLUX.1's
 together, tanh GELU MLP, gated residual updates).
 
 Per double block: the two streams' QKV projections write into one
-[Lt + Li, 3C] buffer (text rows first) with q and k normalised in the
-epilogue, so attention needs no concatenation; the output projections and
-the MLP's second linears update the residual streams in place through the
-gated-residual epilogue.  Per single block: the fused projection writes
-[q | k | v | GELU(mlp)] (norm and activation in its epilogue); the
+[Lt + Li, 3C] buffer (text rows first) with q and k normalised and rotated
+in the epilogue, so attention needs no concatenation; the output
+projections and the MLP's second linears update the residual streams in
+place through the gated-residual epilogue.  Per single block: the fused projection writes
+[q | k | v | GELU(mlp)] (norm, rotation and activation in its epilogue); the
 attention output overwrites the v columns, so the second linear reads
 [attention | mlp] as one strided view of that buffer.  The adaLN modulation
 vectors of every block depend only on vec: one batch of GEMVs computes them
@@ -64,13 +64,16 @@ def apply_rope(x: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor) -> torch.T
     return torch.stack((a * c - b * s, a * s + b * c), dim=-1).flatten(-2).to(torch.bfloat16)
 
 
-def attention(qkv: torch.Tensor, cos, sin, hidden: int) -> torch.Tensor:
+def attention(qkv: torch.Tensor, hidden: int, cos=None, sin=None) -> torch.Tensor:
     """softmax(q k^T / sqrt(D)) v over all tokens of qkv [L, 3C] (q, k
-    already normalised), q and k rotated first; returns [H, L, D] bf16."""
+    already normalised; rotated here when cos and sin are given, else
+    already rotated); returns [H, L, D] bf16."""
     L = qkv.shape[0]
     H = hidden // HEAD_DIM
-    q = apply_rope(qkv[:, :hidden].view(L, H, HEAD_DIM), cos, sin)
-    k = apply_rope(qkv[:, hidden:2 * hidden].view(L, H, HEAD_DIM), cos, sin)
+    q = qkv[:, :hidden].view(L, H, HEAD_DIM)
+    k = qkv[:, hidden:2 * hidden].view(L, H, HEAD_DIM)
+    if cos is not None:
+        q, k = apply_rope(q, cos, sin), apply_rope(k, cos, sin)
     v = qkv[:, 2 * hidden:3 * hidden].view(L, H, HEAD_DIM)
     o = F.scaled_dot_product_attention(q.transpose(0, 1)[None], k.transpose(0, 1)[None], v.transpose(0, 1)[None])
     return o[0]
@@ -134,8 +137,9 @@ class TernaryFlux:
             tern.linear_batch(probs[g:g + 15], stream=self.stream)
         return outs
 
-    def double_block(self, i: int, img: torch.Tensor, txt: torch.Tensor, mods, cos, sin, buf):
-        """Updates img [Li, C] and txt [Lt, C] in place."""
+    def double_block(self, i: int, img: torch.Tensor, txt: torch.Tensor, mods, cs, buf):
+        """Updates img [Li, C] and txt [Lt, C] in place; cs [Lt + Li, 64, 2]
+        the rotary (cos, sin) of every token row (text first)."""
         C = self.cfg.hidden
         q = self.blocks[("double", i)]
         Lt = txt.shape[0]
@@ -146,9 +150,9 @@ class TernaryFlux:
             xm = buf[s + "xm"]
             tern.adaln_modulate(x, m[:, C:2 * C], m[:, :C], LN_EPS, out=xm, stream=self.stream)
             probs.append(self._lin(q[s + "qkv"], xm, qkv[rows], norm_col0=0, norm_col1=2 * C,
-                                   norm_weight=q[s + "norm_w"], norm_eps=QK_EPS))
+                                   norm_weight=q[s + "norm_w"], norm_eps=QK_EPS, rope_cs=cs[rows]))
         tern.linear_batch_epilogue(probs, stream=self.stream)
-        o = attention(qkv, cos, sin, C)  # [H, L, D]
+        o = attention(qkv, C)  # [H, L, D]; q and k rotated in the epilogue
         att = buf["att"]
         att.view(att.shape[0], -1, HEAD_DIM).copy_(o.transpose(0, 1))
         probs = []
@@ -167,7 +171,7 @@ class TernaryFlux:
                  for s, x in (("img.", img), ("txt.", txt))]
         tern.linear_batch_epilogue(probs, stream=self.stream)
 
-    def single_block(self, i: int, x: torch.Tensor, mods, cos, sin, buf):
+    def single_block(self, i: int, x: torch.Tensor, mods, cs, buf):
         """Updates x [Lt + Li, C] in place."""
         C, Fm = self.cfg.hidden, self.cfg.mlp
         q = self.blocks[("single", i)]
@@ -176,8 +180,8 @@ class TernaryFlux:
         tern.adaln_modulate(x, m[:, C:2 * C], m[:, :C], LN_EPS, out=xm, stream=self.stream)
         tern.linear_batch_epilogue([self._lin(q["linear1"], xm, z, act=tern.ACT_GELU_TANH, act_col0=3 * C,
                                               norm_col0=0, norm_col1=2 * C, norm_weight=q["norm_w"],
-                                              norm_eps=QK_EPS)], stream=self.stream)
-        o = attention(z, cos, sin, C)
+                                              norm_eps=QK_EPS, rope_cs=cs)], stream=self.stream)
+        o = attention(z, C)
         z[:, 2 * C:3 * C].view(z.shape[0], -1, HEAD_DIM).copy_(o.transpose(0, 1))
         packed, scales, b = q["linear2"]
         tern.linear_strided(z[:, 2 * C:], packed, scales, b, x, stream=self.stream, residual=x, gate=m[0, 2 * C:])
@@ -199,6 +203,7 @@ class TernaryFlux:
         ns = cfg.n_single if n_single is None else n_single
         Li, Lt = img.shape[0], txt.shape[0]
         cos, sin = rope_cos_sin(ids.to(self.device))
+        cs = torch.stack([cos, sin], dim=-1).contiguous()  # [L, 64, 2], read by the q/k epilogues
         mods = self.modulations(vec)
         buf = self.buffers(Li, Lt)
         x = torch.empty(Lt + Li, cfg.hidden, dtype=torch.bfloat16, device=self.device)
@@ -206,9 +211,9 @@ class TernaryFlux:
         x[Lt:].copy_(img)
         img_s, txt_s = x[Lt:], x[:Lt]  # the streams live in their rows of x
         for i in range(nd):
-            self.double_block(i, img_s, txt_s, mods, cos, sin, buf)
+            self.double_block(i, img_s, txt_s, mods, cs, buf)
         for i in range(ns):
-            self.single_block(i, x, mods, cos, sin, buf)
+            self.single_block(i, x, mods, cs, buf)
         return x
 
 
@@ -262,7 +267,7 @@ def dense_forward(model: TernaryFlux, dense: Dict, img, txt, vec, ids, n_double=
             t = lin(d[s + "qkv"], modln(streams[s], mods[s][1], mods[s][0]))
             w = d[s + "norm_w"]
             qkv.append(torch.cat([qk_norm(t[:, :C], w[:C]), qk_norm(t[:, C:2 * C], w[C:2 * C]), t[:, 2 * C:]], 1))
-        o = attention(torch.cat(qkv, 0), cos, sin, C).transpose(0, 1).reshape(Lt + Li, C)
+        o = attention(torch.cat(qkv, 0), C, cos, sin).transpose(0, 1).reshape(Lt + Li, C)
         new = []
         for s, a in (("txt.", o[:Lt]), ("img.", o[Lt:])):
             sh1, sc1, g1, sh2, sc2, g2 = mods[s]
@@ -277,7 +282,7 @@ def dense_forward(model: TernaryFlux, dense: Dict, img, txt, vec, ids, n_double=
         t = lin(d["linear1"], modln(x, sc, sh))
         w = d["norm_w"]
         qkv = torch.cat([qk_norm(t[:, :C], w[:C]), qk_norm(t[:, C:2 * C], w[C:2 * C]), t[:, 2 * C:3 * C]], 1)
-        o = attention(qkv, cos, sin, C).transpose(0, 1).reshape(x.shape[0], C)
+        o = attention(qkv, C, cos, sin).transpose(0, 1).reshape(x.shape[0], C)
         x = x + g * lin(d["linear2"], torch.cat([o, F.gelu(t[:, 3 * C:], approximate="tanh")], 1))
     return x
 

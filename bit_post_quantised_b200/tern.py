@@ -57,7 +57,7 @@ class Epilogue(ctypes.Structure):
     """Mirror of tern_epilogue."""
     _fields_ = [("act", ctypes.c_int), ("act_col0", ctypes.c_int64), ("residual", ctypes.c_void_p),
                 ("gate", ctypes.c_void_p), ("norm_col0", ctypes.c_int64), ("norm_col1", ctypes.c_int64),
-                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float), ("rope_cs", ctypes.c_void_p)]
 
 
 ACT_NONE = 0       # tern_act values
@@ -274,33 +274,39 @@ def _linear_args(p: dict) -> LinearArgs:
 def _epilogue(p: dict, strided: bool = False) -> Epilogue:
     if not strided:
         _dense(p.get("residual"))
+    rope = p.get("rope_cs")
+    if rope is not None and (rope.dtype != torch.float32 or not rope.is_contiguous() or rope.shape[-2:] != (64, 2)
+                             or rope.shape[0] < p["y"].shape[0]):
+        raise ValueError("rope_cs must be contiguous fp32 [>= M, 64, 2] (cos, sin) pairs")
     return Epilogue(p.get("act", ACT_NONE), p.get("act_col0", 0), _ptr(p.get("residual")), _ptr(p.get("gate")),
                     p.get("norm_col0", 0), p.get("norm_col1", 0), _ptr(p.get("norm_weight")),
-                    p.get("norm_eps", 0.0))
+                    p.get("norm_eps", 0.0), _ptr(rope))
 
 
 def linear_epilogue(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
                     bias: Optional[torch.Tensor] = None, act: int = ACT_NONE, act_col0: int = 0,
                     residual: Optional[torch.Tensor] = None, gate: Optional[torch.Tensor] = None,
                     norm_cols=(0, 0), norm_weight: Optional[torch.Tensor] = None, norm_eps: float = 0.0,
-                    out: Optional[torch.Tensor] = None, stream=None):
+                    out: Optional[torch.Tensor] = None, stream=None, rope_cs: Optional[torch.Tensor] = None):
     """tern_linear_epilogue: y = residual + gate * act(norm(x . T^T * s + b))
     (see tern_epilogue); `out` may be `residual` itself for an in-place
-    update; norm_cols = (first, end) of the RMS-normalised columns."""
+    update; norm_cols = (first, end) of the RMS-normalised columns; rope_cs
+    fp32 [M, 64, 2] (cos, sin) rotates the normalised columns' channel pairs."""
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
     a = _linear_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
     e = _epilogue(dict(act=act, act_col0=act_col0, residual=residual, gate=gate, norm_col0=norm_cols[0],
-                       norm_col1=norm_cols[1], norm_weight=norm_weight, norm_eps=norm_eps))
+                       norm_col1=norm_cols[1], norm_weight=norm_weight, norm_eps=norm_eps, rope_cs=rope_cs, y=out))
     _check(lib().tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
     return out
 
 
 def linear_batch_epilogue(problems: Sequence[dict], stream=None) -> None:
     """tern_linear_batch_epilogue over dicts as linear_batch's plus the
-    optional keys act, act_col0, residual and gate."""
+    optional keys act, act_col0, residual, gate, norm_col0, norm_col1,
+    norm_weight, norm_eps and rope_cs."""
     n = max(1, len(problems))
     args, epis = (LinearArgs * n)(), (Epilogue * n)()
     for i, p in enumerate(problems):
@@ -353,7 +359,7 @@ def linear_strided(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, 
     gate, norm_col0, norm_col1, norm_weight, norm_eps); a residual has out's
     row stride."""
     a = _strided_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
-    e = _epilogue(epilogue, strided=True)
+    e = _epilogue(dict(epilogue, y=out), strided=True)
     _check(lib().tern_linear_strided(ctypes.byref(a), ctypes.byref(e), _stream(stream)))
     return out
 

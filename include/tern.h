@@ -218,6 +218,17 @@ typedef struct {
   int64_t norm_col0, norm_col1;
   const void* norm_weight; /* [N] bf16 or NULL (weight 1) */
   float norm_eps;          /* > 0 and finite when a normalisation is requested */
+  /* Rotary position embedding of the normalised columns (FLUX.1 rotates q
+   * and k after their RMS norm), or NULL: fp32 (cos, sin) pairs, 64 per
+   * token row (row m at rope_cs + 128 m, 8-byte aligned, read only): channels
+   * (2j, 2j + 1) of every normalised 128-column group of row m become
+   *     (a cos - b sin, a sin + b cos),  (cos, sin) = pair j of row m,
+   * applied to the normalised fp32 values before the one rounding (the
+   * value before the normalisation was rounded to bf16, so a rotated value
+   * is within 3 * 2^-9 of (|a| + |b|) of the exact one).  Only
+   * with a normalisation and with no activation, residual or gate on the
+   * normalised columns (TERN_ERR_INVALID_ARG otherwise). */
+  const float* rope_cs;
 } tern_epilogue;
 
 /* tern_linear of *args with the fused epilogue *epilogue (NULL: none). */

@@ -26,9 +26,9 @@ Functions (each follows page "1.58-bit FLUX", arXiv 2412.18653 HTML v1):
   first linear applies.  The pages quantise every linear of FLUX's blocks
   (Section 3.1) but do not describe the operations between them; this is
   FLUX.1's MLP activation, written from its definition.
-* ``rms_norm_groups``, ``linear_epilogue(...)`` -- the fused epilogues of
-  FLUX.1's blocks: q/k RMS normalisation per head, the activation, and the
-  gated residual update.
+* ``rms_norm_groups``, ``rotate_pairs``, ``linear_epilogue(...)`` -- the
+  fused epilogues of FLUX.1's blocks: q/k RMS normalisation per head and
+  their rotary embedding, the activation, and the gated residual update.
 * ``adaln_modulate(x_bits, scale_bits, shift_bits, eps, tokens_per_row)`` --
   layer normalisation of each token row (no affine) modulated by a row of
   the adaLN modulation output: ``(x - mean) / sqrt(var + eps) * (1 + scale)
@@ -264,19 +264,38 @@ def rms_norm_groups(y: np.ndarray, col0: int, col1: int, eps: float, w_bits=None
     return y
 
 
+def rotate_pairs(y: np.ndarray, col0: int, col1: int, cs: np.ndarray, group: int = 128) -> np.ndarray:
+    """Rotary embedding of columns [col0, col1) of y [M, N]: in every group of
+    `group` columns, channels (2j, 2j + 1) of row m become (a cos - b sin,
+    a sin + b cos) with (cos, sin) = cs[m, j] (cs [M, group / 2, 2])."""
+    y = np.array(y, dtype=np.float64, order="C", copy=True)
+    cs = np.asarray(cs, dtype=np.float64)
+    c, sn = cs[:, :, 0], cs[:, :, 1]
+    for g0 in range(col0, col1, group):
+        a = y[:, g0:g0 + group:2].copy()
+        b = y[:, g0 + 1:g0 + group:2].copy()
+        y[:, g0:g0 + group:2] = a * c - b * sn
+        y[:, g0 + 1:g0 + group:2] = a * sn + b * c
+    return y
+
+
 def linear_epilogue(x_bits: np.ndarray, T: np.ndarray, s: np.ndarray, b_bits=None, act: int = ACT_NONE,
                     col0: int = 0, residual_bits=None, gate_bits=None, norm_cols=(0, 0), norm_w_bits=None,
-                    norm_eps: float = 0.0) -> np.ndarray:
+                    norm_eps: float = 0.0, rope_cs=None) -> np.ndarray:
     """The layer with a fused epilogue, in float64: v = linear(...),
     RMS-normalised per 128-column group on norm_cols, a = act(v) on columns
     [col0, N), then residual + gate * a (residual [M, N] and gate [N] are bf16
     bit patterns; absent residual = 0, absent gate = 1).  FLUX.1 normalises
     q and k per head and adds its attention and MLP outputs to the residual
     stream scaled by an adaLN-Zero gate; the pages describe no operation
-    between the quantised linears, so this follows that model's definition."""
+    between the quantised linears, so this follows that model's definition.
+    rope_cs [M, 64, 2]: the rotary embedding of the normalised columns'
+    channel pairs after the normalisation (FLUX.1 rotates q and k there)."""
     v = linear(x_bits, T, s, b_bits)
     if norm_cols[1] > norm_cols[0]:
         v = rms_norm_groups(v, norm_cols[0], norm_cols[1], norm_eps, norm_w_bits)
+        if rope_cs is not None:
+            v = rotate_pairs(v, norm_cols[0], norm_cols[1], rope_cs)
     if act == ACT_GELU_TANH:
         a = gelu_tanh(v, col0)
     elif act == ACT_NONE:

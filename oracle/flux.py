@@ -15,8 +15,10 @@ GELU MLP, and gated residual updates.
 
 Every tensor that the GPU path keeps in bf16 between two operations is
 rounded to bf16 here at the same point (``bf16``: round to nearest even from
-float64), so the oracle is FLUX.1's unfused sequence of operations with
-bf16 activations, each operation itself exact.  Linears go through
+float64), so the oracle is FLUX.1's sequence of operations with bf16
+activations, each operation itself exact; where the GPU path fuses two
+(q/k norm and rotary embedding in the projection's epilogue) there is one
+rounding after both.  Linears go through
 ``oracle.linear`` / ``linear_act`` / ``linear_epilogue`` with the codes and
 scales of the ternary weights.
 
@@ -29,7 +31,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import (ACT_GELU_TANH, adaln_modulate, bf16_bits_to_f64, gelu_tanh, linear, linear_act, linear_epilogue,
-               rms_norm_groups)
+               rms_norm_groups, rotate_pairs)
 
 HEAD_DIM = 128
 LN_EPS = 1e-6
@@ -115,16 +117,23 @@ def _lin(x, lin, **kw):
     return linear_epilogue(bits(x), T, s, b, **kw)
 
 
-def _qk_normed(y: np.ndarray, q_norm, k_norm, hidden: int) -> np.ndarray:
+def cos_sin(angles: np.ndarray) -> np.ndarray:
+    """(cos, sin) pairs [L, 64, 2] of rotation angles [L, 64]."""
+    return np.stack([np.cos(angles), np.sin(angles)], axis=-1)
+
+
+def _qk_normed(y: np.ndarray, q_norm, k_norm, hidden: int, angles: np.ndarray) -> np.ndarray:
     """q, k and v columns of a projection's bf16 output y, q and k normalised
-    per head (fp64, rounded to bf16)."""
+    per head and then rotated (fp64, one rounding to bf16: the GPU path does
+    both in the projection's epilogue)."""
     qk = rms_norm_groups(y[:, :2 * hidden], 0, 2 * hidden, QK_EPS, _qk_norm_weight(q_norm, k_norm, hidden))
+    qk = rotate_pairs(qk, 0, 2 * hidden, cos_sin(angles))
     return np.concatenate([bf16(qk), y[:, 2 * hidden:3 * hidden]], axis=1)
 
 
-def _attend(qkv: np.ndarray, angles: np.ndarray, hidden: int) -> np.ndarray:
+def _attend(qkv: np.ndarray, hidden: int) -> np.ndarray:
+    """Attention over all rows of qkv (q and k already rotated)."""
     q, k, v = _heads(qkv[:, :hidden]), _heads(qkv[:, hidden:2 * hidden]), _heads(qkv[:, 2 * hidden:])
-    q, k = bf16(apply_rope(q, angles)), bf16(apply_rope(k, angles))
     return bf16(_tokens(attention(q, k, v)))
 
 
@@ -140,12 +149,12 @@ def double_block(img: np.ndarray, txt: np.ndarray, vec: np.ndarray, p: dict, ang
         m = bf16(_lin(y, p[s + ".mod"]))[0]
         mods[s] = [m[i * hidden:(i + 1) * hidden] for i in range(6)]  # shift1 scale1 gate1 shift2 scale2 gate2
     qkv = {}
-    for s, x in (("img", img), ("txt", txt)):
+    lt = txt.shape[0]
+    for s, x, ang in (("img", img, angles[lt:]), ("txt", txt, angles[:lt])):
         sh1, sc1 = mods[s][0], mods[s][1]
         xm = bf16(adaln_modulate(bits(x), bits(sc1[None]), bits(sh1[None]), LN_EPS))
-        qkv[s] = _qk_normed(bf16(_lin(xm, p[s + ".qkv"])), p[s + ".q_norm"], p[s + ".k_norm"], hidden)
-    att = _attend(np.concatenate([qkv["txt"], qkv["img"]], axis=0), angles, hidden)
-    lt = txt.shape[0]
+        qkv[s] = _qk_normed(bf16(_lin(xm, p[s + ".qkv"])), p[s + ".q_norm"], p[s + ".k_norm"], hidden, ang)
+    att = _attend(np.concatenate([qkv["txt"], qkv["img"]], axis=0), hidden)
     for s, x, a in (("img", img, att[lt:]), ("txt", txt, att[:lt])):
         sh1, sc1, g1, sh2, sc2, g2 = mods[s]
         x1 = bf16(_lin(a, p[s + ".proj"], residual_bits=bits(x), gate_bits=bits(g1)))
@@ -167,9 +176,9 @@ def single_block(x: np.ndarray, vec: np.ndarray, p: dict, angles: np.ndarray) ->
     xm = bf16(adaln_modulate(bits(x), bits(sc[None]), bits(sh[None]), LN_EPS))
     T, s1, b1 = p["linear1"]
     z = linear(bits(xm), T, s1, b1)
-    qkv = _qk_normed(bf16(z[:, :3 * hidden]), p["q_norm"], p["k_norm"], hidden)
+    qkv = _qk_normed(bf16(z[:, :3 * hidden]), p["q_norm"], p["k_norm"], hidden, angles)
     mlp = bf16(gelu_tanh(z[:, 3 * hidden:]))
-    att = _attend(qkv, angles, hidden)
+    att = _attend(qkv, hidden)
     return bf16(_lin(np.concatenate([att, mlp], axis=1), p["linear2"], residual_bits=bits(x), gate_bits=bits(g)))
 
 

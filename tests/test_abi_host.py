@@ -208,6 +208,22 @@ def test_norm_epilogue_rejects_on_host(L):
     assert call(N=384, c1=128) == SHAPE   # would run on the fallback kernel
 
 
+def test_rope_epilogue_rejects_on_host(L):
+    """The rotary table: only with a normalisation, no activation, residual or
+    gate on the normalised columns, 8-byte aligned, not overlapping y."""
+    def call(c1=256, act=0, col0=0, residual=None, gate=None, rope=F + 0x600000):
+        a = tern.LinearArgs(F, F + 0x100000, F + 0x200000, None, F + 0x300000, 40, 512, 256)
+        e = tern.Epilogue(act, col0, residual, gate, 0, c1, None, 1e-6, rope)
+        return L.tern_linear_epilogue(ctypes.byref(a), ctypes.byref(e), None)
+    assert call(c1=0) == INVALID                     # nothing normalised
+    assert call(act=1, col0=128) == INVALID          # GELU on normalised columns
+    assert call(residual=F + 0x700000) == INVALID
+    assert call(gate=F + 0x700000) == INVALID
+    assert call(rope=F + 0x600004) == MISALIGNED
+    assert call(rope=F + 0x300000 + 512) == INVALID  # inside y
+    assert call(act=1, col0=256, rope=F + 0x600004) == MISALIGNED  # GELU past the normalised columns is fine
+
+
 def test_adaln_rejects_on_host(L):
     """tern_adaln_modulate's shape, alignment and overlap checks, before any
     device work; M = 0 is a successful no-op."""

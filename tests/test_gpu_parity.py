@@ -509,6 +509,82 @@ def test_linear_epilogue_rms_norm_flux_qkv_full():
     check_y(y, ref)
 
 
+def check_y_rotated(y_gpu: torch.Tensor, y_ref: np.ndarray, cols):
+    """check_y, with the bar on the rotated columns [cols) taken over both
+    channels of each pair: the rotation mixes a channel with its partner,
+    each carrying the bf16 rounding of the value before the normalisation
+    (2^-9 relative), so the error scales with |a| + |b| of the pair, not
+    with the rotated output alone."""
+    y = y_gpu.detach().cpu().double().numpy()
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    mag = np.abs(y_ref).copy()
+    c0, c1 = cols
+    pair = np.abs(y_ref[:, c0:c1]).reshape(y_ref.shape[0], -1, 2).sum(axis=2)
+    mag[:, c0:c1] = np.repeat(pair, 2, axis=1)
+    err = np.abs(y - y_ref)
+    bad = err > Y_RTOL * mag + Y_RMS * rms
+    assert not bad.any(), (f"{int(bad.sum())} of {bad.size} outputs out of tolerance; "
+                           f"worst err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}")
+
+
+def rope_table(M, seed):
+    """fp32 (cos, sin) pairs [M, 64, 2] of seeded angles in [-60, 60)."""
+    a = torch.rand(M, 64, generator=torch.Generator().manual_seed(seed), dtype=torch.float64) * 120 - 60
+    return torch.stack([torch.cos(a), torch.sin(a)], dim=-1).float()
+
+
+@pytest.mark.parametrize("M,N,K,cols", [
+    (300, 512, 192, (0, 512)),      # CTA-pair tiles, every column normalised and rotated
+    (1024, 768, 320, (0, 512)),     # several tiles per pair, v-like columns untouched
+    (40, 512, 256, (128, 384)),     # 64-token tiles
+    (17, 256, 128, (0, 256)),       # 64-token tile, one token past the GEMV range
+])
+def test_linear_epilogue_rms_norm_rope(M, N, K, cols):
+    """q/k norm followed by the rotary embedding of the normalised columns'
+    channel pairs, one rounding; ragged token tails read no table row past M.
+    The value before the normalisation is rounded to bf16 (the norm's
+    two-rounding path), and the rotation mixes it with its partner channel:
+    the bar covers both channels' magnitudes (check_y_rotated)."""
+    W = rand_bf16((N, K), 0.02, M + 29 * N)
+    x = rand_bf16((M, K), 1.0, M + 31 * K)
+    b = rand_bf16((N,), 0.01, N + 37)
+    w = (torch.rand(N, generator=torch.Generator().manual_seed(N + 1)) + 0.5).to(torch.bfloat16)
+    cs = rope_table(M, M + N)
+    packed, scales = quantize_on_gpu(W)
+    T, s = check_quantize(W, packed, scales, {})
+    y = tern.linear_epilogue(x.cuda(), packed, scales, b.cuda(), norm_cols=cols, norm_weight=w.cuda(),
+                             norm_eps=1e-6, rope_cs=cs.cuda())
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    ref = oracle.linear_epilogue(bits(x), T, s, bits(b), 0, 0, None, None, cols, bits(w), 1e-6,
+                                 rope_cs=cs.double().numpy())
+    check_y_rotated(y, ref, cols)
+
+
+def test_linear_batch_epilogue_rope_row_offsets():
+    """Two problems writing the halves of one buffer, each with its own rows
+    of one rotary table (the caller offsets the table pointer)."""
+    M1, M2, N, K = 96, 200, 512, 256
+    cs = rope_table(M1 + M2, 7)
+    buf = torch.empty(M1 + M2, N, dtype=torch.bfloat16, device="cuda")
+    probs, refs = [], []
+    for i, (r0, r1) in enumerate([(0, M1), (M1, M1 + M2)]):
+        W = rand_bf16((N, K), 0.02, 1500 + i)
+        x = rand_bf16((r1 - r0, K), 1.0, 1600 + i)
+        b = rand_bf16((N,), 0.01, 1700 + i)
+        packed, scales = quantize_on_gpu(W)
+        T, s = check_quantize(W, packed, scales, {})
+        probs.append(dict(x=x.cuda(), packed=packed, scales=scales, bias=b.cuda(), y=buf[r0:r1], norm_col0=0,
+                          norm_col1=256, norm_eps=1e-6, rope_cs=cs[r0:r1].cuda()))
+        refs.append(oracle.linear_epilogue(bits(x), T, s, bits(b), 0, 0, None, None, (0, 256), None, 1e-6,
+                                           rope_cs=cs[r0:r1].double().numpy()))
+    tern.linear_batch_epilogue(probs)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    for p, ref in zip(probs, refs):
+        check_y_rotated(p["y"], ref, (0, 256))
+
+
 def test_linear_batch_epilogue_with_norm():
     """A batch where one pair-tile problem normalises and the others do not:
     the whole launch runs the normalising kernel."""

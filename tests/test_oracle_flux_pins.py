@@ -149,3 +149,18 @@ def test_single_block_zero_gate_and_zero_second_linear():
     g = OF.bf16(oracle.linear(OF.bits(OF.bf16(OF.silu(vec))), T, s, b))[0, 2 * C:]
     want = OF.bf16(x + g[None, :] * OF.from_bits(p["linear2"][2])[None, :])
     assert np.array_equal(out, want)
+
+
+def test_rotate_pairs_matches_the_pinned_rotary_embedding():
+    """oracle.rotate_pairs (the fused epilogue's rotation of the normalised
+    columns) against OF.apply_rope (pinned above) on two heads."""
+    rng = np.random.default_rng(9)
+    L = 7
+    y = rng.standard_normal((L, 3 * 128))
+    ids = np.stack([np.zeros(L), rng.integers(0, 60, L), rng.integers(0, 60, L)], axis=1).astype(float)
+    ang = OF.rope_angles(ids)
+    got = oracle.rotate_pairs(y, 0, 256, OF.cos_sin(ang))
+    heads = y[:, :256].reshape(L, 2, 128).transpose(1, 0, 2)
+    want = OF.apply_rope(heads, ang).transpose(1, 0, 2).reshape(L, 256)
+    assert np.allclose(got[:, :256], want, rtol=0, atol=1e-14)
+    assert np.array_equal(got[:, 256:], y[:, 256:])
