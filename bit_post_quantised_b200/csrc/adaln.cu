@@ -18,6 +18,7 @@
 // of a FLUX.1 single block's stream run in one wave.
 #include "internal.h"
 #include "kernel_common.cuh"
+#include "ptx.cuh"
 
 namespace tern {
 
@@ -86,6 +87,8 @@ __global__ void __launch_bounds__(kAdaRows * 32, 4)
     adaln_modulate_kernel(const uint16_t* x, int M, int K, const uint16_t* __restrict__ scale,
                           const uint16_t* __restrict__ shift, int mod_ld, int tokens_per_row, float eps,
                           uint16_t* out) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * kAdaRows + warp;
   if (m >= M) return;
@@ -144,9 +147,8 @@ template <int NV>
 cudaError_t launch_nv(const uint16_t* x, int M, int K, const uint16_t* scale, const uint16_t* shift, int mod_ld,
                       int tokens_per_row, float eps, uint16_t* out, cudaStream_t stream) {
   const int grid = (M + kAdaRows - 1) / kAdaRows;
-  adaln_modulate_kernel<NV><<<grid, kAdaRows * 32, 0, stream>>>(x, M, K, scale, shift, mod_ld, tokens_per_row,
-                                                                 eps, out);
-  return cudaGetLastError();
+  return launch_pdl(adaln_modulate_kernel<NV>, dim3(grid), dim3(kAdaRows * 32), 0, stream, 1, x, M, K, scale, shift,
+                    mod_ld, tokens_per_row, eps, out);
 }
 
 }  // namespace

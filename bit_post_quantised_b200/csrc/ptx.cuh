@@ -114,6 +114,20 @@ __device__ __forceinline__ bool mbar_wait_both(uint32_t bar0, uint32_t parity0, 
   return (d0 || mbar_wait(bar0, parity0, limit_ns, status)) && (d1 || mbar_wait(bar1, parity1, limit_ns, status));
 }
 
+// Programmatic dependent launch.  Our kernels are launched with it allowed,
+// so a grid may start while the previous kernel of its stream still runs:
+// every kernel calls pdl_wait() before it touches global memory (it returns
+// once the previous grid has finished and its writes are visible; at once
+// when there is none), then pdl_trigger() lets the next kernel be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Asks L2 to fetch [p, p + bytes) (16-byte aligned, a multiple of 16 bytes);
+// a hint with no result and no ordering.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Asks for the 128-byte line holding `p` to be brought into L2 (no register
 // result, no ordering).
 __device__ __forceinline__ void prefetch_l2(const void* p) {

@@ -111,6 +111,8 @@ __device__ __forceinline__ uint32_t group_codes_int(const uint4& v, uint32_t thr
 // != 0): their code words are zero and they have no scale.  One thread per
 // 32-bit word (word w of a row holds k = 16w .. 16w + 15).
 __global__ void zero_pad_rows_kernel(uint8_t* __restrict__ packed, int N, int K) {
+  pdl_wait();
+  pdl_trigger();
   const int words = K >> 4;
   const int pad_rows = ((N + 127) & ~127) - N;
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -128,6 +130,8 @@ template <int NV>
 __global__ void __launch_bounds__(kRowsPerCta * 32)
     quantize_pack_regs_kernel(const uint16_t* __restrict__ W, int N, int K, float eps,
                               uint8_t* __restrict__ packed, float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kRowsPerCta + warp;
   if (n >= N) return;
@@ -173,6 +177,8 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 __global__ void __launch_bounds__(kRowsPerCta * 32)
     quantize_pack_long_kernel(const uint16_t* __restrict__ W, int N, int K, float eps,
                               uint8_t* __restrict__ packed, float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int NV = 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kRowsPerCta + warp;
@@ -222,6 +228,8 @@ __global__ void __launch_bounds__(kRowsPerCta * 32)
 // ---- dequantise: one thread per 16-byte group (row n, 64-wide chunk c)
 __global__ void dequantize_kernel(const uint8_t* __restrict__ packed, const float* __restrict__ scales,
                                   int N, int K, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const size_t groups = size_t(N) * (K >> 6);
   const size_t g = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= groups) return;
@@ -271,21 +279,22 @@ cudaError_t launch_quantize_pack(const __nv_bfloat16* W, int N, int K, float eps
   const uint16_t* w = reinterpret_cast<const uint16_t*>(W);
   // Rows of up to 4096 values stay in registers (one read of W); longer rows
   // are read twice, the second time mostly from L2.
+  const dim3 g(grid), b(kRowsPerCta * 32);
+  cudaError_t e;
   if (K <= 32 * 8 * 4)
-    quantize_pack_regs_kernel<4><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+    e = launch_pdl(quantize_pack_regs_kernel<4>, g, b, 0, stream, 1, w, N, K, eps, packed, scales);
   else if (K <= 32 * 8 * 8)
-    quantize_pack_regs_kernel<8><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+    e = launch_pdl(quantize_pack_regs_kernel<8>, g, b, 0, stream, 1, w, N, K, eps, packed, scales);
   else if (K <= 32 * 8 * 12)
-    quantize_pack_regs_kernel<12><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+    e = launch_pdl(quantize_pack_regs_kernel<12>, g, b, 0, stream, 1, w, N, K, eps, packed, scales);
   else if (K <= 32 * 8 * 16)
-    quantize_pack_regs_kernel<16><<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
+    e = launch_pdl(quantize_pack_regs_kernel<16>, g, b, 0, stream, 1, w, N, K, eps, packed, scales);
   else
-    quantize_pack_long_kernel<<<grid, kRowsPerCta * 32, 0, stream>>>(w, N, K, eps, packed, scales);
-  if (N % 128 != 0) {
-    const long long n_words = (long long)(((N + 127) & ~127) - N) * (K >> 4);
-    zero_pad_rows_kernel<<<unsigned((n_words + 255) / 256), 256, 0, stream>>>(packed, N, K);
-  }
-  return cudaGetLastError();
+    e = launch_pdl(quantize_pack_long_kernel, g, b, 0, stream, 1, w, N, K, eps, packed, scales);
+  if (e != cudaSuccess || N % 128 == 0) return e;
+  const long long n_words = (long long)(((N + 127) & ~127) - N) * (K >> 4);
+  return launch_pdl(zero_pad_rows_kernel, dim3(unsigned((n_words + 255) / 256)), dim3(256), 0, stream, 1, packed, N,
+                    K);
 }
 
 cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N, int K,
@@ -293,8 +302,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int N,
   const size_t groups = size_t(N) * (K >> 6);
   const int threads = 256;
   const size_t grid = (groups + threads - 1) / threads;
-  dequantize_kernel<<<unsigned(grid), threads, 0, stream>>>(packed, scales, N, K, out);
-  return cudaGetLastError();
+  return launch_pdl(dequantize_kernel, dim3(unsigned(grid)), dim3(threads), 0, stream, 1, packed, scales, N, K, out);
 }
 
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, unsigned int* status,

@@ -70,6 +70,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 template <int NV>
 __global__ void __launch_bounds__(256, NV > 6 ? 2 : 4) quantize_act_e4m3_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                                  uint8_t* __restrict__ xq, float* __restrict__ a) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= M) return;
@@ -298,6 +300,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(F8Cfg::kThreads, 1)
   }
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers exist and TMEM is allocated
+  pdl_wait();
+  pdl_trigger();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
@@ -505,12 +509,12 @@ cudaError_t launch_quantize_act_e4m3(const __nv_bfloat16* x, int M, int K, uint8
   if (M <= 0) return cudaSuccess;
   const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
   const dim3 grid((M + 7) / 8);
-  if (K <= 512 * 2) quantize_act_e4m3_kernel<2><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
-  else if (K <= 512 * 4) quantize_act_e4m3_kernel<4><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
-  else if (K <= 512 * 6) quantize_act_e4m3_kernel<6><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
-  else if (K <= 512 * 8) quantize_act_e4m3_kernel<8><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
-  else quantize_act_e4m3_kernel<0><<<grid, 256, 0, stream>>>(xb, M, K, xq, a);
-  return cudaGetLastError();
+  const dim3 b(256);
+  if (K <= 512 * 2) return launch_pdl(quantize_act_e4m3_kernel<2>, grid, b, 0, stream, 1, xb, M, K, xq, a);
+  if (K <= 512 * 4) return launch_pdl(quantize_act_e4m3_kernel<4>, grid, b, 0, stream, 1, xb, M, K, xq, a);
+  if (K <= 512 * 6) return launch_pdl(quantize_act_e4m3_kernel<6>, grid, b, 0, stream, 1, xb, M, K, xq, a);
+  if (K <= 512 * 8) return launch_pdl(quantize_act_e4m3_kernel<8>, grid, b, 0, stream, 1, xb, M, K, xq, a);
+  return launch_pdl(quantize_act_e4m3_kernel<0>, grid, b, 0, stream, 1, xb, M, K, xq, a);
 }
 
 cudaError_t launch_ternary_fp8(const Batch& batch, int pairs, cudaStream_t stream) {
@@ -525,8 +529,7 @@ cudaError_t launch_ternary_fp8(const Batch& batch, int pairs, cudaStream_t strea
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
-  ternary_fp8_pair_kernel<<<2 * pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
-  return cudaGetLastError();
+  return launch_pdl(ternary_fp8_pair_kernel, dim3(2 * pairs), dim3(C::kThreads), C::kSmemBytes, stream, 1, batch);
 }
 
 }  // namespace tern

@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   // (The host never launches otherwise; the test is uniform over the grid,
   // so every CTA leaves here and the host reads TERN_ERR_LAUNCH_CONFIG.)
   if (splits > 1 && ustep < units) {
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(st, kStatusLaunchConfig);
     return;
   }
@@ -165,6 +166,21 @@ __global__ void __launch_bounds__(GemvCfg<NT>::kThreads, 1)
   }
   const int nprob = batch.count;
   __syncthreads();
+  // The previous kernel of the stream may still be running (programmatic
+  // dependent launch): the producer first asks L2 for the codes of its first
+  // stages (a hint: a write by that kernel still reaches the readers through
+  // L2), then every thread waits for it before touching global memory.
+  if (warp == C::kWarps && lane == 0 && u0 < units) {
+    int slab;
+    const GemvProb& P = probs[unit_problem(probs, nprob, u0, &slab)];
+    const int kc_total = P.K >> 6;
+    const int kc0 = rank * P.chunks_per_split;
+    const int nk = max(0, min(kc_total, kc0 + P.chunks_per_split) - kc0);
+    if (nk > 0)
+      prefetch_l2_bulk(P.packed + (size_t(slab) * kc_total + kc0) * 2048, uint32_t(min(nk, S * C::kChunks)) * 2048u);
+  }
+  pdl_wait();
+  pdl_trigger();
   const int grp = warp;  // 16-channel group of a consumer warp
 
   if (warp == C::kWarps) {
@@ -363,19 +379,8 @@ static cudaError_t launch_nt(const Batch& batch, int splits, int ctas, cudaStrea
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(splits), unsigned(ctas), 1);
-  cfg.blockDim = dim3(C::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<NT>, batch);
+  return launch_pdl(ternary_gemv_kernel<NT>, dim3(unsigned(splits), unsigned(ctas), 1), dim3(C::kThreads),
+                    C::kSmemBytes, stream, unsigned(splits), batch);
 }
 
 cudaError_t launch_ternary_gemv(int nt, const Batch& batch, int splits, int ctas, cudaStream_t stream) {

@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(TileCfg<TOK>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
@@ -263,8 +265,8 @@ static cudaError_t launch_tok(const Batch& batch, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, 1ull << dev, __ATOMIC_RELEASE);
   }
-  ternary_mma_kernel<TOK><<<batch.total_units, C::kThreads, C::kSmemBytes, stream>>>(batch);
-  return cudaGetLastError();
+  return launch_pdl(ternary_mma_kernel<TOK>, dim3(batch.total_units), dim3(C::kThreads), C::kSmemBytes, stream, 1,
+                    batch);
 }
 
 int smem_bytes_for_tok(int tok) {

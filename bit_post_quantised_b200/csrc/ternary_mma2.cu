@@ -263,6 +263,18 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
   }
   tc_fence_before();
   T::sync_all();  // (both CTAs') barriers exist and TMEM is allocated
+  // The previous kernel of the stream may still be running (programmatic
+  // dependent launch): the producer first asks L2 for the codes of its first
+  // stages (a hint: a write by that kernel still reaches the readers through
+  // L2), then every thread waits for it before touching global memory.
+  if (warp == 0 && lane == 0 && u0 < units) {
+    const Tile2 t = tile_of(batch, u0);
+    const int kc_total = t.P->K >> 6;
+    const uint8_t* codes = t.P->packed + size_t(t.n_tile * C::kCtas + int(rank)) * kc_total * C::kCSub;
+    prefetch_l2_bulk(codes, uint32_t(min(kc_total, S * C::kChunks)) * C::kCSub);
+  }
+  pdl_wait();
+  pdl_trigger();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
@@ -810,8 +822,8 @@ static cudaError_t launch_tile(const Batch& batch, int ctas_or_pairs, cudaStream
   using C = Cfg2<TOK, PAIR, EPI>;
   cudaError_t e = configure_tile<TOK, PAIR, EPI>();
   if (e != cudaSuccess) return e;
-  tile_kernel<TOK, PAIR, EPI>()<<<C::kCtas * ctas_or_pairs, C::kThreads, C::kSmemBytes, stream>>>(batch);
-  return cudaGetLastError();
+  return launch_pdl(tile_kernel<TOK, PAIR, EPI>(), dim3(C::kCtas * ctas_or_pairs), dim3(C::kThreads), C::kSmemBytes,
+                    stream, 1, batch);
 }
 
 cudaError_t launch_ternary_mma2(int tok, bool pair, const Batch& batch, int ctas_or_pairs, cudaStream_t stream) {
