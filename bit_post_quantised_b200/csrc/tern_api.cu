@@ -426,10 +426,17 @@ tern_status fill_problem_2sm(const LinArgs& a, int tok, Problem* p, int64_t* til
   return TERN_OK;
 }
 
-// Launches the problems `idx` of `args` (all with pair_tok == tok) on the
-// pair-tile kernel, up to kMaxProblems per launch.
-tern_status launch_2sm_group(const LinArgs* args, const tern_epilogue* epis, const std::vector<int>& idx, int tok,
+// Launches the problems `idx_in` of `args` (all with pair_tok == tok) on the
+// pair-tile kernel, up to kMaxProblems per launch.  The kernel hands tile u
+// of a launch to CTA (pair) u mod #resident, in problem order; problems go in
+// by decreasing K (a tile's cost), so the long tiles are dealt out first and
+// spread evenly (a FLUX double block's batch, whose MLP-down tiles take four
+// times the others: the busiest pair holds 36 instead of 39 tile-units for
+// an even share of 35).
+tern_status launch_2sm_group(const LinArgs* args, const tern_epilogue* epis, const std::vector<int>& idx_in, int tok,
                              Batch& batch, const DeviceState* ds, cudaStream_t cs) {
+  std::vector<int> idx(idx_in);
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return args[a].K > args[b].K; });
   for (size_t g0 = 0; g0 < idx.size(); g0 += kMaxProblems) {
     std::memset(static_cast<void*>(&batch), 0, sizeof batch);
     int64_t total = 0;
