@@ -644,13 +644,14 @@ def stack_rows(device, peaks, stream):
 
 
 def forward_rows(device, peaks, stream):
-    """The blocks of a FLUX.1-shaped forward at 1024x1024 (19 double + 38
-    single, seeded random weights, synthetic activations): every linear
+    """A FLUX.1-shaped forward at 1024x1024 (19 double + 38 single blocks,
+    seeded random weights, synthetic inputs): the unquantised input layers
+    and embedders and the final layer in bf16 (cuBLAS), every block linear
     ternary through the library with its fused epilogues (the rotary
-    embedding in the q/k epilogue), attention from torch; against the same blocks in bf16 with dense
-    weights (T*s) through cuBLAS and torch's unfused operations, the bf16
-    model of the pages' Table 3 comparison.  The two are timed in turns
-    (CUDA events, medians of 3)."""
+    embedding in the q/k epilogue), attention from torch; against the same
+    model with the blocks in bf16 with dense weights (T*s) through cuBLAS and
+    torch's unfused operations, the bf16 model of the pages' Table 3
+    comparison.  The two are timed in turns (CUDA events, medians of 3)."""
     import statistics
 
     import torch
@@ -659,10 +660,12 @@ def forward_rows(device, peaks, stream):
 
     cfg = workloads.FluxConfig()
     model = flux.TernaryFlux(cfg, device=device)
-    img, txt, vec, ids = (t.to(device) for t in workloads.flux_inputs(cfg))
+    io = {k: (W.to(device), b.to(device)) for k, (W, b) in workloads.flux_io_weights(cfg).items()}
+    img, txt, pooled, t, g, ids = workloads.flux_model_inputs(cfg)
+    args = (img.to(device), txt.to(device), pooled.to(device), t, g, ids.to(device))
     dense = flux.dense_weights(model)
-    runs = {"ternary": lambda: model.forward(img, txt, vec, ids),
-            "dense_bf16": lambda: flux.dense_forward(model, dense, img, txt, vec, ids)}
+    runs = {"ternary": lambda: flux.model_forward(model, io, *args),
+            "dense_bf16": lambda: flux.dense_model_forward(model, dense, io, *args)}
     for f in runs.values():
         f()
     torch.cuda.synchronize()
@@ -679,17 +682,21 @@ def forward_rows(device, peaks, stream):
     fl = flux.forward_flop(cfg)
     packed = sum(q[n][0].numel() for q in model.blocks.values() for n in q if not n.endswith("norm_w"))
     dense_b = sum(d[n][0].numel() * 2 for d in dense.values() for n in d if not n.endswith("norm_w"))
+    io_b = sum(W.numel() * 2 for W, _ in io.values())
     t_ter, t_den = statistics.median(times["ternary"]), statistics.median(times["dense_bf16"])
     del dense, model
     torch.cuda.empty_cache()
-    return {"flux_forward_blocks": {
-        "blocks": f"{cfg.n_double} double + {cfg.n_single} single, {cfg.img_tokens} image + {cfg.txt_tokens} text tokens",
+    return {"flux_forward": {
+        "model": f"{cfg.n_double} double + {cfg.n_single} single blocks, {cfg.img_tokens} image + "
+                 f"{cfg.txt_tokens} text tokens, input layers, embedders and final layer",
         "ternary_ms": t_ter, "dense_bf16_ms": t_den, "speedup_vs_dense_bf16": t_den / t_ter,
         "linear_gflop": fl["linear"] / 1e9, "attention_gflop": fl["attention"] / 1e9,
         "ternary_tflops": (fl["linear"] + fl["attention"]) / (t_ter * 1e-3) / 1e12,
         "block_weight_gb_ternary": packed / 1e9, "block_weight_gb_bf16": dense_b / 1e9,
-        "outside": "attention (torch SDPA) and SiLU: torch; all linears (with q/k norm and rotary embedding, "
-                   "GELU, gated residual in their epilogues) and the adaLN pass: this library"}}
+        "io_layer_weight_gb_bf16": io_b / 1e9,
+        "outside": "attention (torch SDPA), SiLU and the unquantised input/output layers (bf16 cuBLAS): torch; "
+                   "all block linears (with q/k norm and rotary embedding, GELU, gated residual in their "
+                   "epilogues) and the adaLN passes: this library"}}
 
 
 def gpu_id_for_smi(local: int) -> str:

@@ -217,6 +217,45 @@ class TernaryFlux:
         return x
 
 
+def timestep_embedding(t: float, device, dim: int = 256, max_period: float = 10000.0,
+                       time_factor: float = 1000.0) -> torch.Tensor:
+    """FLUX.1's sinusoidal embedding of a scalar (timestep or guidance) as
+    [1, dim] bf16: cos and sin of 1000 t * max_period^(-j / (dim / 2))."""
+    half = dim // 2
+    freqs = torch.exp(-math.log(max_period) * torch.arange(half, dtype=torch.float32, device=device) / half)
+    args = time_factor * t * freqs
+    return torch.cat([torch.cos(args), torch.sin(args)])[None].to(torch.bfloat16)
+
+
+def io_layers_in(io: Dict, img_lat, txt_ctx, pooled, t: float, guidance: float):
+    """The unquantised input layers (bf16, cuBLAS): image and text
+    projections, and vec = time + guidance + pooled-text embedders, each
+    Linear -> SiLU -> Linear.  Returns img [Li, C], txt [Lt, C], vec [1, C]."""
+    dev = img_lat.device
+
+    def mlp(x, a, b):
+        return F.linear(F.silu(F.linear(x, *io[a])), *io[b])
+
+    vec = (mlp(timestep_embedding(t, dev), "time_in.0", "time_in.1")
+           + mlp(timestep_embedding(guidance, dev), "guidance_in.0", "guidance_in.1")
+           + mlp(pooled, "vector_in.0", "vector_in.1"))
+    return F.linear(img_lat, *io["img_in"]), F.linear(txt_ctx, *io["txt_in"]), vec
+
+
+def model_forward(model: "TernaryFlux", io: Dict, img_lat, txt_ctx, pooled, t: float, guidance: float, ids,
+                  n_double=None, n_single=None) -> torch.Tensor:
+    """The whole transformer: the bf16 input layers, every block through the
+    library, and the final layer (adaLN modulation row from SiLU(vec) in
+    bf16, layer norm and modulation of the image tokens by the library's
+    adaLN pass, the bf16 output projection).  Returns [Li, in_channels]."""
+    img, txt, vec = io_layers_in(io, img_lat, txt_ctx, pooled, t, guidance)
+    x = model.forward(img, txt, vec, ids, n_double, n_single)
+    C = model.cfg.hidden
+    mod = F.linear(F.silu(vec), *io["final.mod"])  # [shift | scale]
+    h = tern.adaln_modulate(x[txt.shape[0]:], mod[:, C:], mod[:, :C], LN_EPS, stream=model.stream)
+    return F.linear(h, *io["final.out"])
+
+
 def dense_weights(model: TernaryFlux) -> Dict:
     """bf16 dense weights T * s of every ternary linear of `model` (what the
     bf16 model would hold), plus the biases and norm weights."""
@@ -306,3 +345,15 @@ def max_abs_rel(a: torch.Tensor, b: torch.Tensor) -> float:
     """max |a - b| / rms(b) (diagnostic)."""
     d = (a.float() - b.float()).abs().max().item()
     return d / max(math.sqrt(b.float().pow(2).mean().item()), 1e-30)
+
+
+def dense_model_forward(model: TernaryFlux, dense: Dict, io: Dict, img_lat, txt_ctx, pooled, t: float,
+                        guidance: float, ids, n_double=None, n_single=None) -> torch.Tensor:
+    """model_forward with the blocks in dense bf16 (dense_forward) and the
+    final layer norm and modulation from torch."""
+    img, txt, vec = io_layers_in(io, img_lat, txt_ctx, pooled, t, guidance)
+    x = dense_forward(model, dense, img, txt, vec, ids, n_double, n_single)
+    C = model.cfg.hidden
+    mod = F.linear(F.silu(vec), *io["final.mod"])
+    h = F.layer_norm(x[txt.shape[0]:], (C,), eps=LN_EPS) * (1 + mod[:, C:]) + mod[:, :C]
+    return F.linear(h, *io["final.out"])

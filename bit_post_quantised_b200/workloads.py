@@ -230,3 +230,40 @@ def flux_inputs(cfg: FluxConfig, seed: int = 5):
     ids[cfg.txt_tokens:, 1] = r.float()
     ids[cfg.txt_tokens:, 2] = c.float()
     return img, txt, vec, ids
+
+
+def flux_io_weights(cfg: FluxConfig, device=None):
+    """Seeded bf16 parameters of the unquantised input and output layers of a
+    FLUX.1-shaped transformer (the 0.5 % of parameters the pages leave in
+    16 bits): image and text input projections, the time, guidance and
+    pooled-text embedders (Linear -> SiLU -> Linear), the final adaLN
+    modulation and output projection; each (W [N, K] ~ N(0, 0.02),
+    b [N] ~ N(0, 0.01))."""
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed * 1000003 + 999)
+    C = cfg.hidden
+
+    def lin(N, K):
+        W = (torch.randn((N, K), generator=gen, device=dev) * W_STD).to(torch.bfloat16)
+        b = (torch.randn((N,), generator=gen, device=dev) * B_STD).to(torch.bfloat16)
+        return W, b
+
+    return {"img_in": lin(C, cfg.in_channels), "txt_in": lin(C, cfg.context_dim),
+            "time_in.0": lin(C, 256), "time_in.1": lin(C, C), "guidance_in.0": lin(C, 256),
+            "guidance_in.1": lin(C, C), "vector_in.0": lin(C, 768), "vector_in.1": lin(C, C),
+            "final.mod": lin(2 * C, C), "final.out": lin(cfg.in_channels, C)}
+
+
+def flux_model_inputs(cfg: FluxConfig, seed: int = 6):
+    """Seeded CPU inputs of the whole transformer: packed image latents
+    [Li, in_channels] and text encoder states [Lt, context_dim] (bf16,
+    N(0, 1)), pooled text vector [1, 768], the timestep and guidance value
+    (scalars in [0, 1) and [1, 5)), and the token positions as flux_inputs."""
+    gen = torch.Generator().manual_seed(seed)
+    img = _normal((cfg.img_tokens, cfg.in_channels), 1.0, gen)
+    txt = _normal((cfg.txt_tokens, cfg.context_dim), 1.0, gen)
+    pooled = _normal((1, 768), 1.0, gen)
+    t = float(torch.rand(1, generator=gen))
+    guidance = 1.0 + 4.0 * float(torch.rand(1, generator=gen))
+    ids = flux_inputs(cfg)[3]
+    return img, txt, pooled, t, guidance, ids

@@ -18,7 +18,9 @@ Full size (hidden 3072, 4096 + 512 tokens), one double and one single
 block against the same blocks in bf16 with dense weights (cuBLAS, torch's
 unfused operations): a consistency check of the fused path at full size,
 rms(out - dense) <= 2^-5 rms(dense) (the dense path rounds to bf16 after
-each unfused operation and uses T*s rounded to bf16 as its weights).
+each unfused operation and uses T*s rounded to bf16 as its weights); and
+the whole transformer (the unquantised input layers and embedders, the
+blocks, the final layer) the same way.
 """
 from __future__ import annotations
 
@@ -98,4 +100,23 @@ def test_full_size_blocks_agree_with_dense_bf16():
     assert torch.isfinite(out.float()).all()
     d = (out.float() - dense.float()).pow(2).mean().sqrt().item()
     r = dense.float().pow(2).mean().sqrt().item()
+    assert d <= 2.0 ** -5 * r, f"rms diff {d / r:.3e}"
+
+
+def test_whole_model_agrees_with_dense_bf16():
+    """Input projections, time/guidance/pooled-text embedders, one double and
+    one single block, the final layer: [4096, 64] out, against the same model
+    with the blocks in dense bf16."""
+    cfg = workloads.FluxConfig(n_double=1, n_single=1)
+    model = flux.TernaryFlux(cfg, device="cuda")
+    io = {k: (W.cuda(), b.cuda()) for k, (W, b) in workloads.flux_io_weights(cfg).items()}
+    img, txt, pooled, t, g, ids = workloads.flux_model_inputs(cfg)
+    args = (img.cuda(), txt.cuda(), pooled.cuda(), t, g, ids.cuda())
+    out = flux.model_forward(model, io, *args)
+    ref = flux.dense_model_forward(model, flux.dense_weights(model), io, *args)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    assert out.shape == (cfg.img_tokens, cfg.in_channels) and torch.isfinite(out.float()).all()
+    d = (out.float() - ref.float()).pow(2).mean().sqrt().item()
+    r = ref.float().pow(2).mean().sqrt().item()
     assert d <= 2.0 ** -5 * r, f"rms diff {d / r:.3e}"
