@@ -651,7 +651,8 @@ def forward_rows(device, peaks, stream):
     embedding in the q/k epilogue), attention from torch; against the same
     model with the blocks in bf16 with dense weights (T*s) through cuBLAS and
     torch's unfused operations, the bf16 model of the pages' Table 3
-    comparison.  The two are timed in turns (CUDA events, medians of 3)."""
+    comparison.  The two are timed in turns (CUDA events, medians of 3),
+    launched from Python and replayed from CUDA graphs."""
     import statistics
 
     import torch
@@ -669,6 +670,23 @@ def forward_rows(device, peaks, stream):
     for f in runs.values():
         f()
     torch.cuda.synchronize()
+    # the same forwards replayed from CUDA graphs (no host launch gaps)
+    graphs = {}
+    side = torch.cuda.Stream(device)
+    for k, f in list(runs.items()):
+        side.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(side):
+            f()
+        torch.cuda.current_stream(device).wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        graphs[k] = g
+        runs[k + "_graph"] = g.replay
+    for k in ("ternary_graph", "dense_bf16_graph"):
+        runs[k]()
+    torch.cuda.synchronize()
     times = {k: [] for k in runs}
     for _ in range(3):
         for k, f in runs.items():
@@ -684,12 +702,14 @@ def forward_rows(device, peaks, stream):
     dense_b = sum(d[n][0].numel() * 2 for d in dense.values() for n in d if not n.endswith("norm_w"))
     io_b = sum(W.numel() * 2 for W, _ in io.values())
     t_ter, t_den = statistics.median(times["ternary"]), statistics.median(times["dense_bf16"])
-    del dense, model
+    tg_ter, tg_den = statistics.median(times["ternary_graph"]), statistics.median(times["dense_bf16_graph"])
+    del graphs, runs, dense, model
     torch.cuda.empty_cache()
     return {"flux_forward": {
         "model": f"{cfg.n_double} double + {cfg.n_single} single blocks, {cfg.img_tokens} image + "
                  f"{cfg.txt_tokens} text tokens, input layers, embedders and final layer",
         "ternary_ms": t_ter, "dense_bf16_ms": t_den, "speedup_vs_dense_bf16": t_den / t_ter,
+        "ternary_graph_ms": tg_ter, "dense_bf16_graph_ms": tg_den, "speedup_graph": tg_den / tg_ter,
         "linear_gflop": fl["linear"] / 1e9, "attention_gflop": fl["attention"] / 1e9,
         "ternary_tflops": (fl["linear"] + fl["attention"]) / (t_ter * 1e-3) / 1e12,
         "block_weight_gb_ternary": packed / 1e9, "block_weight_gb_bf16": dense_b / 1e9,
