@@ -341,12 +341,6 @@ def forward_flop(cfg: workloads.FluxConfig, n_double=None, n_single=None) -> Dic
     return {"linear": lin, "attention": att}
 
 
-def max_abs_rel(a: torch.Tensor, b: torch.Tensor) -> float:
-    """max |a - b| / rms(b) (diagnostic)."""
-    d = (a.float() - b.float()).abs().max().item()
-    return d / max(math.sqrt(b.float().pow(2).mean().item()), 1e-30)
-
-
 def dense_model_forward(model: TernaryFlux, dense: Dict, io: Dict, img_lat, txt_ctx, pooled, t: float,
                         guidance: float, ids, n_double=None, n_single=None) -> torch.Tensor:
     """model_forward with the blocks in dense bf16 (dense_forward) and the
