@@ -489,8 +489,21 @@ def side_table(device, peaks, stream):
             fused = [(lambda p=p, s=s: tern.linear_epilogue(x, p, s, b, norm_cols=(0, 2 * workloads.HIDDEN),
                                                             norm_weight=nw, norm_eps=1e-6, out=y))
                      for p, s in packs]
+            # and the rotary embedding of the image tokens' positions (0, row,
+            # column) on the 64 x 64 grid after the normalisation
+            from bit_post_quantised_b200 import flux
+            side = int(round(L.M ** 0.5))
+            ids = torch.zeros(L.M, 3, dtype=torch.float64)
+            ids[:, 1] = torch.arange(L.M, dtype=torch.float64) // side
+            ids[:, 2] = torch.arange(L.M, dtype=torch.float64) % side
+            cs = torch.stack(flux.rope_cos_sin(ids), dim=-1).contiguous().to(device)
+            roped = [(lambda p=p, s=s: tern.linear_epilogue(x, p, s, b, norm_cols=(0, 2 * workloads.HIDDEN),
+                                                            norm_weight=nw, norm_eps=1e-6, rope_cs=cs, out=y))
+                     for p, s in packs]
         if fused is None:
             t = graph_time(calls * reps, 5, stream)
+        elif name == "qkv":
+            t, tf, tr = interleaved_time([c * (reps // 2 or 1) for c in (calls, fused, roped)], 8, stream)
         else:
             t, tf = interleaved_time([calls * (reps // 2 or 1), fused * (reps // 2 or 1)], 8, stream)
         flop_t = 2.0 * L.M * L.N * L.K / peaks["bf16_tflops"] / 1e12
@@ -506,6 +519,7 @@ def side_table(device, peaks, stream):
         elif name == "qkv":
             # against the HBM time a separate pass over q and k would need
             entry["qk_norm_fused_us"] = tf * 1e6
+            entry["qk_norm_rope_fused_us"] = tr * 1e6
             entry["qk_norm_separate_pass_us_at_hbm_peak"] = (2 * 2 * L.M * 2 * workloads.HIDDEN / peaks["hbm_gbs"]
                                                               / 1e9 * 1e6)
         entry["cublas_bf16_us"] = cublas_context_us(L, packs, x, b, stream)
