@@ -633,31 +633,50 @@ __device__ __forceinline__ void tile_kernel_body(const Batch& batch) {
         if (!__all_sync(0xffffffffu, ok_n)) break;
         const int row0 = t.m_tile * C::kTokPair + half * kCols;
         const int rows = min(kCols, P.M - row0);
+        // Rotary (cos, sin) of this lane's channel pair, kRG token rows at a
+        // time: the rows come from L2, so a group's loads go out together.
+        // The two lanes of a pair split the rows (the even lane loads the
+        // even rows, the odd lane the odd ones) and swap them by shuffle.
+        constexpr int kRG = 8;
+        static_assert(kCols % kRG == 0, "rotary row groups");
+        const float2* rcs = reinterpret_cast<const float2*>(P.rope);
+        const int pair = (n & 127) >> 1;
+        float2 cs[kRG / 2];  // rows c0 + 2i + (lane & 1)
+        auto load_cs = [&](int c0) {
+#pragma unroll
+          for (int i = 0; i < kRG / 2; ++i) {
+            const int m = row0 + c0 + 2 * i + (lane & 1);
+            cs[i] = m < P.M ? __ldg(rcs + size_t(m) * 64 + pair) : make_float2(1.f, 0.f);
+          }
+        };
         // Rotary embedding (the same for the whole problem): channel pair
         // (2p, 2p + 1) of the group turns by the angle of pair p of its row;
         // the partner channel is the neighbouring lane.  Even channel:
         // a cos - b sin, odd: a cos + b sin (b the partner's value).
-        const float2* rcs = reinterpret_cast<const float2*>(P.rope);
-        const int pair = (n & 127) >> 1;
         const float sgn = (n & 1) ? 1.f : -1.f;
-#pragma unroll
-        for (int j = 0; j < kCols / 2; ++j) {
-          const float lo = __uint_as_float(out[j] << 16), hi = __uint_as_float(out[j] & 0xFFFF0000u);
-          float a0 = lo * (norm_inv[half * kCols + 2 * j] * w), a1 = hi * (norm_inv[half * kCols + 2 * j + 1] * w);
-          if (rcs) {
-            const float b0 = __shfl_xor_sync(0xffffffffu, a0, 1), b1 = __shfl_xor_sync(0xffffffffu, a1, 1);
-            const int m0 = row0 + 2 * j;
-            const float2 c0 = m0 < P.M ? __ldg(rcs + size_t(m0) * 64 + pair) : make_float2(1.f, 0.f);
-            const float2 c1 = m0 + 1 < P.M ? __ldg(rcs + size_t(m0 + 1) * 64 + pair) : make_float2(1.f, 0.f);
-            a0 = fmaf(a0, c0.x, sgn * b0 * c0.y);
-            a1 = fmaf(a1, c1.x, sgn * b1 * c1.y);
-          }
-          out[j] = pack_bf16x2(a0, a1);
-        }
         uint16_t* yp = reinterpret_cast<uint16_t*>(P.y) + size_t(row0) * P.ldy + n;
 #pragma unroll
-        for (int c = 0; c < kCols; ++c)
-          if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+        for (int g = 0; g < kCols; g += kRG) {
+          if (rcs) load_cs(g);
+#pragma unroll
+          for (int j = g / 2; j < (g + kRG) / 2; ++j) {
+            const float lo = __uint_as_float(out[j] << 16), hi = __uint_as_float(out[j] & 0xFFFF0000u);
+            float a0 = lo * (norm_inv[half * kCols + 2 * j] * w), a1 = hi * (norm_inv[half * kCols + 2 * j + 1] * w);
+            if (rcs) {
+              const float b0 = __shfl_xor_sync(0xffffffffu, a0, 1), b1 = __shfl_xor_sync(0xffffffffu, a1, 1);
+              const float2 mine = cs[j - g / 2];  // row 2j + (lane & 1)
+              const float2 other = make_float2(__shfl_xor_sync(0xffffffffu, mine.x, 1),
+                                               __shfl_xor_sync(0xffffffffu, mine.y, 1));
+              const float2 c0 = (lane & 1) ? other : mine, c1 = (lane & 1) ? mine : other;
+              a0 = fmaf(a0, c0.x, sgn * b0 * c0.y);
+              a1 = fmaf(a1, c1.x, sgn * b1 * c1.y);
+            }
+            out[j] = pack_bf16x2(a0, a1);
+          }
+#pragma unroll
+          for (int c = g; c < g + kRG; ++c)
+            if (c < rows) yp[size_t(c) * P.ldy] = uint16_t(out[c >> 1] >> ((c & 1) * 16));
+        }
       } else if (EPI == 3 && n - r >= P.norm_col0 && n - r < P.norm_col1) {
         // RMS normalisation combined with an activation, a residual or a
         // gate on the same channels: fp32 throughout with one rounding.  The
