@@ -28,6 +28,7 @@ the bf16 model that the pages compare against, for latency context.
 """
 from __future__ import annotations
 
+import contextlib
 import math
 from typing import Dict, Optional
 
@@ -79,6 +80,17 @@ def attention(qkv: torch.Tensor, hidden: int, cos=None, sin=None) -> torch.Tenso
     return o[0]
 
 
+def _on(stream):
+    """Makes `stream` current (when given), after the work already queued on
+    the current stream (the caller's inputs), so that the torch operations
+    between the library calls run on the stream those calls are given.  The
+    results are then ready on `stream`."""
+    if stream is None:
+        return contextlib.nullcontext()
+    stream.wait_stream(torch.cuda.current_stream(stream.device))
+    return torch.cuda.stream(stream)
+
+
 def _qk_norm_weight(q_norm: torch.Tensor, k_norm: torch.Tensor, hidden: int, N: int) -> torch.Tensor:
     """[N] bf16 epilogue weight: the per-head q and k norm weights over
     columns [0, 2C), 1 elsewhere (unused there)."""
@@ -95,13 +107,21 @@ class TernaryFlux:
     ``weights`` maps ("double" | "single", index) to the bf16 parameters of
     ``workloads.flux_block_weights``; every linear is quantised with
     ``tern.quantize_pack`` at construction (eps = workloads.EPS) and only the
-    codes, scales and biases are kept."""
+    codes, scales and biases are kept.  With ``stream`` given, construction
+    and every forward run on it, the torch operations included, after the
+    work queued before the call on the current stream; results are ready on
+    ``stream``."""
 
     def __init__(self, cfg: workloads.FluxConfig, weights: Optional[Dict] = None, device="cuda", stream=None):
         self.cfg = cfg
         self.device = torch.device(device)
         self.stream = stream
         self.blocks = {}
+        with _on(stream):
+            self._quantize(weights)
+
+    def _quantize(self, weights):
+        cfg, stream = self.cfg, self.stream
         C, Fm = cfg.hidden, cfg.mlp
         for kind, n in (("double", cfg.n_double), ("single", cfg.n_single)):
             for i in range(n):
@@ -198,6 +218,10 @@ class TernaryFlux:
         device), token positions ids [Lt + Li, 3]; returns the stream
         [Lt + Li, C] after the last single block (text rows first).  The
         inputs are not modified."""
+        with _on(self.stream):
+            return self._forward(img, txt, vec, ids, n_double, n_single)
+
+    def _forward(self, img, txt, vec, ids, n_double, n_single):
         cfg = self.cfg
         nd = cfg.n_double if n_double is None else n_double
         ns = cfg.n_single if n_single is None else n_single
@@ -248,12 +272,13 @@ def model_forward(model: "TernaryFlux", io: Dict, img_lat, txt_ctx, pooled, t: f
     library, and the final layer (adaLN modulation row from SiLU(vec) in
     bf16, layer norm and modulation of the image tokens by the library's
     adaLN pass, the bf16 output projection).  Returns [Li, in_channels]."""
-    img, txt, vec = io_layers_in(io, img_lat, txt_ctx, pooled, t, guidance)
-    x = model.forward(img, txt, vec, ids, n_double, n_single)
-    C = model.cfg.hidden
-    mod = F.linear(F.silu(vec), *io["final.mod"])  # [shift | scale]
-    h = tern.adaln_modulate(x[txt.shape[0]:], mod[:, C:], mod[:, :C], LN_EPS, stream=model.stream)
-    return F.linear(h, *io["final.out"])
+    with _on(model.stream):
+        img, txt, vec = io_layers_in(io, img_lat, txt_ctx, pooled, t, guidance)
+        x = model.forward(img, txt, vec, ids, n_double, n_single)
+        C = model.cfg.hidden
+        mod = F.linear(F.silu(vec), *io["final.mod"])  # [shift | scale]
+        h = tern.adaln_modulate(x[txt.shape[0]:], mod[:, C:], mod[:, :C], LN_EPS, stream=model.stream)
+        return F.linear(h, *io["final.out"])
 
 
 def dense_weights(model: TernaryFlux) -> Dict:

@@ -89,6 +89,20 @@ def test_double_then_single_block_matches_oracle(small):
     check(out, ref)
 
 
+def test_forward_on_a_side_stream_matches(small):
+    """A model given its own stream (construction and forward on it, torch
+    operations included) gives the same bits as on the current stream."""
+    cfg, weights, model, (img, txt, vec, ids), _ = small
+    ref = model.forward(img, txt, vec, ids)
+    s = torch.cuda.Stream()
+    side = flux.TernaryFlux(cfg, weights, device="cuda", stream=s)
+    out = side.forward(img, txt, vec, ids)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    assert torch.equal(out, ref)
+
+
 def test_full_size_blocks_agree_with_dense_bf16():
     cfg = workloads.FluxConfig(n_double=1, n_single=1)
     model = flux.TernaryFlux(cfg, device="cuda")
