@@ -137,6 +137,15 @@ def _stream(stream: Optional[torch.cuda.Stream]):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _empty(*shape, dtype, device, stream=None) -> torch.Tensor:
+    """An output buffer allocated on the stream the call launches on, so that
+    the caching allocator orders its reuse after that stream's work."""
+    if stream is None:
+        return torch.empty(*shape, dtype=dtype, device=device)
+    with torch.cuda.stream(stream):
+        return torch.empty(*shape, dtype=dtype, device=device)
+
+
 def packed_bytes(N: int, K: int) -> int:
     return int(lib().tern_packed_bytes(N, K))
 
@@ -146,9 +155,9 @@ def quantize_pack(W: torch.Tensor, eps: float = 1e-5, packed: Optional[torch.Ten
     """tern_quantize_pack: W bf16 [N,K] -> (packed uint8 [N*K/4], scales fp32 [N])."""
     N, K = W.shape
     if packed is None:
-        packed = torch.empty(max(packed_bytes(N, K), 1), dtype=torch.uint8, device=W.device)
+        packed = _empty(max(packed_bytes(N, K), 1), dtype=torch.uint8, device=W.device, stream=stream)
     if scales is None:
-        scales = torch.empty(N, dtype=torch.float32, device=W.device)
+        scales = _empty(N, dtype=torch.float32, device=W.device, stream=stream)
     _check(lib().tern_quantize_pack(_ptr(W), N, K, float(eps), _ptr(packed), _ptr(scales),
                                     _stream(stream)))
     return packed, scales
@@ -176,7 +185,7 @@ def adaln_modulate(x: torch.Tensor, scale: torch.Tensor, shift: torch.Tensor, ep
             raise ValueError(f"{name} holds fewer than the {G} modulation rows of {K} values that "
                              f"{M} rows at {T} tokens per row need")
     if out is None:
-        out = torch.empty_like(x)
+        out = _empty(*x.shape, dtype=x.dtype, device=x.device, stream=stream)
     _check(lib().tern_adaln_modulate(_ptr(x), M, K, _ptr(scale), _ptr(shift), int(mod_ld), max(T, 1), float(eps),
                                      _ptr(out), _stream(stream)))
     return out
@@ -197,7 +206,7 @@ def linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        out = _empty(M, N, dtype=torch.bfloat16, device=x.device, stream=stream)
     _dense(x, out)
     _check(lib().tern_linear(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
                              _stream(stream)))
@@ -213,7 +222,7 @@ def linear_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        out = _empty(M, N, dtype=torch.bfloat16, device=x.device, stream=stream)
     _dense(x, out)
     _check(lib().tern_linear_noalloc(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N,
                                      _ptr(out), _stream(stream)))
@@ -241,7 +250,7 @@ def linear_act(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        out = _empty(M, N, dtype=torch.bfloat16, device=x.device, stream=stream)
     _dense(x, out)
     _check(lib().tern_linear_act(_ptr(x), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, act, act_col0,
                                  _ptr(out), _stream(stream)))
@@ -295,7 +304,7 @@ def linear_epilogue(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     M, K = x.shape
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        out = _empty(M, N, dtype=torch.bfloat16, device=x.device, stream=stream)
     a = _linear_args(dict(x=x, packed=packed, scales=scales, bias=bias, y=out))
     e = _epilogue(dict(act=act, act_col0=act_col0, residual=residual, gate=gate, norm_col0=norm_cols[0],
                        norm_col1=norm_cols[1], norm_weight=norm_weight, norm_eps=norm_eps, rope_cs=rope_cs, y=out))
@@ -321,9 +330,9 @@ def quantize_act_e4m3(x: torch.Tensor, xq: Optional[torch.Tensor] = None, a: Opt
     interleaved k order of include/tern.h, a fp32 [M] per-token scales)."""
     M, K = x.shape
     if xq is None:
-        xq = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+        xq = _empty(M, K, dtype=torch.uint8, device=x.device, stream=stream)
     if a is None:
-        a = torch.empty(M, dtype=torch.float32, device=x.device)
+        a = _empty(M, dtype=torch.float32, device=x.device, stream=stream)
     _check(lib().tern_quantize_act_e4m3(_ptr(x), M, K, _ptr(xq), _ptr(a), _stream(stream)))
     return xq, a
 
@@ -334,7 +343,7 @@ def linear_e4m3(xq: torch.Tensor, a: torch.Tensor, packed: torch.Tensor, scales:
     M, K = xq.shape
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+        out = _empty(M, N, dtype=torch.bfloat16, device=xq.device, stream=stream)
     _check(lib().tern_linear_e4m3(_ptr(xq), _ptr(a), M, K, _ptr(packed), _ptr(scales), _ptr(bias), N, _ptr(out),
                                   _stream(stream)))
     return out
@@ -380,7 +389,7 @@ def dequantize(packed: torch.Tensor, scales: torch.Tensor, K: int, out: Optional
     """tern_dequantize: codes -> bf16 [N,K] with W'[n,k] = T[n,k] * s_n."""
     N = scales.shape[0]
     if out is None:
-        out = torch.empty(N, K, dtype=torch.bfloat16, device=scales.device)
+        out = _empty(N, K, dtype=torch.bfloat16, device=scales.device, stream=stream)
     _check(lib().tern_dequantize(_ptr(packed), _ptr(scales), N, K, _ptr(out), _stream(stream)))
     return out
 
