@@ -1,7 +1,8 @@
 """Host-side pieces of the FLUX.1 forward (bit_post_quantised_b200.flux) on
 the CPU, against the fp64 block oracle's own forms: the rotary angles' cos /
 sin table the q/k epilogue reads, torch's rotary embedding of the dense
-path, the sinusoidal timestep embedding, and the token positions."""
+path, the sinusoidal timestep embedding, the token positions, and the
+dense-bf16 twin of the blocks as a whole."""
 from __future__ import annotations
 
 import math
@@ -57,3 +58,50 @@ def test_token_positions():
     img = ids[cfg.txt_tokens:]
     assert torch.equal(img[:, 0], torch.zeros(cfg.img_tokens))
     assert torch.equal(img[cfg.img_w + 3], torch.tensor([0.0, 1.0, 3.0]))  # row 1, column 3
+
+
+def test_dense_twin_matches_the_block_oracle():
+    """flux.dense_forward (the bf16 model with dense weights that the forward
+    is timed against) on the CPU, one double and one single block of the
+    small config, with weights bf16(T * s) from the oracle's quantisation,
+    against the fp64 block oracle on the same T and s.  The scales are taken
+    8x larger than the seeded weights give, so that the blocks' updates
+    outweigh the residual streams they are added to (with the seeded scales
+    the gates keep them near 1 % of the stream, below what the bf16 stream
+    resolves).  The dense twin rounds to bf16 after each unfused torch
+    operation and its weights carry one more rounding: rms 2^-6 of the
+    output; a missing q/k norm weight, swapped position axes or a dropped
+    projection each exceed it."""
+    import types
+
+    import oracle
+
+    cfg = workloads.FLUX_SMALL
+    C = cfg.hidden
+    dense, params = {}, {}
+    for kind in ("double", "single"):
+        w = workloads.flux_block_weights(cfg, kind, 0)
+        d, p = {}, {}
+        for name, N, K in workloads.flux_block_shapes(cfg, kind):
+            W, b = w[name]
+            T, s = oracle.quantize(workloads.bf16_bits(W), workloads.EPS)
+            s = 8.0 * s
+            d[name] = (torch.from_numpy(T * s[:, None]).to(torch.bfloat16), b)
+            p[name] = (T, s, workloads.bf16_bits(b))
+        for st in (("img.", "txt.") if kind == "double" else ("",)):
+            N = 3 * C if kind == "double" else 3 * C + cfg.mlp
+            d[st + "norm_w"] = flux._qk_norm_weight(w[st + "q_norm"], w[st + "k_norm"], C, N)
+            p[st + "q_norm"] = workloads.bf16_bits(w[st + "q_norm"])
+            p[st + "k_norm"] = workloads.bf16_bits(w[st + "k_norm"])
+        dense[(kind, 0)], params[kind] = d, p
+    img, txt, vec, ids = workloads.flux_inputs(cfg)
+    out = flux.dense_forward(types.SimpleNamespace(cfg=cfg), dense, img, txt, vec, ids, 1, 1)
+    f = lambda t: OF.from_bits(workloads.bf16_bits(t))  # noqa: E731
+    ang = OF.rope_angles(ids.numpy())
+    oi, ot = OF.double_block(f(img), f(txt), f(vec), params["double"], ang)
+    ref = OF.single_block(np.concatenate([ot, oi]), f(vec), params["single"], ang)
+    x0 = np.concatenate([f(txt), f(img)])
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    assert float(np.sqrt(np.mean((ref - x0) ** 2))) > 0.5 * rms  # the update dominates
+    assert out.shape == (cfg.txt_tokens + cfg.img_tokens, C)
+    assert float(np.sqrt(np.mean((out.double().numpy() - ref) ** 2))) <= 2.0 ** -6 * rms
