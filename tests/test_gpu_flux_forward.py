@@ -69,6 +69,40 @@ def small():
     return cfg, weights, model, (img.cuda(), txt.cuda(), vec.cuda(), ids), ref_in
 
 
+@pytest.fixture(scope="module")
+def small_strong():
+    """The small config with every ternary weight 8x larger (exact in bf16,
+    the same codes, 8x the scales): the blocks' updates then outweigh the
+    residual streams, so a wrong update cannot hide under the streams' bf16
+    rounding (with the seeded weights the gates keep the updates near 1 % of
+    the stream)."""
+    cfg = workloads.FLUX_SMALL
+    weights = {}
+    for k in ("double", "single"):
+        w = workloads.flux_block_weights(cfg, k, 0)
+        for name, _, _ in workloads.flux_block_shapes(cfg, k):
+            W, b = w[name]
+            w[name] = (W * 8, b)
+        weights[(k, 0)] = w
+    model = flux.TernaryFlux(cfg, weights, device="cuda")
+    img, txt, vec, ids = workloads.flux_inputs(cfg)
+    f = lambda t: OF.from_bits(workloads.bf16_bits(t))  # noqa: E731
+    ref_in = (f(img), f(txt), f(vec), OF.rope_angles(ids.numpy()))
+    return cfg, weights, model, (img.cuda(), txt.cuda(), vec.cuda(), ids), ref_in
+
+
+def test_blocks_with_dominant_updates_match_oracle(small_strong):
+    cfg, weights, model, (img, txt, vec, ids), (i64, t64, v64, ang) = small_strong
+    out = model.forward(img, txt, vec, ids)
+    torch.cuda.synchronize()
+    assert tern.device_status() == 0
+    oi, ot = OF.double_block(i64, t64, v64, oracle_params(model, weights, cfg, "double"), ang)
+    ref = OF.single_block(np.concatenate([ot, oi]), v64, oracle_params(model, weights, cfg, "single"), ang)
+    x0 = np.concatenate([t64, i64])
+    assert np.sqrt(np.mean((ref - x0) ** 2)) > 0.5 * np.sqrt(np.mean(ref ** 2))  # the update dominates
+    check(out, ref)
+
+
 def test_double_block_matches_oracle(small):
     cfg, weights, model, (img, txt, vec, ids), (i64, t64, v64, ang) = small
     out = model.forward(img, txt, vec, ids, n_double=1, n_single=0)
