@@ -360,3 +360,39 @@ def test_adaln_binding_checks_modulation_rows(T, rows):
     mod = torch.zeros(rows, 6 * K, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="modulation rows"):
         tern.adaln_modulate(x, mod[:, K:2 * K], mod[:, :K], 1e-6, tokens_per_row=T)
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "tern.h"
+
+int main(void) {
+  /* host-only calls: no device memory is touched */
+  size_t bytes = tern_packed_bytes(9216, 3072);
+  uintptr_t f = (uintptr_t)0x7F0000000000ull;  /* never dereferenced */
+  tern_status s = tern_linear((const void*)f, 16, 100, (const void*)(f + 0x100000),
+                              (const float*)(f + 0x200000), NULL, 256, (void*)(f + 0x300000), NULL);
+  printf("%zu %d %s|%s\n", bytes, (int)s, tern_status_string(s), tern_last_error());
+  return (bytes == (size_t)9216 * 3072 / 4 && s == TERN_ERR_UNSUPPORTED_SHAPE) ? 0 : 1;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(tmp_path, L):
+    """A plain C99 client of include/tern.h, built with gcc against libtern.so
+    (no CUDA headers, no C++): the boundary is usable from C.  It calls only
+    host-side paths (the packed size and a shape the library refuses before
+    any CUDA call)."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(tern.library_path())
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                           os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-ltern",
+                           f"-Wl,-rpath,{libdir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    bytes_, status, rest = out.stdout.split(" ", 2)
+    assert int(bytes_) == 9216 * 3072 // 4 and int(status) == -2
+    assert "K" in rest.split("|", 1)[1]  # the message names the failing dimension
