@@ -105,3 +105,21 @@ def test_dense_twin_matches_the_block_oracle():
     assert float(np.sqrt(np.mean((ref - x0) ** 2))) > 0.5 * rms  # the update dominates
     assert out.shape == (cfg.txt_tokens + cfg.img_tokens, C)
     assert float(np.sqrt(np.mean((out.double().numpy() - ref) ** 2))) <= 2.0 ** -6 * rms
+
+
+def test_parameter_count_matches_the_pages():
+    """The synthetic transformer's parameters (ternary block linears, their
+    biases and q/k norm weights, and the bf16 input/output layers and
+    embedders) add up to the 11.9B the pages give for FLUX.1-dev, and the
+    ternary weights to the 99.5 % they quantise ("1.58-bit FLUX", Abstract
+    and Section 1): a check of every layer shape of the forward."""
+    cfg = workloads.FluxConfig()
+    blocks = [s for kind, n in (("double", cfg.n_double), ("single", cfg.n_single))
+              for _ in range(n) for s in workloads.flux_block_shapes(cfg, kind)]
+    ternary = sum(N * K for _, N, K in blocks)
+    biases = sum(N for _, N, _ in blocks)
+    norms = (4 * cfg.n_double + 2 * cfg.n_single) * workloads.HEAD_DIM
+    io = sum(W.numel() + b.numel() for W, b in workloads.flux_io_weights(cfg).values())
+    total = ternary + biases + norms + io
+    assert abs(total / 1e9 - 11.9) < 0.05
+    assert abs(ternary / total - 0.995) < 2e-3
